@@ -1,0 +1,160 @@
+/*
+ * swiglu.h -- C ABI of the B200 (sm_100a) fused SwiGLU gate/up projection
+ * library (libswiglu_b200.so).
+ *
+ * Operation (forward):
+ *     G = X * Wg^T,  U = X * Wu^T,  H = silu(G) (.) U,  silu(x) = x*sigmoid(x)
+ * computed as ONE fused op: both projections share one read of X and the
+ * SiLU-and-gate step runs on the fp32 accumulators in the epilogue, so G and
+ * U never reach global memory.  This is the "dual gemm with activations" of
+ * Liger-Kernel issue #937 ("Another MLP implementation along with multiplier
+ * support", approach 3), i.e. the "gate/up GEMM + SwiGLU in a single kernel"
+ * of Liger-Kernel issue #1383 ("[RFC] Testing Methodology for FP32
+ * Convergence Tests on Fused SwiGLU/dSwiGLU Kernels", Background).
+ *
+ * Operation (backward, elementwise "dSwiGLU", issue #1383 title/Background):
+ *     dU = dH (.) silu(G),   dG = dH (.) U (.) silu'(G),
+ *     silu'(x) = sigmoid(x) * (1 + x*(1 - sigmoid(x))).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers to caller-owned memory on the
+ *    current CUDA device, row-major and contiguous.  The library keeps no
+ *    reference to them after the call returns.  Work is enqueued on `stream`
+ *    (0 = legacy default stream) and runs asynchronously.
+ *  - Layouts follow nn.Linear (TensorRT-LLM PR #17693 passes weight.t() to
+ *    addmm and flattens rank>=3 activations to [M, in]):
+ *        X [M, K], Wg [N, K], Wu [N, K], H [M, N].
+ *  - Return value: SWIGLU_OK (0) or one of the SWIGLU_ERR_* codes below.
+ *    Argument errors are detected on the host before anything is enqueued.
+ *    A device-side wait that gave up (a bounded wait; kernels never spin
+ *    forever) is reported later by swiglu_sync_status().
+ *  - There is no CPU fallback and no environment-driven dispatch: routing is
+ *    a pure function of (M, K, dtype), see swiglu_route_for().
+ */
+#ifndef SWIGLU_B200_H
+#define SWIGLU_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same definition as the CUDA runtime's (driver_types.h); repeating an
+ * identical typedef is legal in C11 and C++. */
+typedef struct CUstream_st *cudaStream_t;
+
+#if defined(_WIN32)
+#define SWIGLU_API __declspec(dllexport)
+#else
+#define SWIGLU_API __attribute__((visibility("default")))
+#endif
+
+/* Element types. */
+enum swiglu_dtype {
+    SWIGLU_BF16 = 0, /* bf16 in/out, fp32 accumulate, bf16 RNE output       */
+    SWIGLU_FP32 = 1  /* fp32 in/out, near-IEEE via 3xTF32 on tensor cores  */
+};
+
+/* Status codes. */
+enum swiglu_status {
+    SWIGLU_OK = 0,
+    SWIGLU_ERR_NULL_POINTER = 1,     /* a required pointer is NULL          */
+    SWIGLU_ERR_BAD_DIM = 2,          /* a size is negative or too large     */
+    SWIGLU_ERR_MISALIGNED_DIM = 3,   /* K or N not a multiple of 8 (bf16) or
+                                        4 (fp32): rows must be 16-B strided */
+    SWIGLU_ERR_MISALIGNED_PTR = 4,   /* a pointer is not 16-byte aligned    */
+    SWIGLU_ERR_BAD_DTYPE = 5,        /* dtype is not a swiglu_dtype         */
+    SWIGLU_ERR_UNSUPPORTED_DEVICE = 6, /* current device is not sm_100      */
+    SWIGLU_ERR_CUDA = 7,             /* a CUDA runtime/driver call failed   */
+    SWIGLU_ERR_TIMEOUT = 8,          /* a device-side bounded wait gave up  */
+    SWIGLU_ERR_OVERLAP = 9,          /* an output overlaps an input         */
+    SWIGLU_ERR_NO_DEVICE = 10        /* no CUDA device is usable            */
+};
+
+/* Kernel routes (which kernel a swiglu_fwd call enqueues). */
+enum swiglu_route {
+    SWIGLU_ROUTE_NONE = 0,        /* empty problem: nothing enqueued        */
+    SWIGLU_ROUTE_ZERO_K = 1,      /* K == 0: H is filled with zeros         */
+    SWIGLU_ROUTE_DECODE_BF16 = 2, /* bf16, M <= 8: weight-streaming kernel  */
+    SWIGLU_ROUTE_GEMM_BF16 = 3,   /* bf16, M > 8: tcgen05 dual GEMM         */
+    SWIGLU_ROUTE_GEMM_TF32X3 = 4  /* fp32: 3xTF32 tcgen05 dual GEMM         */
+};
+
+/*
+ * swiglu_fwd -- H = silu(X Wg^T) (.) (X Wu^T).
+ *
+ *  X   [M, K] device, dtype elements, 16-byte aligned.
+ *  Wg  [N, K] device, dtype elements, 16-byte aligned (gate_proj.weight).
+ *  Wu  [N, K] device, dtype elements, 16-byte aligned (up_proj.weight).
+ *  H   [M, N] device, dtype elements, 16-byte aligned; written, never read.
+ *  M, K, N >= 0.  K and N multiples of 8 (bf16) / 4 (fp32).
+ *  dtype  SWIGLU_BF16 or SWIGLU_FP32.
+ *
+ *  M == 0 or N == 0: returns SWIGLU_OK, enqueues nothing (pointers unchecked).
+ *  K == 0: H is set to +0.
+ *  H must not overlap X, Wg or Wu (SWIGLU_ERR_OVERLAP).  X, Wg, Wu may alias.
+ *  bf16: accumulation in fp32, SiLU and product in fp32 on the accumulators,
+ *  one round-to-nearest-even to bf16; NaN/Inf propagate (no saturation).
+ *  fp32: each operand is split a = hi + lo (hi, lo TF32), and the three
+ *  products hi*hi + hi*lo + lo*hi are accumulated in fp32 on tensor cores.
+ *  No call allocates device memory.
+ */
+SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu,
+                          void *H, int64_t M, int64_t K, int64_t N, int dtype,
+                          cudaStream_t stream);
+
+/*
+ * dswiglu_bwd -- elementwise dSwiGLU, bf16.
+ *
+ *  dH, G, U  [n] device bf16 inputs, 16-byte aligned.
+ *  dG, dU    [n] device bf16 outputs, 16-byte aligned.
+ *  n >= 0 (n == 0: no-op).  Math in fp32, one RNE rounding per output.
+ *  dG may be exactly G (in place) and dU exactly U; any other overlap of an
+ *  output with an input, or of dG with dU, is SWIGLU_ERR_OVERLAP.
+ */
+SWIGLU_API int dswiglu_bwd(const void *dH, const void *G, const void *U,
+                           void *dG, void *dU, int64_t n, cudaStream_t stream);
+
+/* dswiglu_bwd with an explicit dtype (SWIGLU_BF16 or SWIGLU_FP32). */
+SWIGLU_API int dswiglu_bwd_dtype(const void *dH, const void *G, const void *U,
+                                 void *dG, void *dU, int64_t n, int dtype,
+                                 cudaStream_t stream);
+
+/* Route swiglu_fwd takes for these arguments (pure host function; returns a
+ * swiglu_route, or -1 for arguments swiglu_fwd would reject). */
+SWIGLU_API int swiglu_route_for(int64_t M, int64_t K, int64_t N, int dtype);
+
+/* Route of the last swiglu_fwd call on this host thread that returned
+ * SWIGLU_OK (SWIGLU_ROUTE_NONE before the first).  Lets tests assert that
+ * the fused kernel actually ran. */
+SWIGLU_API int swiglu_last_route(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SWIGLU_API const char *swiglu_status_string(int status);
+
+/*
+ * Wait for `stream`, then read and clear the device status words of the
+ * current device.  Returns SWIGLU_ERR_TIMEOUT if any kernel's bounded wait
+ * gave up since the last call, SWIGLU_ERR_CUDA if the stream reports an
+ * error, else SWIGLU_OK.
+ */
+SWIGLU_API int swiglu_sync_status(cudaStream_t stream);
+
+/*
+ * Bench-only probe: stream-read `bytes` bytes from each of A and B (device,
+ * 16-byte aligned, bytes a multiple of 16) with the same 128-bit loads the
+ * decode kernel uses, and write one 32-bit word per CTA to `sink`
+ * (device, at least swiglu_read_floor_sink_words() words).  Measures the
+ * practical cold-read floor the decode kernel is compared with (AstrAI
+ * swiglu_benchmark.md, "HBM re-measurement and kernel simplification").
+ */
+SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes,
+                                 void *sink, cudaStream_t stream);
+SWIGLU_API int64_t swiglu_read_floor_sink_words(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWIGLU_B200_H */

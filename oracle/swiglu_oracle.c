@@ -1,0 +1,282 @@
+/*
+ * swiglu_oracle.c -- plain fp64 CPU oracle for the fused SwiGLU gate/up
+ * projection and its elementwise dSwiGLU backward.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library.  It shares no
+ * code, header, table or helper with the CUDA library it checks.
+ *
+ * What it computes (all arithmetic in IEEE double, no fast-math):
+ *
+ *   G[m,n] = sum_k X[m,k] * Wg[n,k]      (ascending k)
+ *   U[m,n] = sum_k X[m,k] * Wu[n,k]      (ascending k)
+ *   H[m,n] = silu(G[m,n]) * U[m,n],  silu(x) = x * sigmoid(x)
+ *
+ * Sources:
+ *  - The operation is the "dual gemm with activations" of Liger-Kernel issue
+ *    #937 ("Another MLP implementation along with multiplier support",
+ *    approach 3): one op takes x, gate_proj.weight and up_proj.weight and
+ *    returns act(x Wg^T) * (x Wu^T).  The weights are nn.Linear weights,
+ *    stored [out, in] = [N, K] row-major (same issue, the MLP code quoted in
+ *    the TL;DR; and TensorRT-LLM PR #17693, which passes weight.t() to addmm).
+ *  - The activation on the gate is SiLU, as in LigerSiLUMulFunction(gate,
+ *    up) quoted in the TL;DR of issue #937, and the backward is the
+ *    "dSwiGLU" named in the title and Background of Liger-Kernel issue #1383.
+ *  - Inputs are [M, in] after flattening, per TensorRT-LLM PR #17693
+ *    (description of _fused_up_proj_gelu).
+ *  - The fused epilogue applies the activation to the un-rounded accumulator
+ *    (TensorRT-LLM PR #17693, the numerics note of the follow-up commit that
+ *    gates the GELU epilogue): the oracle therefore keeps G and U in double
+ *    and never rounds them before the activation.
+ *
+ * The pages never write the SiLU or its derivative out; the oracle uses the
+ * textbook definitions: sigmoid(x) = 1/(1+exp(-x)), silu(x) = x*sigmoid(x),
+ * silu'(x) = sigmoid(x) * (1 + x*(1 - sigmoid(x))).
+ *
+ * bf16 inputs arrive as their 16-bit patterns and are decoded here by a bit
+ * shift into the top half of an IEEE float (exact), then widened to double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_API __attribute__((visibility("default")))
+
+/* ---- scalar definitions ------------------------------------------------ */
+
+ORACLE_API double oracle_sigmoid(double x)
+{
+    /* Two algebraically equal forms; the branch only avoids exp overflow. */
+    if (x >= 0.0) {
+        return 1.0 / (1.0 + exp(-x));
+    } else {
+        double e = exp(x);
+        return e / (1.0 + e);
+    }
+}
+
+ORACLE_API double oracle_silu(double x)
+{
+    return x * oracle_sigmoid(x);
+}
+
+ORACLE_API double oracle_dsilu(double x)
+{
+    double s = oracle_sigmoid(x);
+    return s * (1.0 + x * (1.0 - s));
+}
+
+/* ---- input decoding ---------------------------------------------------- */
+
+static double bf16_bits_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+ORACLE_API void oracle_bf16_to_f64(const uint16_t *src, double *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = bf16_bits_to_double(src[i]);
+}
+
+ORACLE_API void oracle_f32_to_f64(const float *src, double *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = (double)src[i];
+}
+
+/* ---- forward on decoded (double) operands ------------------------------ */
+
+/*
+ * One output element: the two dot products over k in ascending order, then
+ * the gate activation and the product.  Also returns the magnitude sums
+ * sum_k |x*wg| and sum_k |x*wu| that bound the rounding error of any
+ * summation order (used by the fp32-mode tolerance).
+ */
+static void one_output(const double *x, const double *wg, const double *wu,
+                       int64_t K, double *g_out, double *u_out, double *h_out,
+                       double *ag_out, double *au_out)
+{
+    double g = 0.0, u = 0.0, ag = 0.0, au = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double pg = x[k] * wg[k];
+        double pu = x[k] * wu[k];
+        g += pg;
+        u += pu;
+        ag += fabs(pg);
+        au += fabs(pu);
+    }
+    if (g_out) *g_out = g;
+    if (u_out) *u_out = u;
+    if (h_out) *h_out = oracle_silu(g) * u;
+    if (ag_out) *ag_out = ag;
+    if (au_out) *au_out = au;
+}
+
+/*
+ * Full forward.  X [M,K], Wg/Wu [N,K], outputs [M,N]; any output pointer may
+ * be NULL.  Rows of the output are independent, so they are spread over
+ * OpenMP threads; each element's sum order does not depend on the thread
+ * count.
+ */
+ORACLE_API void oracle_swiglu_fwd_f64(const double *X, const double *Wg,
+                                      const double *Wu, int64_t M, int64_t K,
+                                      int64_t N, double *G, double *U,
+                                      double *H, double *AG, double *AU)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t o = m * N + n;
+            one_output(X + m * K, Wg + n * K, Wu + n * K, K,
+                       G ? G + o : 0, U ? U + o : 0, H ? H + o : 0,
+                       AG ? AG + o : 0, AU ? AU + o : 0);
+        }
+    }
+}
+
+/*
+ * Sampled forward: only the outputs (idx_m[i], idx_n[i]) for i < count.
+ * Used to check full-size launches element by element without computing all
+ * M*N outputs.
+ */
+ORACLE_API void oracle_swiglu_fwd_points_f64(const double *X, const double *Wg,
+                                             const double *Wu, int64_t K,
+                                             const int64_t *idx_m,
+                                             const int64_t *idx_n,
+                                             int64_t count, double *G,
+                                             double *U, double *H, double *AG,
+                                             double *AU)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        one_output(X + idx_m[i] * K, Wg + idx_n[i] * K, Wu + idx_n[i] * K, K,
+                   G ? G + i : 0, U ? U + i : 0, H ? H + i : 0,
+                   AG ? AG + i : 0, AU ? AU + i : 0);
+    }
+}
+
+/*
+ * Sampled forward straight from the stored operands (full-size operands are
+ * too large to widen to double whole): the three rows an output needs are
+ * decoded into double buffers, then the same one_output() runs.
+ */
+typedef void (*decode_fn)(const void *src, int64_t offset, double *dst,
+                          int64_t n);
+
+static void decode_bf16_rows(const void *src, int64_t offset, double *dst,
+                             int64_t n)
+{
+    const uint16_t *p = (const uint16_t *)src + offset;
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = bf16_bits_to_double(p[i]);
+}
+
+static void decode_f32_rows(const void *src, int64_t offset, double *dst,
+                            int64_t n)
+{
+    const float *p = (const float *)src + offset;
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = (double)p[i];
+}
+
+static int fwd_points(decode_fn dec, const void *X, const void *Wg,
+                      const void *Wu, int64_t K, const int64_t *idx_m,
+                      const int64_t *idx_n, int64_t count, double *G,
+                      double *U, double *H, double *AG, double *AU)
+{
+    int failed = 0;
+#pragma omp parallel reduction(| : failed)
+    {
+        double *buf = (double *)malloc(sizeof(double) * 3 * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(static)
+        for (int64_t i = 0; i < count; ++i) {
+            if (!buf) {
+                failed = 1;
+                continue;
+            }
+            dec(X, idx_m[i] * K, buf, K);
+            dec(Wg, idx_n[i] * K, buf + K, K);
+            dec(Wu, idx_n[i] * K, buf + 2 * K, K);
+            one_output(buf, buf + K, buf + 2 * K, K, G ? G + i : 0,
+                       U ? U + i : 0, H ? H + i : 0, AG ? AG + i : 0,
+                       AU ? AU + i : 0);
+        }
+        free(buf);
+    }
+    return failed ? -1 : 0;
+}
+
+ORACLE_API int oracle_swiglu_fwd_points_bf16(const uint16_t *X,
+                                             const uint16_t *Wg,
+                                             const uint16_t *Wu, int64_t K,
+                                             const int64_t *idx_m,
+                                             const int64_t *idx_n,
+                                             int64_t count, double *G,
+                                             double *U, double *H, double *AG,
+                                             double *AU)
+{
+    return fwd_points(decode_bf16_rows, X, Wg, Wu, K, idx_m, idx_n, count, G,
+                      U, H, AG, AU);
+}
+
+ORACLE_API int oracle_swiglu_fwd_points_f32(const float *X, const float *Wg,
+                                            const float *Wu, int64_t K,
+                                            const int64_t *idx_m,
+                                            const int64_t *idx_n,
+                                            int64_t count, double *G,
+                                            double *U, double *H, double *AG,
+                                            double *AU)
+{
+    return fwd_points(decode_f32_rows, X, Wg, Wu, K, idx_m, idx_n, count, G,
+                      U, H, AG, AU);
+}
+
+/* ---- dSwiGLU backward -------------------------------------------------- */
+
+/*
+ * Elementwise backward of h = silu(g) * u with upstream gradient dh:
+ *   dU = dh * silu(g)
+ *   dG = dh * u * silu'(g)
+ * (the "dSwiGLU" of Liger-Kernel issue #1383).
+ */
+static void dswiglu_one(double dh, double g, double u, double *dg, double *du)
+{
+    *du = dh * oracle_silu(g);
+    *dg = dh * u * oracle_dsilu(g);
+}
+
+/* n contiguous elements, double operands. */
+ORACLE_API void oracle_dswiglu_f64(const double *dH, const double *G,
+                                   const double *U, int64_t n, double *dG,
+                                   double *dU)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        dswiglu_one(dH[i], G[i], U[i], dG + i, dU + i);
+}
+
+/* Same, straight from bf16 bit patterns (full-size n is large). */
+ORACLE_API void oracle_dswiglu_bf16(const uint16_t *dH, const uint16_t *G,
+                                    const uint16_t *U, int64_t n, double *dG,
+                                    double *dU)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        dswiglu_one(bf16_bits_to_double(dH[i]), bf16_bits_to_double(G[i]),
+                    bf16_bits_to_double(U[i]), dG + i, dU + i);
+}
+
+/* Same, fp32 operands. */
+ORACLE_API void oracle_dswiglu_f32(const float *dH, const float *G,
+                                   const float *U, int64_t n, double *dG,
+                                   double *dU)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        dswiglu_one((double)dH[i], (double)G[i], (double)U[i], dG + i, dU + i);
+}

@@ -1,0 +1,14 @@
+"""Test configuration: registers the ``gpu`` marker and puts the repository
+root on sys.path so ``oracle`` and ``up_projection_b200`` import without an
+install step."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")

@@ -1,0 +1,286 @@
+"""Pins for the fp64 oracle: checks against facts fixed by the mathematics,
+by an independent library routine, or by brute force -- never against the
+oracle's own formula retyped.
+
+Every pin takes an ``oracle.Oracle`` instance and raises AssertionError on a
+mismatch, so the same suite runs against the committed oracle and against
+copies with a mistake planted in them (test_oracle_mutants.py), which shows
+that each plausible mistake trips at least one pin.
+
+What pins what:
+  scalar_closed_forms   sigmoid/silu/silu' at points with known values, the
+                        identities silu(-x) = silu(x) - x and
+                        sigmoid(x) + sigmoid(-x) = 1, the silu minimum at
+                        x* = -1 - W(1/e) with value -W(1/e) (W = Lambert W,
+                        computed here by Newton's method), the limits
+                        silu(x) -> x and silu(x) -> 0, and silu' against a
+                        central difference of silu.
+  fwd_library           G, U against numpy float64 matmul (independent BLAS);
+                        the magnitudes AG, AU against |X| @ |W|^T.
+  fwd_brute_force       G, U against exactly rounded sums (math.fsum) of the
+                        exact products, on tiny shapes.
+  fwd_gate_up_roles     H(Wg) - H(-Wg) = G * U elementwise (from the identity
+                        above), with G, U from numpy: fixes which operand is
+                        the gate and the sign convention.
+  fwd_zero_cases        U = 0 => H = 0, Wg = 0 => H = 0.
+  fwd_linear_in_up      H(a Wu) = a H.
+  fwd_one_hot           X = e_k selects weight column k: G = Wg[:, k] and
+                        U = Wu[:, k] exactly.
+  fwd_asymptotes        G = +40 => H ~ 40 U, G = -40 => H ~ 0.
+  fwd_points            the sampled forward equals the full forward.
+  bf16_decoder          all 65536 bf16 patterns decode like torch's bf16.
+  dswiglu_finite_diff   dG, dU against central differences of the forward.
+  dswiglu_special       dh = 0, u = 0, g = 0, g = +-40, g = x*.
+  dswiglu_storage       the bf16 and fp32 entry points agree with the double
+                        one on the decoded values.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+
+def lambert_w_inv_e() -> float:
+    """W(1/e): the root of w e^w = 1/e, by Newton's method from w = 0.3."""
+    w = 0.3
+    target = math.exp(-1.0)
+    for _ in range(60):
+        f = w * math.exp(w) - target
+        w -= f / (math.exp(w) * (1.0 + w))
+    return w
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _bf16_exact(a: np.ndarray) -> np.ndarray:
+    """Round float64 values to bf16 and back (torch RNE), so that every
+    product of two such values is exact in double."""
+    return torch.from_numpy(a).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ---- scalar definitions ---------------------------------------------------
+
+def scalar_closed_forms(o):
+    assert o.silu(0.0) == 0.0
+    assert o.sigmoid(0.0) == 0.5
+    assert o.dsilu(0.0) == 0.5
+    # sigmoid(ln 3) = 1 / (1 + 1/3) = 3/4 and sigmoid(-ln 3) = 1/4.
+    assert abs(o.sigmoid(math.log(3.0)) - 0.75) < 1e-15
+    assert abs(o.sigmoid(-math.log(3.0)) - 0.25) < 1e-15
+    # Limits: silu(30) = 30 / (1 + e^-30) is 30 - 2.8e-12; silu(-40) ~ -1.7e-16.
+    s30 = o.silu(30.0)
+    assert 0.0 < 30.0 - s30 < 1e-11, s30
+    assert abs(o.silu(-40.0)) < 1e-15
+    assert o.silu(-40.0) < 0.0
+    for x in np.linspace(-25.0, 25.0, 101):
+        x = float(x)
+        # silu(-x) = -x (1 - sigmoid(x)) = silu(x) - x
+        assert abs(o.silu(-x) - (o.silu(x) - x)) <= 1e-14 * max(1.0, abs(x)), x
+        assert abs(o.sigmoid(x) + o.sigmoid(-x) - 1.0) <= 4.5e-16, x
+        # silu' against a central difference of silu (step 1e-5: truncation
+        # ~1e-11, rounding ~1e-11).
+        h = 1e-5
+        fd = (o.silu(x + h) - o.silu(x - h)) / (2.0 * h)
+        assert abs(o.dsilu(x) - fd) < 1e-8, (x, o.dsilu(x), fd)
+    # Minimum of silu: silu'(x) = 0 <=> x = -(1 + e^x) <=> x* = -1 - W(1/e),
+    # where silu(x*) = x* + 1 = -W(1/e).
+    w = lambert_w_inv_e()
+    xs = -1.0 - w
+    assert abs(o.silu(xs) - (-w)) < 1e-15, (o.silu(xs), -w)
+    assert abs(o.dsilu(xs)) < 1e-15, o.dsilu(xs)
+    assert o.silu(xs - 1e-3) > o.silu(xs) and o.silu(xs + 1e-3) > o.silu(xs)
+
+
+# ---- forward --------------------------------------------------------------
+
+def _random_problem(M, K, N, seed, scale_w=None):
+    r = _rng(seed)
+    sw = (1.0 / math.sqrt(K)) if scale_w is None else scale_w
+    X = _bf16_exact(r.standard_normal((M, K)))
+    Wg = _bf16_exact(r.standard_normal((N, K)) * sw)
+    Wu = _bf16_exact(r.standard_normal((N, K)) * sw)
+    return X, Wg, Wu
+
+
+def fwd_library(o):
+    for (M, K, N, seed) in [(4, 256, 512, 0), (3, 40, 24, 1), (8, 1536, 64, 2),
+                            (130, 72, 136, 3)]:
+        X, Wg, Wu = _random_problem(M, K, N, seed)
+        out = o.swiglu_fwd_f64(X, Wg, Wu, want_magnitudes=True)
+        G_ref = X @ Wg.T
+        U_ref = X @ Wu.T
+        bound_g = 1e-13 * (np.abs(X) @ np.abs(Wg).T) + 1e-300
+        bound_u = 1e-13 * (np.abs(X) @ np.abs(Wu).T) + 1e-300
+        assert np.all(np.abs(out["G"] - G_ref) <= bound_g), (M, K, N)
+        assert np.all(np.abs(out["U"] - U_ref) <= bound_u), (M, K, N)
+        assert np.allclose(out["AG"], np.abs(X) @ np.abs(Wg).T, rtol=1e-13, atol=0)
+        assert np.allclose(out["AU"], np.abs(X) @ np.abs(Wu).T, rtol=1e-13, atol=0)
+
+
+def fwd_brute_force(o):
+    for (M, K, N, seed) in [(2, 7, 3, 10), (3, 16, 5, 11), (1, 33, 2, 12)]:
+        X, Wg, Wu = _random_problem(M, K, N, seed)
+        out = o.swiglu_fwd_f64(X, Wg, Wu, want_magnitudes=True)
+        for m in range(M):
+            for n in range(N):
+                # products of bf16 values are exact in double; fsum rounds once
+                g = math.fsum(float(X[m, k]) * float(Wg[n, k]) for k in range(K))
+                u = math.fsum(float(X[m, k]) * float(Wu[n, k]) for k in range(K))
+                tol_g = K * 2.0 ** -53 * out["AG"][m, n]
+                tol_u = K * 2.0 ** -53 * out["AU"][m, n]
+                assert abs(out["G"][m, n] - g) <= tol_g, (m, n)
+                assert abs(out["U"][m, n] - u) <= tol_u, (m, n)
+
+
+def fwd_gate_up_roles(o):
+    X, Wg, Wu = _random_problem(5, 64, 48, 20, scale_w=0.3)
+    H_pos = o.swiglu_fwd_f64(X, Wg, Wu)["H"]
+    H_neg = o.swiglu_fwd_f64(X, -Wg, Wu)["H"]
+    GU = (X @ Wg.T) * (X @ Wu.T)
+    scale = np.abs(X) @ np.abs(Wg).T * np.abs(X @ Wu.T) + 1e-300
+    assert np.all(np.abs((H_pos - H_neg) - GU) <= 1e-12 * scale)
+    # and the gate really is nonlinear: H is not G*U/2 everywhere
+    assert np.max(np.abs(H_pos - 0.5 * GU)) > 1e-3
+
+
+def fwd_zero_cases(o):
+    X, Wg, Wu = _random_problem(4, 32, 16, 30)
+    assert np.all(o.swiglu_fwd_f64(X, Wg, np.zeros_like(Wu))["H"] == 0.0)
+    assert np.all(o.swiglu_fwd_f64(X, np.zeros_like(Wg), Wu)["H"] == 0.0)
+    # K = 0: empty sums
+    e = o.swiglu_fwd_f64(np.zeros((3, 0)), np.zeros((2, 0)), np.zeros((2, 0)))
+    assert np.all(e["G"] == 0.0) and np.all(e["H"] == 0.0)
+
+
+def fwd_linear_in_up(o):
+    X, Wg, Wu = _random_problem(4, 64, 32, 40)
+    H = o.swiglu_fwd_f64(X, Wg, Wu)["H"]
+    assert np.array_equal(o.swiglu_fwd_f64(X, Wg, 2.0 * Wu)["H"], 2.0 * H)
+    H3 = o.swiglu_fwd_f64(X, Wg, -3.0 * Wu)["H"]
+    assert np.allclose(H3, -3.0 * H, rtol=1e-14, atol=1e-300)
+
+
+def fwd_one_hot(o):
+    r = _rng(50)
+    K, N = 24, 40
+    _, Wg, Wu = _random_problem(1, K, N, 51, scale_w=1.0)
+    ks = [0, 5, K - 1, 13]
+    X = np.zeros((len(ks), K))
+    for m, k in enumerate(ks):
+        X[m, k] = 1.0
+    out = o.swiglu_fwd_f64(X, Wg, Wu)
+    for m, k in enumerate(ks):
+        assert np.array_equal(out["G"][m], Wg[:, k]), (m, k)
+        assert np.array_equal(out["U"][m], Wu[:, k]), (m, k)
+        for n in range(N):
+            assert out["H"][m, n] == o.silu(Wg[n, k]) * Wu[n, k]
+    del r
+
+
+def fwd_asymptotes(o):
+    # X = [1, 0...], Wg[:,0] = +-40 => G = +-40 exactly; U = Wu[:,0].
+    N, K = 16, 8
+    X = np.zeros((1, K))
+    X[0, 0] = 1.0
+    r = _rng(60)
+    Wu = _bf16_exact(r.standard_normal((N, K)))
+    for gval in (40.0, -40.0):
+        Wg = np.zeros((N, K))
+        Wg[:, 0] = gval
+        H = o.swiglu_fwd_f64(X, Wg, Wu)["H"][0]
+        U = Wu[:, 0]
+        if gval > 0:
+            assert np.allclose(H, 40.0 * U, rtol=1e-15, atol=0)
+        else:
+            assert np.all(np.abs(H) <= 40.0 * math.exp(-40.0) * np.abs(U) * 1.01)
+
+
+def fwd_points(o):
+    from up_projection_b200 import synth  # seeded inputs only
+    M, K, N = 9, 136, 72
+    for dtype in ("bf16", "f32"):
+        X, Wg, Wu = synth.swiglu_inputs(M, K, N, dtype=dtype, seed=7)
+        full = o.swiglu_fwd(X, Wg, Wu, dtype=dtype, want_magnitudes=True)
+        r = _rng(70)
+        im = r.integers(0, M, size=200)
+        inn = r.integers(0, N, size=200)
+        pts = o.swiglu_fwd_points(X, Wg, Wu, im, inn, dtype=dtype)
+        for key in ("G", "U", "H", "AG", "AU"):
+            assert np.array_equal(pts[key], full[key][im, inn]), (dtype, key)
+        # and against numpy on the decoded operands
+        Xd = X.to(torch.float64).numpy()
+        Wgd = Wg.to(torch.float64).numpy()
+        G_np = np.einsum("ik,ik->i", Xd[im], Wgd[inn])
+        assert np.all(np.abs(pts["G"] - G_np) <= 1e-13 * pts["AG"] + 1e-300)
+
+
+def bf16_decoder(o):
+    bits = np.arange(65536, dtype=np.uint16)
+    ours = o.decode_bf16(bits)
+    theirs = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16) \
+        .to(torch.float64).numpy()
+    nan = np.isnan(theirs)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], theirs[~nan])
+    # signed zeros keep their sign
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(theirs[~nan]))
+
+
+# ---- backward ------------------------------------------------------------
+
+def _fwd_scalar(o, g, u):
+    """h(g, u) = silu(g) u through the oracle's FORWARD path (K = 1)."""
+    return float(o.swiglu_fwd_f64(np.array([[1.0]]), np.array([[g]]),
+                                  np.array([[u]]))["H"][0, 0])
+
+
+def dswiglu_finite_diff(o):
+    r = _rng(80)
+    g = np.concatenate([r.standard_normal(40) * 3.0, [0.0, -1.2784, 5.0, -6.0]])
+    u = r.standard_normal(g.size)
+    dh = r.standard_normal(g.size)
+    dG, dU = o.dswiglu_f64(dh, g, u)
+    d = 1e-6
+    for i in range(g.size):
+        fd_g = (_fwd_scalar(o, g[i] + d, u[i]) - _fwd_scalar(o, g[i] - d, u[i])) / (2 * d)
+        fd_u = (_fwd_scalar(o, g[i], u[i] + d) - _fwd_scalar(o, g[i], u[i] - d)) / (2 * d)
+        sg = abs(dh[i]) * (abs(u[i]) + 1.0)
+        su = abs(dh[i]) * (abs(g[i]) + 1.0)
+        assert abs(dG[i] - dh[i] * fd_g) <= 2e-8 * sg, (i, g[i], dG[i], dh[i] * fd_g)
+        assert abs(dU[i] - dh[i] * fd_u) <= 2e-8 * su, (i, g[i], dU[i], dh[i] * fd_u)
+
+
+def dswiglu_special(o):
+    w = lambert_w_inv_e()
+    g = np.array([0.0, 1.0, 40.0, -40.0, -1.0 - w, 2.0])
+    u = np.array([3.0, 0.0, 2.0, 2.0, 1.5, -1.0])
+    dh = np.array([2.0, 1.0, 1.0, 1.0, 1.0, 0.0])
+    dG, dU = o.dswiglu_f64(dh, g, u)
+    assert dU[0] == 0.0 and dG[0] == 2.0 * 3.0 * 0.5      # g = 0
+    assert dG[1] == 0.0                                    # u = 0
+    assert abs(dU[1] - o.silu(1.0)) < 1e-16
+    assert abs(dU[2] - 40.0) < 1e-14 and abs(dG[2] - 2.0) < 1e-14   # g -> +inf
+    assert abs(dU[3]) < 1e-15 and abs(dG[3]) < 1e-15                # g -> -inf
+    assert abs(dG[4]) < 1e-15                               # silu'(x*) = 0
+    assert abs(dU[4] - 1.0 * (-w)) < 1e-15                  # silu(x*) = -W(1/e)
+    assert dG[5] == 0.0 and dU[5] == 0.0                   # dh = 0
+
+
+def dswiglu_storage(o):
+    from up_projection_b200 import synth
+    for dtype in ("bf16", "f32"):
+        dH, G, U = synth.dswiglu_inputs(1000, dtype=dtype, seed=9)
+        dG, dU = o.dswiglu(dH, G, U, dtype=dtype)
+        dG2, dU2 = o.dswiglu_f64(o.decode(dH, dtype), o.decode(G, dtype),
+                                 o.decode(U, dtype))
+        assert np.array_equal(dG, dG2) and np.array_equal(dU, dU2), dtype
+
+
+ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
+            fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
+            fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
+            dswiglu_special, dswiglu_storage]
