@@ -1,0 +1,88 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/swiglu.h declares, and validates arguments on the host before any
+CUDA call (so the error codes are the same with or without a device)."""
+import os
+import re
+
+import pytest
+
+from up_projection_b200 import _capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "swiglu.h")).read()
+    return re.findall(r"SWIGLU_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert {"swiglu_fwd", "dswiglu_bwd", "dswiglu_bwd_dtype"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _capi.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _capi.SIGNATURES, f"binding lacks {name}"
+
+
+def test_routes_are_a_pure_function_of_shape():
+    r = _capi.swiglu_route_for
+    assert r(8, 1536, 6912, 0) == _capi.ROUTE_DECODE_BF16
+    assert r(1, 4096, 11008, 0) == _capi.ROUTE_DECODE_BF16
+    assert r(9, 4096, 11008, 0) == _capi.ROUTE_GEMM_BF16
+    assert r(8192, 4096, 14336, 0) == _capi.ROUTE_GEMM_BF16
+    assert r(2048, 5120, 13824, 1) == _capi.ROUTE_GEMM_TF32X3
+    assert r(8, 64, 64, 1) == _capi.ROUTE_GEMM_TF32X3
+    assert r(4, 65536, 64, 0) == _capi.ROUTE_GEMM_BF16   # X stage too big for decode
+    assert r(0, 64, 64, 0) == _capi.ROUTE_NONE
+    assert r(4, 64, 0, 0) == _capi.ROUTE_NONE
+    assert r(4, 0, 64, 0) == _capi.ROUTE_ZERO_K
+    assert r(4, 60, 64, 0) == -1          # K not a multiple of 8 (bf16)
+    assert r(4, 60, 64, 1) == _capi.ROUTE_GEMM_TF32X3   # multiple of 4 is fine for fp32
+    assert r(4, 64, 66, 1) == -1
+    assert r(-1, 64, 64, 0) == -1
+    assert r(1 << 31, 64, 64, 0) == -1
+    assert r(4, 64, 64, 2) == -1
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, None, None, None, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((16, 32, 48, 17, 4, 64, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_PTR),
+    ((16, 32, 48, 64, 4, 64, 64, 3), _capi.SWIGLU_ERR_BAD_DTYPE),
+    ((16, 32, 48, 64, 4, 63, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, -4, 64, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
+    # H [4,64] bf16 at 1 MiB overlaps X [4,64] placed inside it
+    ((1 << 20, 1 << 24, 1 << 25, (1 << 20) - 16, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),
+    ((None, None, None, None, 0, 64, 64, 0), _capi.SWIGLU_OK),
+])
+def test_fwd_host_validation(args, code):
+    assert _capi.lib().swiglu_fwd(*args, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, 16, 32, 48, 64, 10), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((16, 32, 48, 64, 80, -1), _capi.SWIGLU_ERR_BAD_DIM),
+    ((16, 32, 48, 65, 80, 10), _capi.SWIGLU_ERR_MISALIGNED_PTR),
+    ((1 << 20, 1 << 21, 1 << 22, 1 << 20, 1 << 23, 1000), _capi.SWIGLU_ERR_OVERLAP),  # dG == dH
+    ((1 << 20, 1 << 21, 1 << 22, (1 << 21) + 16, 1 << 23, 1000), _capi.SWIGLU_ERR_OVERLAP),
+    ((None, None, None, None, None, 0), _capi.SWIGLU_OK),
+])
+def test_bwd_host_validation(args, code):
+    assert _capi.lib().dswiglu_bwd(*args, None) == code
+
+
+def test_no_device_is_an_error_not_a_fallback():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _capi.lib().swiglu_fwd(1 << 20, 1 << 21, 1 << 22, 1 << 23, 4, 64, 64, 0, None)
+    assert st == _capi.SWIGLU_ERR_NO_DEVICE
+
+
+def test_status_strings():
+    for code in range(11):
+        assert _capi.status_string(code)
+    assert _capi.status_string(999) == "unknown status"

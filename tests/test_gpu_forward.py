@@ -1,0 +1,152 @@
+"""Fused forward kernels (decode weight streaming, tcgen05 dual GEMM) vs the
+fp64 oracle, through the C ABI: element by element on small and ragged
+shapes, on sampled outputs at the full workload sizes, bit-exact on integer
+inputs, with guard canaries around every output."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_bf16_close, assert_guards_intact, dev, f64, guarded_empty,
+                      sample_indices, to_dev)
+from up_projection_b200 import _capi, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(X, Wg, Wu, expect_route=None):
+    M, K = X.shape
+    N = Wg.shape[0]
+    Xd, Wgd, Wud = to_dev(X, Wg, Wu)
+    full, H = guarded_empty(M * N, X.dtype)
+    _capi.swiglu_fwd(Xd, Wgd, Wud, H.view(M, N))
+    st = _capi.swiglu_sync_status()
+    assert st == _capi.SWIGLU_OK, _capi.status_string(st)
+    if expect_route is not None:
+        assert _capi.swiglu_last_route() == expect_route
+    assert_guards_intact(full)
+    return H.view(M, N).cpu()
+
+
+def check_full(X, Wg, Wu, expect_route, what):
+    H = run_fwd(X, Wg, Wu, expect_route)
+    ref = oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"]
+    assert_bf16_close(f64(H), ref, what)
+    return H
+
+
+# ---------------------------------------------------------------- decode
+
+def test_tiny_config():
+    """X bf16 [4, 256], Wg/Wu [512, 256] ~ N(0, 1/K), seed 0."""
+    X, Wg, Wu = synth.swiglu_inputs(4, 256, 512, "bf16", seed=0)
+    check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, "tiny")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("K,N", [(256, 512), (264, 72), (8, 8), (1536, 6912), (40, 1032)])
+def test_decode_shapes(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 1000 + K)
+    check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"decode M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_decode_llama7b_full(M):
+    """LLaMA-2 7B up/gate shape: K = 4096, N = 11008 (all outputs checked)."""
+    X, Wg, Wu = synth.swiglu_inputs(M, 4096, 11008, "bf16", seed=7 + M)
+    check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"llama7b M={M}")
+
+
+def test_decode_integer_exact():
+    """Integer operands with every gate pre-activation >= 17: sigmoid rounds
+    to 1 in fp32, so H = bf16_rne(fp32(G * U)) exactly, for every tile and
+    lane position -- any indexing or layout slip changes bits."""
+    for M, K, N in [(8, 256, 512), (3, 136, 1024), (1, 64, 8)]:
+        X, Wg, Wu = synth.integer_inputs(M, K, N, seed=M + K)
+        H = run_fwd(X, Wg, Wu, _capi.ROUTE_DECODE_BF16)
+        G = X.to(torch.float64) @ Wg.to(torch.float64).T
+        U = X.to(torch.float64) @ Wu.to(torch.float64).T
+        assert float(G.min()) >= 17.0
+        expect = (G * U).to(torch.float32).to(torch.bfloat16)
+        assert torch.equal(H.view(torch.int16), expect.view(torch.int16)), (M, K, N)
+
+
+def test_decode_deterministic():
+    X, Wg, Wu = synth.swiglu_inputs(8, 1536, 6912, "bf16", seed=3)
+    a = run_fwd(X, Wg, Wu)
+    b = run_fwd(X, Wg, Wu)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# --------------------------------------------------------------- dual GEMM
+
+@pytest.mark.parametrize("M,K,N", [
+    (9, 256, 512),       # smallest GEMM-route M
+    (128, 64, 128),      # one tile, one k-block
+    (128, 128, 256),     # two k-blocks, two N tiles
+    (129, 72, 136),      # ragged M, ragged K (not a multiple of 64), ragged N
+    (300, 520, 392),     # several ragged tiles
+    (256, 4096, 512),    # long K: the smem ring wraps many times
+])
+def test_gemm_small_shapes(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M + K + N)
+    check_full(X, Wg, Wu, _capi.ROUTE_GEMM_BF16, f"gemm M={M} K={K} N={N}")
+
+
+def test_gemm_many_tiles_per_cta():
+    """Enough tiles that every persistent CTA runs many, so both TMEM
+    accumulator buffers and all smem stages are recycled."""
+    M, K, N = 2048, 512, 4096
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=11)
+    check_full(X, Wg, Wu, _capi.ROUTE_GEMM_BF16, "gemm many tiles")
+
+
+def test_gemm_integer_exact():
+    for M, K, N in [(256, 256, 384), (130, 64, 136)]:
+        X, Wg, Wu = synth.integer_inputs(M, K, N, seed=M + N)
+        H = run_fwd(X, Wg, Wu, _capi.ROUTE_GEMM_BF16)
+        G = X.to(torch.float64) @ Wg.to(torch.float64).T
+        U = X.to(torch.float64) @ Wu.to(torch.float64).T
+        assert float(G.min()) >= 17.0
+        expect = (G * U).to(torch.float32).to(torch.bfloat16)
+        diff = (H.view(torch.int16) != expect.view(torch.int16))
+        assert not bool(diff.any()), f"{int(diff.sum())} mismatches, first {diff.nonzero()[:5].tolist()}"
+
+
+def test_prefill_full_size_sampled():
+    """LLaMA-3 8B prefill shape, the launch the bench times: M = 8192,
+    K = 4096, N = 14336; sampled outputs against the oracle, plus a rerun
+    that must be bitwise identical."""
+    M, K, N = 8192, 4096, 14336
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=0)
+    H = run_fwd(X, Wg, Wu, _capi.ROUTE_GEMM_BF16)
+    im, inn = sample_indices(M, N, 4000)
+    ref = oracle.swiglu_fwd_points(X, Wg, Wu, im, inn, "bf16")["H"]
+    assert_bf16_close(f64(H[im, inn]), ref, "prefill sampled")
+    # whole rows/columns at tile boundaries
+    for m in (0, 127, 128, 8191):
+        cols = np.arange(N)
+        r = oracle.swiglu_fwd_points(X, Wg, Wu, np.full(N, m), cols, "bf16")["H"]
+        assert_bf16_close(f64(H[m]), r, f"prefill row {m}")
+    H2 = run_fwd(X, Wg, Wu)
+    assert torch.equal(H.view(torch.int16), H2.view(torch.int16))
+
+
+def test_decode_astrai_full_size_rotated_copies():
+    """AstrAI-1B decode as the bench runs it: 16 rotated weight copies,
+    M in {1, 2, 4, 8}; every output of copies 0 and 15 checked."""
+    K, N, R = 1536, 6912, 16
+    X8, Wg, Wu = synth.swiglu_inputs(8, K, N, "bf16", seed=0)
+    Wgd = torch.empty((R, N, K), dtype=torch.bfloat16, device=dev())
+    Wud = torch.empty_like(Wgd)
+    Wgd[:] = Wg.to(dev())
+    Wud[:] = Wu.to(dev())
+    for M in (1, 2, 4, 8):
+        X = X8[:M].contiguous()
+        ref = oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"]
+        Xd = X.to(dev())
+        for r in (0, R - 1):
+            H = _capi.swiglu_fwd(Xd, Wgd[r], Wud[r])
+            assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+            assert _capi.swiglu_last_route() == _capi.ROUTE_DECODE_BF16
+            assert_bf16_close(f64(H), ref, f"astrai M={M} copy={r}")

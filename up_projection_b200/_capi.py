@@ -1,0 +1,187 @@
+"""ctypes binding of libswiglu_b200.so (the C ABI of include/swiglu.h).
+
+Argument marshalling only: torch tensors become device pointers and the
+current CUDA stream becomes a cudaStream_t; the library does all the work.
+The library is loaded on first use; if it is missing or cannot be loaded the
+call raises -- there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libswiglu_b200.so")
+
+# enum swiglu_dtype
+SWIGLU_BF16 = 0
+SWIGLU_FP32 = 1
+# enum swiglu_status
+SWIGLU_OK = 0
+SWIGLU_ERR_NULL_POINTER = 1
+SWIGLU_ERR_BAD_DIM = 2
+SWIGLU_ERR_MISALIGNED_DIM = 3
+SWIGLU_ERR_MISALIGNED_PTR = 4
+SWIGLU_ERR_BAD_DTYPE = 5
+SWIGLU_ERR_UNSUPPORTED_DEVICE = 6
+SWIGLU_ERR_CUDA = 7
+SWIGLU_ERR_TIMEOUT = 8
+SWIGLU_ERR_OVERLAP = 9
+SWIGLU_ERR_NO_DEVICE = 10
+# enum swiglu_route
+ROUTE_NONE = 0
+ROUTE_ZERO_K = 1
+ROUTE_DECODE_BF16 = 2
+ROUTE_GEMM_BF16 = 3
+ROUTE_GEMM_TF32X3 = 4
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+
+# name -> (restype, argtypes), mirroring include/swiglu.h
+SIGNATURES = {
+    "swiglu_fwd": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
+    "dswiglu_bwd": (_I, [_P, _P, _P, _P, _P, _I64, _P]),
+    "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
+    "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
+    "swiglu_last_route": (_I, []),
+    "swiglu_status_string": (ctypes.c_char_p, [_I]),
+    "swiglu_sync_status": (_I, [_P]),
+    "swiglu_read_floor": (_I, [_P, _P, _I64, _P, _P]),
+    "swiglu_read_floor_sink_words": (_I64, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SwigluError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it is not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m up_projection_b200.build` (nvcc, sm_100a)")
+            handle = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(handle, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().swiglu_status_string(int(status)).decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn: str, st: int):
+    if st != SWIGLU_OK:
+        raise SwigluError(fn, st)
+
+
+_DT = {torch.bfloat16: SWIGLU_BF16, torch.float32: SWIGLU_FP32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+    return _DT[t.dtype]
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
+               H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = silu(X Wg^T) * (X Wu^T) through the C ABI.  X [..., K] (leading
+    dims are flattened to M rows, as the TensorRT-LLM fused up-projection
+    does), Wg/Wu [N, K]; bf16 or fp32, all contiguous on one GPU."""
+    for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
+        _dev(t, n)
+    if not (X.dtype == Wg.dtype == Wu.dtype):
+        raise TypeError("X, Wg and Wu must share a dtype")
+    K = X.shape[-1]
+    N = Wg.shape[0]
+    if Wg.shape != (N, K) or Wu.shape != (N, K):
+        raise ValueError(f"weights must be [N, K] = [{N}, {K}]")
+    lead = X.shape[:-1]
+    M = 1
+    for d in lead:
+        M *= d
+    if H is None:
+        H = torch.empty((*lead, N), dtype=X.dtype, device=X.device)
+    else:
+        _dev(H, "H")
+        if H.dtype != X.dtype or H.numel() != M * N:
+            raise ValueError("H has the wrong dtype or size")
+    st = lib().swiglu_fwd(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
+                          M, K, N, _dtype_code(X), _stream(stream))
+    _check("swiglu_fwd", st)
+    return H
+
+
+def dswiglu_bwd(dH: torch.Tensor, G: torch.Tensor, U: torch.Tensor,
+                dG: torch.Tensor | None = None, dU: torch.Tensor | None = None,
+                stream=None):
+    """(dG, dU) of h = silu(g) * u through the C ABI (bf16 or fp32)."""
+    for t, n in ((dH, "dH"), (G, "G"), (U, "U")):
+        _dev(t, n)
+    if not (dH.dtype == G.dtype == U.dtype) or dH.shape != G.shape or G.shape != U.shape:
+        raise ValueError("dH, G, U must share dtype and shape")
+    dG = torch.empty_like(G) if dG is None else dG
+    dU = torch.empty_like(U) if dU is None else dU
+    _dev(dG, "dG")
+    _dev(dU, "dU")
+    st = lib().dswiglu_bwd_dtype(dH.data_ptr(), G.data_ptr(), U.data_ptr(), dG.data_ptr(),
+                                 dU.data_ptr(), G.numel(), _dtype_code(G), _stream(stream))
+    _check("dswiglu_bwd", st)
+    return dG, dU
+
+
+def swiglu_route_for(M: int, K: int, N: int, dtype: int) -> int:
+    return lib().swiglu_route_for(M, K, N, dtype)
+
+
+def swiglu_last_route() -> int:
+    return lib().swiglu_last_route()
+
+
+def swiglu_sync_status(stream=None) -> int:
+    return lib().swiglu_sync_status(_stream(stream))
+
+
+def swiglu_read_floor(A: torch.Tensor, B: torch.Tensor, sink: torch.Tensor,
+                      stream=None) -> None:
+    """Bench-only: stream-read A and B (same byte size) once."""
+    _dev(A, "A")
+    _dev(B, "B")
+    nbytes = A.numel() * A.element_size()
+    if B.numel() * B.element_size() != nbytes:
+        raise ValueError("A and B must have the same size in bytes")
+    st = lib().swiglu_read_floor(A.data_ptr(), B.data_ptr(), nbytes, sink.data_ptr(),
+                                 _stream(stream))
+    _check("swiglu_read_floor", st)

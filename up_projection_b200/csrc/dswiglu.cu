@@ -1,0 +1,223 @@
+// dswiglu.cu -- elementwise dSwiGLU backward (the "dSwiGLU" of Liger-Kernel
+// issue #1383) and the bench-only read-floor probe.
+//
+//   dU = dH * silu(G),   dG = dH * U * silu'(G),
+//   silu(g) = g s,  silu'(g) = s (1 + g (1 - s)),  s = sigmoid(g).
+//
+// HBM-bound (3 loads + 2 stores per element): 128-bit vector accesses,
+// L1-bypassing loads, streaming stores, a grid of a few CTAs per SM looping
+// over the vectors.  The sigmoid is evaluated from t = exp(-|g|) so that both
+// s and 1 - s are formed without cancellation:
+//   g >= 0:  s = 1/(1+t),  1-s = t/(1+t);     g < 0:  s = t/(1+t),  1-s = 1/(1+t).
+// fp32 I/O uses expf and IEEE division (a few ulp); bf16 I/O uses the fast
+// hardware approximations, far below the bf16 output rounding.
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace swiglu {
+namespace {
+
+using namespace dev;
+
+constexpr int kThreads = 256;
+constexpr int kBlocksPerSm = 8;
+constexpr int kUnroll = 2;
+
+template <bool kFast>
+__device__ __forceinline__ void dswiglu_elem(float dh, float g, float u, float &dg, float &du) {
+    const float a = fabsf(g);
+    float t, r;
+    if (kFast) {
+        t = __expf(-a);
+        r = __frcp_rn(1.0f + t);
+    } else {
+        t = expf(-a);
+        r = 1.0f / (1.0f + t);
+    }
+    const float tr = t * r;
+    const bool pos = g >= 0.0f;
+    const float s = pos ? r : tr;      // sigmoid(g)
+    const float oms = pos ? tr : r;    // 1 - sigmoid(g)
+    const float silu = g * s;
+    const float dsilu = s * (1.0f + g * oms);
+    du = dh * silu;
+    dg = dh * u * dsilu;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// One 16-byte vector of each operand: 8 bf16 elements.
+__device__ __forceinline__ void vec_bf16(const uint4 &dh, const uint4 &g, const uint4 &u,
+                                         uint4 &dg, uint4 &du) {
+    const uint32_t *pdh = &dh.x, *pg = &g.x, *pu = &u.x;
+    uint32_t *pdg = &dg.x, *pdu = &du.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float g0, u0, g1, u1;
+        dswiglu_elem<true>(bf_lo(pdh[i]), bf_lo(pg[i]), bf_lo(pu[i]), g0, u0);
+        dswiglu_elem<true>(bf_hi(pdh[i]), bf_hi(pg[i]), bf_hi(pu[i]), g1, u1);
+        pdg[i] = pack_bf16x2(g0, g1);
+        pdu[i] = pack_bf16x2(u0, u1);
+    }
+}
+
+// 4 fp32 elements.
+__device__ __forceinline__ void vec_f32(const uint4 &dh, const uint4 &g, const uint4 &u,
+                                        uint4 &dg, uint4 &du) {
+    const uint32_t *pdh = &dh.x, *pg = &g.x, *pu = &u.x;
+    uint32_t *pdg = &dg.x, *pdu = &du.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float a, b;
+        dswiglu_elem<false>(__uint_as_float(pdh[i]), __uint_as_float(pg[i]),
+                            __uint_as_float(pu[i]), a, b);
+        pdg[i] = __float_as_uint(a);
+        pdu[i] = __float_as_uint(b);
+    }
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kThreads)
+    dswiglu_kernel(const uint4 *dH, const uint4 *G, const uint4 *U, uint4 *dG, uint4 *dU,
+                   int64_t nvec, const void *dH_tail, const void *G_tail, const void *U_tail,
+                   void *dG_tail, void *dU_tail, int tail) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    for (; i + (kUnroll - 1) * stride < nvec; i += kUnroll * stride) {
+        uint4 a[kUnroll], b[kUnroll], c[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            a[j] = ld_stream_v4(dH + i + j * stride);
+            b[j] = ld_stream_v4(G + i + j * stride);
+            c[j] = ld_stream_v4(U + i + j * stride);
+        }
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            uint4 og, ou;
+            if (kBf16) vec_bf16(a[j], b[j], c[j], og, ou);
+            else vec_f32(a[j], b[j], c[j], og, ou);
+            st_stream_v4(dG + i + j * stride, og);
+            st_stream_v4(dU + i + j * stride, ou);
+        }
+    }
+    for (; i < nvec; i += stride) {
+        const uint4 a = ld_stream_v4(dH + i), b = ld_stream_v4(G + i), c = ld_stream_v4(U + i);
+        uint4 og, ou;
+        if (kBf16) vec_bf16(a, b, c, og, ou);
+        else vec_f32(a, b, c, og, ou);
+        st_stream_v4(dG + i, og);
+        st_stream_v4(dU + i, ou);
+    }
+    // Elements after the last whole vector (fewer than one vector's worth).
+    if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < tail) {
+        const int j = threadIdx.x;
+        if (kBf16) {
+            const __nv_bfloat16 *pdh = static_cast<const __nv_bfloat16 *>(dH_tail);
+            const __nv_bfloat16 *pg = static_cast<const __nv_bfloat16 *>(G_tail);
+            const __nv_bfloat16 *pu = static_cast<const __nv_bfloat16 *>(U_tail);
+            float og, ou;
+            dswiglu_elem<true>(__bfloat162float(pdh[j]), __bfloat162float(pg[j]),
+                               __bfloat162float(pu[j]), og, ou);
+            static_cast<__nv_bfloat16 *>(dG_tail)[j] = __float2bfloat16_rn(og);
+            static_cast<__nv_bfloat16 *>(dU_tail)[j] = __float2bfloat16_rn(ou);
+        } else {
+            const float *pdh = static_cast<const float *>(dH_tail);
+            const float *pg = static_cast<const float *>(G_tail);
+            const float *pu = static_cast<const float *>(U_tail);
+            float og, ou;
+            dswiglu_elem<false>(pdh[j], pg[j], pu[j], og, ou);
+            static_cast<float *>(dG_tail)[j] = og;
+            static_cast<float *>(dU_tail)[j] = ou;
+        }
+    }
+}
+
+// ------------------------------------------------------------ read floor
+
+constexpr int kProbeThreads = 512;
+constexpr int kProbeBlocksPerSm = 4;
+constexpr int kProbeUnroll = 4;
+
+__global__ void __launch_bounds__(kProbeThreads)
+    read_floor_kernel(const uint4 *A, const uint4 *B, int64_t nvec, uint32_t *sink) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kProbeThreads;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * kProbeThreads + threadIdx.x;
+    uint32_t acc = 0;
+    for (; i + (kProbeUnroll - 1) * stride < nvec; i += kProbeUnroll * stride) {
+        uint4 a[kProbeUnroll], b[kProbeUnroll];
+#pragma unroll
+        for (int j = 0; j < kProbeUnroll; ++j) {
+            a[j] = ld_nc_stream_v4(A + i + j * stride);
+            b[j] = ld_nc_stream_v4(B + i + j * stride);
+        }
+#pragma unroll
+        for (int j = 0; j < kProbeUnroll; ++j)
+            acc ^= a[j].x ^ a[j].y ^ a[j].z ^ a[j].w ^ b[j].x ^ b[j].y ^ b[j].z ^ b[j].w;
+    }
+    for (; i < nvec; i += stride) {
+        const uint4 a = ld_nc_stream_v4(A + i), b = ld_nc_stream_v4(B + i);
+        acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    __shared__ uint32_t part[kProbeThreads / 32];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t x = 0;
+        for (int w = 0; w < kProbeThreads / 32; ++w) x ^= part[w];
+        sink[blockIdx.x] = x;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG, void *dU,
+                           int64_t n, int dtype, const DeviceInfo &dev, cudaStream_t stream) {
+    const int per_vec = dtype == 0 ? 8 : 4;
+    const int esize = dtype == 0 ? 2 : 4;
+    const int64_t nvec = n / per_vec;
+    const int tail = static_cast<int>(n - nvec * per_vec);
+    const int64_t off = nvec * per_vec * esize;
+    const char *tdh = static_cast<const char *>(dH) + off;
+    const char *tg = static_cast<const char *>(G) + off;
+    const char *tu = static_cast<const char *>(U) + off;
+    char *tdg = static_cast<char *>(dG) + off;
+    char *tdu = static_cast<char *>(dU) + off;
+    const int64_t want_blocks = (nvec + kThreads - 1) / kThreads;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * kBlocksPerSm;
+    int grid = static_cast<int>(want_blocks < cap ? want_blocks : cap);
+    if (grid < 1) grid = 1;
+    if (dtype == 0) {
+        dswiglu_kernel<true><<<grid, kThreads, 0, stream>>>(
+            static_cast<const uint4 *>(dH), static_cast<const uint4 *>(G),
+            static_cast<const uint4 *>(U), static_cast<uint4 *>(dG), static_cast<uint4 *>(dU), nvec,
+            tdh, tg, tu, tdg, tdu, tail);
+    } else {
+        dswiglu_kernel<false><<<grid, kThreads, 0, stream>>>(
+            static_cast<const uint4 *>(dH), static_cast<const uint4 *>(G),
+            static_cast<const uint4 *>(U), static_cast<uint4 *>(dG), static_cast<uint4 *>(dU), nvec,
+            tdh, tg, tu, tdg, tdu, tail);
+    }
+    return cudaGetLastError();
+}
+
+int read_floor_grid(const DeviceInfo &dev) { return dev.sm_count * kProbeBlocksPerSm; }
+
+cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
+                              const DeviceInfo &dev, cudaStream_t stream) {
+    read_floor_kernel<<<read_floor_grid(dev), kProbeThreads, 0, stream>>>(
+        static_cast<const uint4 *>(A), static_cast<const uint4 *>(B), bytes / 16,
+        static_cast<uint32_t *>(sink));
+    return cudaGetLastError();
+}
+
+}  // namespace swiglu

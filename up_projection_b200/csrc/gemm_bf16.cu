@@ -1,0 +1,352 @@
+// gemm_bf16.cu -- fused SwiGLU dual GEMM for bf16, sm_100a.
+//
+//   H[m, n] = silu(sum_k X[m,k] Wg[n,k]) * (sum_k X[m,k] Wu[n,k])
+//
+// The "dual gemm with activations" of Liger-Kernel issue #937 (approach 3),
+// written for Blackwell's 5th-generation tensor cores:
+//
+//  * one CTA per SM, persistent over 128 x 128 output tiles;
+//  * warp 0 (one thread): TMA producer.  Per 64-deep k-block it loads the X
+//    tile [128 x 64] once and the Wg and Wu tiles [128 x 64] stacked into one
+//    256-row B tile, into a 4-stage shared-memory ring (128-byte swizzle);
+//  * warp 1 (one thread): MMA issuer.  One tcgen05.mma (M=128, N=256, K=16)
+//    per 16-deep step multiplies the shared X tile by the stacked [Wg; Wu]
+//    tile, so both projections share one read of X from shared memory and
+//    the accumulator holds the gate in columns 0..127 and the up projection
+//    in columns 128..255 (fp32, in tensor memory).  The accumulator is double
+//    buffered (2 x 256 of the 512 TMEM columns) so the next tile's MMAs run
+//    while the epilogue drains the previous one;
+//  * warps 2..5: epilogue.  tcgen05.ld brings matching gate/up columns of a
+//    row into registers, h = g * sigmoid(g) * u is formed in fp32 on the
+//    accumulators (no intermediate rounding, as the numerics note of
+//    TensorRT-LLM PR #17693 describes for a fused epilogue), rounded once to
+//    bf16, written to a swizzled staging buffer and stored by TMA.  G and U
+//    never reach global memory.
+//
+// Edge tiles: TMA zero-fills rows/columns/k beyond the tensor on load and
+// clips the store.  Every wait is bounded (ptx.cuh): a stuck pipeline sets
+// the status word and the kernel returns after releasing what it holds.
+#include <cuda_bf16.h>
+
+#include <atomic>
+
+#include "gemm_common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace swiglu {
+
+// Status word of this translation unit's kernel; bit 0 = a bounded wait
+// gave up.  Read and cleared by gemm_bf16_status_fetch_and_clear().
+__device__ unsigned int g_gemm_bf16_status;
+
+namespace {
+
+using namespace dev;
+using gemm::mbar_wait_drain;
+using gemm::tile_coords;
+
+constexpr int kBM = 128;                // rows of X per tile (= MMA M)
+constexpr int kBN = 128;                // columns of H per tile (gate, up each)
+constexpr int kBK = 64;                 // k per stage: one 128-byte bf16 row
+constexpr int kStages = 4;
+constexpr int kUmmaK = 16;              // k per tcgen05.mma, kind::f16
+constexpr int kAccCols = 2 * kBN;       // TMEM columns per accumulator buffer
+constexpr int kTmemCols = 2 * kAccCols; // double buffered: all 512 columns
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+constexpr uint32_t kABytes = kBM * kBK * 2;           // 16 KB
+constexpr uint32_t kBBytes = 2 * kBN * kBK * 2;       // 32 KB: Wg rows, Wu rows
+constexpr uint32_t kStageBytes = kABytes + kBBytes;   // 48 KB
+constexpr uint32_t kEpiBufBytes = 32 * 128;           // 32 rows x 64 bf16
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+constexpr uint32_t kOffEpi = kOffB + kStages * kBBytes;
+constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
+constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tfull, tempty, drain
+constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
+constexpr uint32_t kSmemUsed = kOffAbort + 8;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;       // slack for 1024-B alignment
+
+static_assert(kBN % 64 == 0, "epilogue works in 64-column chunks");
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+
+__device__ __forceinline__ float silu_mul_fast(uint32_t gbits, uint32_t ubits) {
+    const float g = __uint_as_float(gbits);
+    const float u = __uint_as_float(ubits);
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    swiglu_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_x,
+                            const __grid_constant__ CUtensorMap tm_wg,
+                            const __grid_constant__ CUtensorMap tm_wu,
+                            const __grid_constant__ CUtensorMap tm_h, int M, int N, int K,
+                            int num_m_tiles, int num_n_tiles) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+
+    const uint32_t sa = base + kOffA;
+    const uint32_t sb = base + kOffB;
+    const uint32_t se = base + kOffEpi;
+    const uint32_t bar_full = base + kOffBar;
+    const uint32_t bar_empty = bar_full + 8 * kStages;
+    const uint32_t bar_tfull = bar_empty + 8 * kStages;
+    const uint32_t bar_tempty = bar_tfull + 16;
+    const uint32_t bar_drain = bar_tempty + 16;
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + kOffTmemPtr);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int num_tiles = num_m_tiles * num_n_tiles;
+    const int num_kb = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, kEpiWarps);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_wg);
+        tma_prefetch_desc(&tm_wu);
+        tma_prefetch_desc(&tm_h);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
+
+    bool failed = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+                const int m0 = mt * kBM, n0 = nt * kBN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t a_dst = sa + stage * kABytes;
+                    const uint32_t b_dst = sb + stage * kBBytes;
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    tma_load_2d(&tm_x, fb, a_dst, kb * kBK, m0);
+                    tma_load_2d(&tm_wg, fb, b_dst, kb * kBK, n0);
+                    tma_load_2d(&tm_wu, fb, b_dst + kBBytes / 2, kb * kBK, n0);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Never leave while a load issued here may still write shared memory.
+            for (int s = 0; s < kStages; ++s) {
+                if (issued > s) {
+                    const long long uses = (issued - 1 - s) / kStages + 1;
+                    mbar_wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------- MMA issuer
+            constexpr uint32_t idesc = make_idesc(1u, kBM, 2 * kBN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sw128_kmajor_desc(sa + stage * kABytes);
+                    const uint64_t bdesc = sw128_kmajor_desc(sb + stage * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        // +32 bytes along K inside the swizzled row = +2 in the
+                        // descriptor's start-address field.
+                        mma_f16(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc,
+                                (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_empty + 8 * stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (failed) break;
+                mma_commit(bar_tfull + 8 * acc);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // Every MMA issued here must finish before TMEM is released.
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------- epilogue
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may read
+        const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t buf = se + static_cast<uint32_t>(warp - 2) * kEpiBufBytes;
+        const uint32_t swz = static_cast<uint32_t>(lane & 7);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            int mt, nt;
+            tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+            const int m0 = mt * kBM, n0 = nt * kBN;
+            if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kAccCols);
+#pragma unroll 1
+            for (int c = 0; c < kBN / 64; ++c) {
+                // The previous store from this buffer must have read it.
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t g[32], u[32];
+                    const uint32_t col = static_cast<uint32_t>(c * 64 + h * 32);
+                    tmem_ld_32x32b_x32(tacc + col, g);
+                    tmem_ld_32x32b_x32(tacc + kBN + col, u);
+                    tmem_ld_wait(g);
+                    tmem_ld_wait(u);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 v;
+                        v.x = pack_bf16x2(silu_mul_fast(g[8 * j + 0], u[8 * j + 0]),
+                                          silu_mul_fast(g[8 * j + 1], u[8 * j + 1]));
+                        v.y = pack_bf16x2(silu_mul_fast(g[8 * j + 2], u[8 * j + 2]),
+                                          silu_mul_fast(g[8 * j + 3], u[8 * j + 3]));
+                        v.z = pack_bf16x2(silu_mul_fast(g[8 * j + 4], u[8 * j + 4]),
+                                          silu_mul_fast(g[8 * j + 5], u[8 * j + 5]));
+                        v.w = pack_bf16x2(silu_mul_fast(g[8 * j + 6], u[8 * j + 6]),
+                                          silu_mul_fast(g[8 * j + 7], u[8 * j + 7]));
+                        // 16-byte chunk (h*4 + j) of this lane's 128-byte row,
+                        // placed where the TMA 128-byte swizzle expects it.
+                        const uint32_t chunk = static_cast<uint32_t>(h * 4 + j);
+                        sts_v4(buf + static_cast<uint32_t>(lane) * 128u + ((chunk ^ swz) << 4), v);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = n0 + c * 64;
+                    const int y = m0 + quad * 32;
+                    if (x < N && y < M) {
+                        tma_store_2d(&tm_h, buf, x, y);
+                        bulk_commit();
+                    }
+                }
+            }
+            // All tcgen05.ld of this buffer have completed (waited above).
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) bulk_wait<0>();
+    }
+
+    if (failed) atomicOr(&g_gemm_bf16_status, 1u);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        __syncwarp();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+std::atomic<unsigned> g_attr_set_mask{0};
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
+                             int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
+    CUtensorMap tx, twg, twu, th;
+    const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!encode_tmap_2d(&tx, X, bf16, K, M, static_cast<uint64_t>(K) * 2, kBK, kBM, sw) ||
+        !encode_tmap_2d(&twg, Wg, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
+        !encode_tmap_2d(&twu, Wu, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
+        !encode_tmap_2d(&th, H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32, sw)) {
+        return cudaErrorInvalidValue;
+    }
+    const unsigned bit = 1u << (dev.device & 31);
+    if (!(g_attr_set_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bf16_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        g_attr_set_mask.fetch_or(bit);
+    }
+    const int num_m = (M + kBM - 1) / kBM;
+    const int num_n = (N + kBN - 1) / kBN;
+    const long long tiles = static_cast<long long>(num_m) * num_n;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    swiglu_gemm_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tx, twg, twu, th, M, N, K,
+                                                                   num_m, num_n);
+    return cudaGetLastError();
+}
+
+cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host_out, g_gemm_bf16_status, sizeof(unsigned int),
+                                              0, cudaMemcpyDeviceToHost, stream);
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_gemm_bf16_status, &zero, sizeof(unsigned int), 0,
+                                cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
+}
+
+}  // namespace swiglu

@@ -1,0 +1,397 @@
+// gemm_tf32x3.cu -- fused SwiGLU dual GEMM for fp32 inputs, near-IEEE
+// accuracy on the tensor cores by 3xTF32 splitting, sm_100a.
+//
+// Why: Liger-Kernel issue #1383 ("[RFC] Testing Methodology for FP32
+// Convergence Tests ...", Root Cause) shows a fused gate/up kernel whose fp32
+// matmuls ran on the TF32 tensor-core path failing fp32 parity, while forcing
+// IEEE FMA overflowed shared memory.  Here every fp32 operand is split
+//     a = hi + lo,   hi = rna_tf32(a),   lo = rna_tf32(a - hi)
+// and each product is formed as hi*hi + hi*lo + lo*hi (the lo*lo term, below
+// 2^-22 relative, is dropped), all accumulated in fp32 in tensor memory.
+// This is the split-precision refinement of Markidis et al. (2018, "NVIDIA
+// Tensor Core Programmability, Performance & Precision") in the error-
+// corrected TF32 form of Ootomo & Yokota (2022, "Recovering single precision
+// accuracy from Tensor Cores while surpassing the FP32 theoretical peak
+// performance"), written here from the mathematics.
+//
+// Structure (one CTA per SM, persistent over 128 x 128 output tiles):
+//  * warp 0 (one thread): TMA producer -- raw fp32 X [128 x 16] and the
+//    stacked [Wg; Wu] tile [256 x 16] per 16-deep k-block, 64-byte swizzle,
+//    into a 4-stage ring;
+//  * warps 2..5: split -- each raw stage is rewritten in place as hi and a
+//    lo copy is written to a parallel buffer with the same (swizzled) layout;
+//  * warp 1 (one thread): MMA issuer -- per 8-deep step three
+//    tcgen05.mma kind::tf32 (M=128, N=256): Xhi*[Wg;Wu]hi, Xhi*[Wg;Wu]lo,
+//    Xlo*[Wg;Wu]hi into a double-buffered accumulator (gate columns 0..127,
+//    up columns 128..255);
+//  * warps 6..9: epilogue -- h = g * sigmoid(g) * u in fp32 with expf and
+//    IEEE division, fp32 result staged (128-byte swizzle) and stored by TMA.
+// All waits are bounded as in the bf16 kernel.
+#include <atomic>
+
+#include "gemm_common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace swiglu {
+
+// Status word of this translation unit's kernel (bit 0 = a wait gave up).
+__device__ unsigned int g_gemm_tf32x3_status;
+
+namespace {
+
+using namespace dev;
+using gemm::mbar_wait_drain;
+using gemm::tile_coords;
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;                 // H columns per tile (gate, up each)
+constexpr int kBK = 16;                  // fp32 k per stage: one 64-byte row
+constexpr int kStages = 4;
+constexpr int kUmmaK = 8;                // k per tcgen05.mma, kind::tf32
+constexpr int kAccCols = 2 * kBN;
+constexpr int kTmemCols = 2 * kAccCols;  // 512
+constexpr int kSplitWarps = 4;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * (kSplitWarps + kEpiWarps);  // 320
+constexpr int kFirstSplitWarp = 2;
+constexpr int kFirstEpiWarp = kFirstSplitWarp + kSplitWarps;   // 6
+
+constexpr uint32_t kABytes = kBM * kBK * 4;            // 8 KB
+constexpr uint32_t kBBytes = 2 * kBN * kBK * 4;        // 16 KB: Wg rows, Wu rows
+constexpr uint32_t kRawBytes = kABytes + kBBytes;      // 24 KB loaded per stage
+constexpr uint32_t kStageBytes = 2 * kRawBytes;        // + lo copies
+constexpr uint32_t kEpiBufBytes = 32 * 128;            // 32 rows x 32 fp32
+// Per stage: [A hi | B hi | A lo | B lo]; the hi half is what TMA loads.
+constexpr uint32_t kOffStages = 0;
+constexpr uint32_t kOffEpi = kOffStages + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
+constexpr uint32_t kNumBars = 3 * kStages + 2 + 2 + 1;  // full, ready, empty, tfull, tempty, drain
+constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
+constexpr uint32_t kSmemUsed = kOffAbort + 8;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
+
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// Split 4 fp32 values in place: returns hi in `v`, lo in `lo`.
+__device__ __forceinline__ void split4(uint4 &v, uint4 &lo) {
+    uint32_t *pv = &v.x, *pl = &lo.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(pv[i]);
+        const uint32_t hi = tf32_rna(a);
+        pl[i] = tf32_rna(a - __uint_as_float(hi));
+        pv[i] = hi;
+    }
+}
+
+// h = silu(g) * u in fp32: sigmoid from t = exp(-|g|) without cancellation,
+// expf and an IEEE division (a few ulp in total).
+__device__ __forceinline__ float silu_mul_accurate(uint32_t gbits, uint32_t ubits) {
+    const float g = __uint_as_float(gbits);
+    const float u = __uint_as_float(ubits);
+    const float t = expf(-fabsf(g));
+    const float r = 1.0f / (1.0f + t);
+    const float s = g >= 0.0f ? r : t * r;
+    return g * s * u;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    swiglu_gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_x,
+                              const __grid_constant__ CUtensorMap tm_wg,
+                              const __grid_constant__ CUtensorMap tm_wu,
+                              const __grid_constant__ CUtensorMap tm_h, int M, int N, int K,
+                              int num_m_tiles, int num_n_tiles) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+
+    const uint32_t sst = base + kOffStages;
+    const uint32_t se = base + kOffEpi;
+    const uint32_t bar_full = base + kOffBar;
+    const uint32_t bar_ready = bar_full + 8 * kStages;
+    const uint32_t bar_empty = bar_ready + 8 * kStages;
+    const uint32_t bar_tfull = bar_empty + 8 * kStages;
+    const uint32_t bar_tempty = bar_tfull + 16;
+    const uint32_t bar_drain = bar_tempty + 16;
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + kOffTmemPtr);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int num_tiles = num_m_tiles * num_n_tiles;
+    const int num_kb = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_ready + 8 * s, kSplitWarps);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, kEpiWarps);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_wg);
+        tma_prefetch_desc(&tm_wu);
+        tma_prefetch_desc(&tm_h);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
+
+    bool failed = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+                const int m0 = mt * kBM, n0 = nt * kBN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t st = sst + stage * kStageBytes;
+                    mbar_arrive_expect_tx(fb, kRawBytes);
+                    tma_load_2d(&tm_x, fb, st, kb * kBK, m0);
+                    tma_load_2d(&tm_wg, fb, st + kABytes, kb * kBK, n0);
+                    tma_load_2d(&tm_wu, fb, st + kABytes + kBBytes / 2, kb * kBK, n0);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < kStages; ++s) {
+                if (issued > s) {
+                    const long long uses = (issued - 1 - s) / kStages + 1;
+                    mbar_wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------- MMA issuer
+            constexpr uint32_t idesc = make_idesc(2u, kBM, 2 * kBN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar_ready + 8 * stage, phase, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = sst + stage * kStageBytes;
+                    const uint64_t a_hi = sw64_kmajor_desc(st);
+                    const uint64_t b_hi = sw64_kmajor_desc(st + kABytes);
+                    const uint64_t a_lo = sw64_kmajor_desc(st + kRawBytes);
+                    const uint64_t b_lo = sw64_kmajor_desc(st + kRawBytes + kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        // +32 bytes along K inside the 64-byte swizzled row.
+                        const uint32_t o = 2u * kk;
+                        const uint32_t first = (kb == 0 && kk == 0) ? 0u : 1u;
+                        mma_tf32(d_tmem, a_lo + o, b_hi + o, idesc, first);
+                        mma_tf32(d_tmem, a_hi + o, b_lo + o, idesc, 1u);
+                        mma_tf32(d_tmem, a_hi + o, b_hi + o, idesc, 1u);
+                    }
+                    mma_commit(bar_empty + 8 * stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (failed) break;
+                mma_commit(bar_tfull + 8 * acc);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else if (warp < kFirstEpiWarp) {
+        // ---------------------------------------------------- hi/lo split
+        const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
+        constexpr int kVecs = kRawBytes / 16;                  // 1536 per stage
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t st = sst + stage * kStageBytes;
+#pragma unroll 4
+                for (int v = sidx; v < kVecs; v += 32 * kSplitWarps) {
+                    uint4 x = lds_v4(st + 16u * v);
+                    uint4 lo;
+                    split4(x, lo);
+                    sts_v4(st + 16u * v, x);
+                    sts_v4(st + kRawBytes + 16u * v, lo);
+                }
+                // make the generic-proxy writes visible to the tensor cores
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_ready + 8 * stage);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t buf = se + static_cast<uint32_t>(warp - kFirstEpiWarp) * kEpiBufBytes;
+        const uint32_t swz = static_cast<uint32_t>(lane & 7);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            int mt, nt;
+            tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+            const int m0 = mt * kBM, n0 = nt * kBN;
+            if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kAccCols);
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+                uint32_t g[32], u[32];
+                tmem_ld_32x32b_x32(tacc + 32u * c, g);
+                tmem_ld_32x32b_x32(tacc + kBN + 32u * c, u);
+                tmem_ld_wait(g);
+                tmem_ld_wait(u);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 v;
+                    v.x = __float_as_uint(silu_mul_accurate(g[4 * j + 0], u[4 * j + 0]));
+                    v.y = __float_as_uint(silu_mul_accurate(g[4 * j + 1], u[4 * j + 1]));
+                    v.z = __float_as_uint(silu_mul_accurate(g[4 * j + 2], u[4 * j + 2]));
+                    v.w = __float_as_uint(silu_mul_accurate(g[4 * j + 3], u[4 * j + 3]));
+                    sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
+                               ((static_cast<uint32_t>(j) ^ swz) << 4),
+                           v);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = n0 + c * 32;
+                    const int y = m0 + quad * 32;
+                    if (x < N && y < M) {
+                        tma_store_2d(&tm_h, buf, x, y);
+                        bulk_commit();
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) bulk_wait<0>();
+    }
+
+    if (failed) atomicOr(&g_gemm_tf32x3_status, 1u);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        __syncwarp();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+std::atomic<unsigned> g_attr_set_mask{0};
+
+}  // namespace
+
+cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, void *H, int M,
+                               int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
+    CUtensorMap tx, twg, twu, th;
+    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!encode_tmap_2d(&tx, X, f32, K, M, static_cast<uint64_t>(K) * 4, kBK, kBM, sw64) ||
+        !encode_tmap_2d(&twg, Wg, f32, K, N, static_cast<uint64_t>(K) * 4, kBK, kBN, sw64) ||
+        !encode_tmap_2d(&twu, Wu, f32, K, N, static_cast<uint64_t>(K) * 4, kBK, kBN, sw64) ||
+        !encode_tmap_2d(&th, H, f32, N, M, static_cast<uint64_t>(N) * 4, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) {
+        return cudaErrorInvalidValue;
+    }
+    const unsigned bit = 1u << (dev.device & 31);
+    if (!(g_attr_set_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_tf32x3_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        g_attr_set_mask.fetch_or(bit);
+    }
+    const int num_m = (M + kBM - 1) / kBM;
+    const int num_n = (N + kBN - 1) / kBN;
+    const long long tiles = static_cast<long long>(num_m) * num_n;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    swiglu_gemm_tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tx, twg, twu, th, M, N, K,
+                                                                     num_m, num_n);
+    return cudaGetLastError();
+}
+
+cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host_out, g_gemm_tf32x3_status,
+                                              sizeof(unsigned int), 0, cudaMemcpyDeviceToHost,
+                                              stream);
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_gemm_tf32x3_status, &zero, sizeof(unsigned int), 0,
+                                cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
+}
+
+}  // namespace swiglu

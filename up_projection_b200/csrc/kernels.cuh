@@ -1,0 +1,56 @@
+// kernels.cuh -- internal launcher interface between the C ABI (api.cu) and
+// the kernel translation units.  Every launcher only enqueues work on
+// `stream` and returns the launch's cudaError_t; arguments are validated by
+// the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace swiglu {
+
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int cc_major;
+    int cc_minor;
+    int max_smem_optin;  // bytes of dynamic shared memory a block may opt into
+};
+
+// bf16 forward, tcgen05 dual GEMM (any M >= 1, K >= 1, N >= 1).
+cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void *H,
+                             int M, int K, int N, const DeviceInfo &dev,
+                             cudaStream_t stream);
+
+// fp32 forward, 3xTF32 tcgen05 dual GEMM.
+cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, void *H,
+                               int M, int K, int N, const DeviceInfo &dev,
+                               cudaStream_t stream);
+
+// bf16 forward for M <= 8: weight streaming with tensor-core dot products.
+// decode_bf16_supported: whether K fits the kernel's shared-memory X stage
+// (a pure function of K; larger K routes to the dual GEMM).
+bool decode_bf16_supported(int K);
+cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H,
+                               int M, int K, int N, const DeviceInfo &dev,
+                               cudaStream_t stream);
+
+// Elementwise dSwiGLU; dtype 0 = bf16, 1 = fp32.
+cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG,
+                           void *dU, int64_t n, int dtype, const DeviceInfo &dev,
+                           cudaStream_t stream);
+
+// Pure streaming read of two buffers (bench-only floor probe).
+int read_floor_grid(const DeviceInfo &dev);
+cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
+                              const DeviceInfo &dev, cudaStream_t stream);
+
+// Device status words of the GEMM kernels (bounded waits that gave up): read
+// one into *host_out, reset it, and wait for the stream.
+cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+
+// Tensor-map encoding through the driver entry point (no libcuda link).
+bool tensor_maps_available();
+
+}  // namespace swiglu
