@@ -1,0 +1,548 @@
+"""Benchmark of the fused SwiGLU gate/up projection on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-extra]
+
+Headline workload (one "step"): decode at the AstrAI-1B MLP shape
+(K = 1536, N = 6912), one fused call at each M in {1, 2, 4, 8}, every call on
+the next of 16 rotated weight copies (680 MB, > 5x the 126 MB L2), so every
+call streams its weights cold from HBM -- the cold-weight protocol of
+AstrAI swiglu_benchmark.md ("HBM re-measurement and kernel simplification").
+Metric: algorithmic bytes (Wg + Wu + X + H) / device time, GB/s.
+
+Also measured (key "also", not part of the step): prefill at the LLaMA-3 8B
+shape (TFLOP/s), dSwiGLU on [8192, 14336] bf16 (GB/s), the fp32 3xTF32 mode
+at the LLaMA-2 13B and GPT-NeoX 20B shapes (TFLOP/s), and the LLaMA-2 7B
+decode shape (GB/s), each with its roofline fraction.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and cuda synchronize, CUDA events on the launching stream, max over ranks.
+The step is replayed from CUDA graphs (one per group of 4 rotated copies) so
+host launch overhead does not starve the GPU.  Multi-GPU (torchrun): every
+rank runs the same per-GPU workload on its own GPU (independent problems, no
+data-path collective): weak scaling, value = all ranks' bytes / max time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference
+implementation of this op here) on a bounded sample of the same workload, on
+the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# Page figure for this exact metric and shape: the fused decode kernel's
+# cold-weight bandwidth at (N, K) = (6912, 1536) on an L20 (sm_89) -- AstrAI
+# swiglu_benchmark.md, "HBM re-measurement and kernel simplification".
+# Another machine's number: context for vs_baseline, not the target.
+PAGE_DECODE_GBS = 702.0
+
+DECODE_SHAPE = (1536, 6912)
+DECODE_MS = (1, 2, 4, 8)
+DECODE_COPIES = 16
+
+# DRAM traffic of the decode kernel per launch from one ncu capture, keyed by
+# the sha256 of the kernel source it was measured on; reported as null when
+# the source has changed since.
+DECODE_TRAFFIC = {"src_sha256": None, "bytes_per_launch_by_M": {}}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def decode_bytes(M, K, N, elem=2):
+    """Algorithmic bytes of one fused call: both weight matrices once, X in,
+    H out."""
+    return elem * (2 * N * K + M * K + M * N)
+
+
+def src_sha(name):
+    path = os.path.join(ROOT, "up_projection_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"swiglu_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r[0] for r in rows if r[2] > 300.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    from up_projection_b200.parallel import max_over_ranks as mor
+    return mor(x) if world > 1 else x
+
+
+# -------------------------------------------------------------- our arm
+
+def timed_events(fn, iters, stream):
+    """Run fn() iters times between two CUDA events on `stream`; returns ms."""
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(iters):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def decode_workload(K, N, Ms, copies, seed=0):
+    """Rotated weight copies (distinct buffers, same values) and X per M."""
+    from up_projection_b200 import synth
+    X8, Wg, Wu = synth.swiglu_inputs(max(Ms), K, N, "bf16", seed=seed)
+    dev = torch.device("cuda")
+    Wg_all = torch.empty((copies, N, K), dtype=torch.bfloat16, device=dev)
+    Wu_all = torch.empty_like(Wg_all)
+    Wg_all[:] = Wg.to(dev)
+    Wu_all[:] = Wu.to(dev)
+    Xs = {M: X8[:M].contiguous() for M in Ms}
+    return Xs, Wg_all, Wu_all
+
+
+def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
+    import up_projection_b200 as up
+    Xs_host, Wg_all, Wu_all = decode_workload(K, N, Ms, copies)
+    dev = torch.device("cuda")
+    Xd = {M: Xs_host[M].to(dev) for M in Ms}
+    Hd = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
+    per_step = len(Ms)
+    groups = copies // per_step   # one graph per group of per_step copies
+
+    def step_calls(g):
+        for i, M in enumerate(Ms):
+            c = g * per_step + i
+            up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream)
+
+    # eager warm-up (tensor maps, function attributes), then capture
+    with torch.cuda.stream(stream):
+        for g in range(groups):
+            step_calls(g)
+    torch.cuda.synchronize()
+    assert up.swiglu_sync_status(stream) == 0
+    graphs = []
+    for g in range(groups):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            step_calls(g)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+
+    state = {"i": 0}
+
+    def one_step():
+        graphs[state["i"] % groups].replay()
+        state["i"] += 1
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(torch.cuda.current_device())
+    with ClockSampler(gpu_id) as clk:
+        with torch.cuda.stream(stream):
+            ms = timed_events(one_step, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    st = up.swiglu_sync_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after decode: {up.status_string(st)}")
+    ms_max = max_over_ranks(ms, world)
+    step_bytes = sum(decode_bytes(M, K, N) for M in Ms)
+    out = {"ms": ms_max, "step_bytes": step_bytes, "clocks": clk.summary(),
+           "launches": args.steps * per_step}
+
+    # per-M launch time (eager, each M alone on rotated copies) for the record
+    per_m = {}
+    with torch.cuda.stream(stream):
+        for M in Ms:
+            j = {"c": 0}
+
+            def call():
+                c = j["c"] % copies
+                up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream)
+                j["c"] += 1
+            gr = torch.cuda.CUDAGraph()
+            # a graph of one full rotation of this M alone
+            with torch.cuda.graph(gr, stream=stream):
+                for _ in range(copies):
+                    call()
+            reps = min(500, max(1, 4 * args.steps // copies))
+            for _ in range(2):
+                gr.replay()
+            t = timed_events(gr.replay, reps, stream) / (reps * copies)
+            per_m[M] = {"us": t * 1e3, "GB/s": decode_bytes(M, K, N) / (t * 1e-3) / 1e9}
+            del gr
+    out["per_M"] = per_m
+
+    if with_e2e:
+        # Through the public API with host buffers: pinned X in, H out, every
+        # call, inside the timed region.
+        Xp = {M: Xs_host[M].pin_memory() for M in Ms}
+        Hp = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+        h2d = sum(Xp[M].numel() * 2 for M in Ms)
+        d2h = sum(Hp[M].numel() * 2 for M in Ms)
+        cnt = {"c": 0}
+
+        def e2e_step():
+            for M in Ms:
+                c = cnt["c"] % copies
+                Xd[M].copy_(Xp[M], non_blocking=True)
+                up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream)
+                Hp[M].copy_(Hd[M], non_blocking=True)
+                cnt["c"] += 1
+        e_steps = min(args.steps, 2000)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                e2e_step()
+            torch.cuda.synchronize()
+            barrier(world)
+            e_ms = timed_events(e2e_step, e_steps, stream)
+        barrier(world)
+        e_ms = max_over_ranks(e_ms, world)
+        out["e2e"] = {"ms": e_ms, "steps": e_steps, "h2d": h2d, "d2h": d2h}
+    for g in graphs:
+        del g
+    del Wg_all, Wu_all
+    torch.cuda.empty_cache()
+    return out
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def run_extras(stream, pk):
+    """Single-GPU extra measurements (rank 0 only)."""
+    import up_projection_b200 as up
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    res = []
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def time_op(fn, iters=10):
+        # inputs are larger than L2 in every case below; L2 is also flushed
+        # between timed calls (flush not timed)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            tot = 0.0
+            for _ in range(iters):
+                flush_l2(flush)
+                tot += timed_events(fn, 1, stream)
+        return tot / iters
+
+    # prefill LLaMA-3 8B
+    M, K, N = 8192, 4096, 14336
+    X = torch.randn((M, K), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    Wg = (torch.randn((N, K), generator=gen, device=dev) / K ** 0.5).to(torch.bfloat16)
+    Wu = (torch.randn((N, K), generator=gen, device=dev) / K ** 0.5).to(torch.bfloat16)
+    H = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ms = time_op(lambda: up.swiglu_fwd(X, Wg, Wu, H, stream=stream))
+    fl = 4.0 * M * N * K
+    tf = fl / (ms * 1e-3) / 1e12
+    res.append({"workload": "prefill LLaMA-3 8B M=8192 K=4096 N=14336 bf16",
+                "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(tf / pk["bf16_tflops"], 4)}})
+    del X, Wg, Wu, H
+    # dSwiGLU on [8192, 14336] bf16
+    n = 8192 * 14336
+    dH = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)
+    G = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)
+    U = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)
+    dG = torch.empty_like(G)
+    dU = torch.empty_like(U)
+    ms = time_op(lambda: up.dswiglu_bwd(dH, G, U, dG, dU, stream=stream))
+    gbs = 10.0 * n / (ms * 1e-3) / 1e9
+    res.append({"workload": "dSwiGLU n=8192*14336 bf16", "metric": "GB/s", "value": round(gbs, 1),
+                "ms": round(ms, 4),
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4)}})
+    del dH, G, U, dG, dU
+    # fp32 3xTF32 at the 13B and NeoX-20B shapes
+    for K, N, name in ((5120, 13824, "LLaMA-2 13B"), (6144, 24576, "GPT-NeoX 20B")):
+        M = 2048
+        X = torch.randn((M, K), generator=gen, device=dev)
+        Wg = torch.randn((N, K), generator=gen, device=dev) / K ** 0.5
+        Wu = torch.randn((N, K), generator=gen, device=dev) / K ** 0.5
+        H = torch.empty((M, N), dtype=torch.float32, device=dev)
+        try:
+            ms = time_op(lambda: up.swiglu_fwd(X, Wg, Wu, H, stream=stream), iters=5)
+        except Exception as exc:  # noqa: BLE001 - report, do not hide
+            res.append({"workload": f"fp32 3xTF32 {name}", "error": str(exc)})
+            continue
+        fl = 4.0 * M * N * K
+        tf = fl / (ms * 1e-3) / 1e12
+        tf32_peak = pk["bf16_tflops"] * 0.5   # nominal dense TF32/BF16 ratio
+        res.append({"workload": f"fp32 3xTF32 {name} M=2048 K={K} N={N}",
+                    "metric": "TFLOP/s (fp32-equivalent)", "value": round(tf, 1),
+                    "ms": round(ms, 4),
+                    "roofline": {"bound": "tensor", "achieved": round(3 * tf, 1),
+                                 "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32 MMA)",
+                                 "frac": round(3 * tf / tf32_peak, 4),
+                                 "frac_vs_bf16_peak_literal": round(tf / pk["bf16_tflops"], 4)}})
+        del X, Wg, Wu, H
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline_decode(K, N, Ms, budget_s=12.0):
+    """Time the fp64 oracle (as it stands) on the decode step, bounded."""
+    import oracle
+    from up_projection_b200 import synth
+    X8, Wg, Wu = synth.swiglu_inputs(max(Ms), K, N, "bf16", seed=0)
+    Xd = oracle.decode_bf16(X8)
+    Wgd = oracle.decode_bf16(Wg)
+    Wud = oracle.decode_bf16(Wu)
+    o = oracle.default()
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        for M in Ms:
+            o.swiglu_fwd_f64(Xd[:M], Wgd, Wud)
+        steps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    step_bytes = sum(decode_bytes(M, K, N) for M in Ms)
+    threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    return {"value": round(step_bytes * steps / dt / 1e9, 4), "unit": "GB/s",
+            "cores": min(threads, max(Ms)), "kind": "oracle",
+            "sample": f"{steps} full decode steps (M=1,2,4,8 at K={K}, N={N}), fp64 C loops, "
+                      f"OpenMP over output rows ({threads} threads available), {dt:.1f} s"}
+
+
+def reference_arm(args, metric, config, K, N, budget_s=120.0):
+    """The fp64 CPU oracle on the host cores, on a bounded sample of the decode
+    step: the step's four calls restricted to the first N' output columns,
+    N' chosen so that warm-up plus all timed steps take about budget_s."""
+    import oracle
+    from up_projection_b200 import synth
+    X8, Wg, Wu = synth.swiglu_inputs(max(DECODE_MS), K, N, "bf16", seed=0)
+    o = oracle.default()
+    Xd, Wgd, Wud = o.decode_bf16(X8), o.decode_bf16(Wg), o.decode_bf16(Wu)
+    t0 = time.perf_counter()
+    for M in DECODE_MS:
+        o.swiglu_fwd_f64(Xd[:M], Wgd, Wud)
+    t_full = time.perf_counter() - t0
+    frac = min(1.0, budget_s / (t_full * (args.steps + args.warmup)))
+    n_s = max(8, int(N * frac) // 8 * 8)
+    Wgs, Wus = Wgd[:n_s], Wud[:n_s]
+
+    def step():
+        for M in DECODE_MS:
+            o.swiglu_fwd_f64(Xd[:M], Wgs, Wus)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    step_bytes = sum(decode_bytes(M, K, n_s) for M in DECODE_MS)
+    value = step_bytes * args.steps / dt / 1e9
+    threads = len(os.sched_getaffinity(0))
+    sample = (f"each step: the four decode calls (M=1,2,4,8, K={K}) on the first {n_s} of "
+              f"{N} output columns; fp64 C oracle, OpenMP over output rows")
+    line = {"impl": "reference", "metric": metric, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config,
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                             "cores": min(threads, max(DECODE_MS)), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 'also' measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    K, N = DECODE_SHAPE
+    metric = "SwiGLU gate/up: decode cold-weight GB/s, prefill TFLOP/s, % of roofline"
+    config = {"workload": f"decode AstrAI-1B: M in {{1,2,4,8}}, K={K}, N={N}, bf16, "
+                          f"{DECODE_COPIES} rotated weight copies",
+              "global_batch": sum(DECODE_MS) * args.gpus, "seq_len": 1,
+              "parallelism": f"independent replicas x{args.gpus} (no collective)",
+              "l2": f"inputs larger than L2 ({DECODE_COPIES} rotated copies, "
+                    f"{DECODE_COPIES * 4 * N * K / 1e6:.0f} MB)"}
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        return reference_arm(args, metric, config, K, N)
+
+    rank, world, local = dist_setup(args.gpus)
+    import up_projection_b200 as up
+    up.lib()  # fail loudly now if the CUDA library is missing
+    pk = peaks()
+    stream = torch.cuda.Stream()
+    dec = run_decode(args, world, K, N, DECODE_MS, DECODE_COPIES, stream, with_e2e=True)
+    total_bytes = dec["step_bytes"] * args.steps * world
+    value = total_bytes / (dec["ms"] * 1e-3) / 1e9
+    # dominant kernel: the decode kernel; average launch = timed region / launches
+    per_launch_ms = dec["ms"] / dec["launches"]
+    per_launch_bytes = dec["step_bytes"] / len(DECODE_MS)
+    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+    sha = src_sha("decode_bf16.cu")
+    traffic = None
+    if DECODE_TRAFFIC["src_sha256"] == sha and DECODE_TRAFFIC["bytes_per_launch_by_M"]:
+        vals = DECODE_TRAFFIC["bytes_per_launch_by_M"]
+        traffic = sum(vals[str(M)] for M in DECODE_MS) / len(DECODE_MS)
+    line = {
+        "metric": metric, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dec["ms"] / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": round(value / world / PAGE_DECODE_GBS, 3),
+        "dtype": "bf16", "data": "synthetic", "config": config,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                     "traffic": traffic, "peak_source": pk["source"],
+                     "kernel": "swiglu_decode_bf16_kernel",
+                     "launch_time": "timed region / launches (graph replay)"},
+        "per_M": {str(M): {k: round(v, 2) for k, v in d.items()} for M, d in dec["per_M"].items()},
+        "e2e": {"value": round(dec["step_bytes"] * dec["e2e"]["steps"] * world
+                               / (dec["e2e"]["ms"] * 1e-3) / 1e9, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
+                "d2h_bytes_per_step": dec["e2e"]["d2h"]},
+        "gpu_launches": dec["launches"],
+        "clocks": dec["clocks"],
+    }
+    if rank == 0 and not args.no_extra:
+        line["also"] = run_extras(stream, pk)
+        # LLaMA-2 7B decode shape as a second cold-weight line
+        s7 = max(40, min(2000, args.steps // 4))
+        d7 = run_decode(argparse.Namespace(steps=s7, warmup=5), 1,
+                        4096, 11008, DECODE_MS, 8, stream, with_e2e=False)
+        v7 = d7["step_bytes"] * s7 / (d7["ms"] * 1e-3) / 1e9
+        line["also"].append({"workload": "decode LLaMA-2 7B: M in {1,2,4,8}, K=4096, N=11008, "
+                                         "8 rotated copies (1.44 GB)",
+                             "metric": "GB/s", "value": round(v7, 1),
+                             "per_M": {str(M): {k: round(v, 2) for k, v in d.items()}
+                                       for M, d in d7["per_M"].items()},
+                             "roofline": {"bound": "hbm", "achieved": round(v7, 1),
+                                          "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                          "frac": round(v7 / pk["hbm_gbs"], 4)}})
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline_decode(K, N, DECODE_MS)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,89 @@
+"""fp32-input mode (3xTF32 tcgen05 dual GEMM) vs the fp64 oracle.
+
+Bound per element (the pages' fp32 target is 1e-5 relative; a pure relative
+error is ill-posed where H ~ 0, so it is taken relative to the magnitude of
+the terms before cancellation):
+    |gpu - ref| <= 1e-5 * (|H| + |silu(G)| * sum_k|x wu| + |U| * |silu'(G)| * sum_k|x wg|)
+test_fp32_tolerance.py (CPU) shows this bound rejects plain TF32."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import FP32_FWD_TOL, assert_guards_intact, assert_within, f64, guarded_empty, \
+    sample_indices, to_dev
+from up_projection_b200 import _capi, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def fp32_bound(G, U, H, AG, AU):
+    s = 1.0 / (1.0 + np.exp(-np.clip(G, -700, 700)))
+    silu = G * s
+    dsilu = s * (1.0 + G * (1.0 - s))
+    return FP32_FWD_TOL * (np.abs(H) + np.abs(silu) * AU + np.abs(U) * np.abs(dsilu) * AG) + 1e-30
+
+
+def run(X, Wg, Wu):
+    M, K = X.shape
+    N = Wg.shape[0]
+    Xd, Wgd, Wud = to_dev(X, Wg, Wu)
+    full, H = guarded_empty(M * N, torch.float32)
+    _capi.swiglu_fwd(Xd, Wgd, Wud, H.view(M, N))
+    st = _capi.swiglu_sync_status()
+    assert st == 0, _capi.status_string(st)
+    assert _capi.swiglu_last_route() == _capi.ROUTE_GEMM_TF32X3
+    assert_guards_intact(full)
+    return H.view(M, N).cpu()
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (4, 256, 512),      # tiny shape in fp32 (M <= 8 also takes the GEMM)
+    (128, 16, 128),     # one tile, one k-block
+    (128, 32, 256),
+    (129, 36, 132),     # ragged M, K (not a multiple of 16), N
+    (300, 520, 392),
+    (256, 2048, 256),   # long K
+])
+def test_fp32_small(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=M + K)
+    H = run(X, Wg, Wu)
+    ref = oracle.swiglu_fwd(X, Wg, Wu, "f32", want_magnitudes=True)
+    assert_within(np.abs(f64(H) - ref["H"]),
+                  fp32_bound(ref["G"], ref["U"], ref["H"], ref["AG"], ref["AU"]),
+                  f"fp32 M={M} K={K} N={N}")
+
+
+def test_fp32_integer_exact():
+    """Small integers are exact in TF32 (lo = 0); gate >= 17 makes sigmoid 1
+    in fp32, so H must equal fp32(G * U) bit for bit."""
+    M, K, N = 130, 64, 136
+    X, Wg, Wu = synth.integer_inputs(M, K, N, seed=3, dtype="f32")
+    H = run(X, Wg, Wu)
+    G = X.double() @ Wg.double().T
+    U = X.double() @ Wu.double().T
+    assert float(G.min()) >= 17.0
+    expect = (G * U).float()
+    assert torch.equal(H.view(torch.int32), expect.view(torch.int32))
+
+
+@pytest.mark.parametrize("K,N", [(5120, 13824), (6144, 24576)])
+def test_fp32_full_size_sampled(K, N):
+    """LLaMA-2 13B and GPT-NeoX 20B shapes at M = 2048 (the bench launch)."""
+    M = 2048
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=K)
+    H = run(X, Wg, Wu)
+    im, inn = sample_indices(M, N, 3000)
+    ref = oracle.swiglu_fwd_points(X, Wg, Wu, im, inn, "f32")
+    err = np.abs(f64(H[im, inn]) - ref["H"])
+    assert_within(err, fp32_bound(ref["G"], ref["U"], ref["H"], ref["AG"], ref["AU"]),
+                  f"fp32 full K={K} N={N}")
+    # For the record (not the bound): error relative to the bound's scale,
+    # norm-wise relative error, and plain relative error away from zero.
+    scale = fp32_bound(ref["G"], ref["U"], ref["H"], ref["AG"], ref["AU"]) / FP32_FWD_TOL
+    rms = np.sqrt(np.mean(ref["H"] ** 2))
+    away = np.abs(ref["H"]) > 0.1 * rms
+    print(f"fp32 K={K} N={N}: max err/scale {np.max(err / scale):.2e}, "
+          f"norm-wise {np.linalg.norm(err) / np.linalg.norm(ref['H']):.2e}, "
+          f"max rel where |H| > 0.1 rms {np.max(err[away] / np.abs(ref['H'][away])):.2e}")
+    assert np.linalg.norm(err) / np.linalg.norm(ref["H"]) < 1e-3

@@ -218,12 +218,14 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = decode_status_fetch_and_clear(&w3, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
 }
 
 SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes, void *sink,

@@ -1,59 +1,112 @@
 // decode_bf16.cu -- fused SwiGLU forward for decode-sized M (1..8), bf16.
 //
 // At M <= 8 the op is a pair of matrix-vector products: every byte of Wg and
-// Wu is used M times, so the time is the time to stream both weight matrices
-// from HBM once (AstrAI swiglu_benchmark.md, "HBM re-measurement and kernel
-// simplification": the fused kernel sits on the dual-stream cold-read
-// floor).  This kernel is built around that:
+// Wu is used at most 8 times, so the time is the time to stream both weight
+// matrices from HBM once (AstrAI swiglu_benchmark.md, "HBM re-measurement
+// and kernel simplification": the fused kernel sits on the dual-stream
+// cold-read floor).  The kernel is built to be that stream:
 //
-//  * a unit of work is 8 consecutive output columns n0..n0+7: 8 rows of Wg
-//    and the same 8 rows of Wu;
-//  * the 4 warps of a CTA split the unit's K range; each lane streams 16 B
-//    (8 bf16) of one Wg row and one Wu row per 32-wide k chunk with
-//    L1-bypassing 128-bit loads, keeping kPrefetch chunks in flight in
-//    registers (weights never touch shared memory);
-//  * the dot products run on the tensor cores as mma.sync m16n8k16: the
-//    16-row A operand is [8 Wg rows; 8 Wu rows], the 8-column B operand is
-//    X^T (rows of X beyond M are zero).  The k order inside each 16-wide
+//  * one CTA per SM; CTA b owns a contiguous, balanced range of units, a unit
+//    being 8 consecutive output columns n0..n0+7 (8 rows of Wg and the same 8
+//    rows of Wu).  Units of 8 rows keep the split across 148 SMs within a few
+//    percent of even at the decode shapes;
+//  * warp 0 (one thread) streams each unit in k-slices with ONE TMA tensor
+//    copy per weight matrix per stage: a 3-D view [N][K/inner][inner] of the
+//    weights lets one box cover 8 rows x kc columns (16-24 KB).  On B200 the
+//    per-SM cost of a bulk copy is nearly independent of its size up to tens
+//    of KB, so few large copies are what reaches HBM speed;
+//  * warps 1..4 split each slice's 32-wide k chunks and run the dot products
+//    on the tensor cores as mma.sync m16n8k16: A = [8 Wg rows; 8 Wu rows],
+//    B = X^T (rows of X beyond M are zero).  The k order inside each 16-wide
 //    step is permuted identically for A and B (a sum does not depend on the
-//    order of its terms) so that every lane feeds its A fragment directly
-//    from its own 16-byte load.  The accumulator then gives each lane both
-//    gate and up for (n0 + lane/4, m = 2*(lane%4) + {0,1}), so the SiLU-and-
-//    gate epilogue is lane-local;
+//    order of its terms) so each lane feeds its fragments from one 16-byte
+//    shared-memory read of each operand.  Each lane then holds gate and up
+//    for (n0 + lane/4, m = 2*(lane%4) + {0,1}), so the SiLU-and-gate
+//    epilogue is lane-local;
 //  * the four warps' fp32 partials are summed in shared memory in a fixed
-//    order (deterministic, no atomics), then h = silu(g) * u in fp32 and one
-//    RNE rounding to bf16.
+//    order (deterministic, no atomics); h = silu(g) * u in fp32, one RNE
+//    rounding to bf16.
 //
-// X [M, K] is staged once per CTA in shared memory (zero padded to 8 rows and
-// to a multiple of 32 columns, row pitch chosen so 8-lane phases of 16-byte
-// reads hit distinct banks).  The first unit's weight loads are issued before
-// X is staged, since they do not depend on it.
+// X [M, K] arrives by bulk copy while the first weight slices stream.  Waits
+// are bounded (ptx.cuh); a stuck pipeline sets the status word and the
+// kernel drains its copies and returns.
 #include <cuda_bf16.h>
 
 #include <atomic>
 
+#include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "tmap.cuh"
 
 namespace swiglu {
+
+// Status word of this translation unit's kernel (bit 0 = a wait gave up).
+__device__ unsigned int g_decode_status;
+
 namespace {
 
 using namespace dev;
+using gemm::mbar_wait_drain;
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kPrefetch = 8;  // 32-wide k chunks in flight per warp
-constexpr int kMaxSmem = 160 * 1024;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxStages = 4;
+constexpr int kSmemBudget = 220 * 1024;  // stages + X stage
+constexpr int kMaxSmem = 227 * 1024;     // B200 opt-in limit per block
+constexpr int kNumBars = 2 * kMaxStages + 4;  // full, empty, x, x_zero, red_full, red_empty
+constexpr int kRedBytes = kConsumerWarps * 32 * 4 * 4;
 
-__host__ __device__ inline int padded_k(int K) { return (K + 31) / 32 * 32; }
+struct Geometry {
+    int inner;    // innermost box extent (elements): largest of 256..8 dividing K
+    int slices;   // k-slices per unit
+    int kc;       // k elements per slice (multiple of inner)
+    int stages;   // ring depth
+    int kx;       // k elements per X row in shared memory (slices * kc >= K)
+    int off_x, off_red, off_bar, smem;
+    bool ok;
+};
 
-__host__ __device__ inline int x_pitch_bytes(int K) {
-    const int b = padded_k(K) * 2;  // a multiple of 64
-    return (b % 128 == 0) ? b + 64 : b;
-}
-
-__host__ __device__ inline int decode_smem_bytes(int K) {
-    return 8 * x_pitch_bytes(K) + kWarps * 32 * 4 * static_cast<int>(sizeof(float));
+__host__ __device__ inline Geometry geometry(int K) {
+    Geometry g{};
+    g.inner = 8;
+    for (int c = 256; c >= 8; c >>= 1)
+        if (K % c == 0) {
+            g.inner = c;
+            break;
+        }
+    g.ok = false;
+    // Fewest slices that still leave room for >= 3 stages (else >= 2); prefer
+    // slices that divide K exactly.
+    for (int pass = 0; pass < 4 && !g.ok; ++pass) {
+        const int min_stages = pass < 2 ? 3 : 2;
+        const bool exact = (pass % 2) == 0;
+        for (int s = 1; s <= 256; ++s) {
+            const int per = (K + s - 1) / s;
+            if (exact && (K % s != 0 || (K / s) % g.inner != 0)) continue;
+            const int kc = (per + g.inner - 1) / g.inner * g.inner;
+            if (kc / g.inner > 256) continue;
+            const int stage = 32 * kc;  // 16 rows x kc bf16
+            const int xbytes = 16 * s * kc;
+            int st = (kSmemBudget - xbytes) / stage;
+            if (st > kMaxStages) st = kMaxStages;
+            if (xbytes < kSmemBudget && st >= min_stages) {
+                g.slices = s;
+                g.kc = kc;
+                g.stages = st;
+                g.ok = true;
+                break;
+            }
+        }
+    }
+    if (!g.ok) return g;
+    g.kx = g.slices * g.kc;
+    g.off_x = g.stages * 32 * g.kc;
+    g.off_red = g.off_x + 16 * g.kx;
+    g.off_bar = g.off_red + kRedBytes;
+    g.smem = g.off_bar + 8 * kNumBars + 16 + 1024;  // + alignment slack
+    if (g.smem > kMaxSmem) g.ok = false;
+    return g;
 }
 
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -69,109 +122,194 @@ __device__ __forceinline__ float silu_mul_fast(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-__global__ void __launch_bounds__(kThreads)
-    swiglu_decode_bf16_kernel(const __nv_bfloat16 *__restrict__ X,
-                              const __nv_bfloat16 *__restrict__ Wg,
-                              const __nv_bfloat16 *__restrict__ Wu,
+__global__ void __launch_bounds__(kThreads, 1)
+    swiglu_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_wg,
+                              const __grid_constant__ CUtensorMap tm_wu,
+                              const __nv_bfloat16 *__restrict__ X,
                               __nv_bfloat16 *__restrict__ H, int M, int K, int N) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int pitch = x_pitch_bytes(K);
-    float *red = reinterpret_cast<float *>(smem + 8 * pitch);
-    const uint32_t xs = smem_u32(smem);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const Geometry geo = geometry(K);
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (sbase - raw);
+    const uint32_t stage_bytes = 32u * geo.kc;
+    const uint32_t xs = sbase + geo.off_x;
+    const uint32_t x_pitch = 2u * geo.kx;
+    float *red = reinterpret_cast<float *>(gbase + geo.off_red);
+    const uint32_t bar_full = sbase + geo.off_bar;
+    const uint32_t bar_empty = bar_full + 8 * kMaxStages;
+    const uint32_t bar_x = bar_empty + 8 * kMaxStages;
+    const uint32_t bar_xzero = bar_x + 8;
+    const uint32_t bar_red_full = bar_xzero + 8;
+    const uint32_t bar_red_empty = bar_red_full + 8;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + geo.off_bar + 8 * kNumBars);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int grp = lane >> 2;  // row of the unit (and column of B = row of X)
-    const int tig = lane & 3;   // which 8-element slice of a 32-wide chunk
     const int units = N / 8;
-    const int chunks = (K + 31) / 32;
-    const int per_warp = (chunks + kWarps - 1) / kWarps;
-    const int c_begin = min(warp * per_warp, chunks);
-    const int c_end = min(c_begin + per_warp, chunks);
+    const int u_begin = static_cast<int>((static_cast<long long>(units) * blockIdx.x) / gridDim.x);
+    const int u_end = static_cast<int>((static_cast<long long>(units) * (blockIdx.x + 1)) / gridDim.x);
 
-    uint4 wg[kPrefetch], wu[kPrefetch];
-
-    // Issue the loads of chunk c of unit u into slot s (zeros past K).
-    auto load_slot = [&](int s, int u, int c) {
-        const int k = c * 32 + tig * 8;
-        if (k < K) {
-            const size_t off = static_cast<size_t>(u * 8 + grp) * K + k;
-            wg[s] = ld_nc_stream_v4(Wg + off);
-            wu[s] = ld_nc_stream_v4(Wu + off);
-        } else {
-            wg[s] = make_uint4(0, 0, 0, 0);
-            wu[s] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < geo.stages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, kConsumerWarps);
         }
-    };
-    auto prologue = [&](int u) {
-#pragma unroll
-        for (int s = 0; s < kPrefetch; ++s)
-            if (c_begin + s < c_end) load_slot(s, u, c_begin + s);
-    };
-
-    int u = blockIdx.x;
-    if (u < units) prologue(u);
-
-    // Stage X (zero rows >= M and columns >= K) while those loads fly.
-    {
-        const int kp = padded_k(K);
-        const int vec_per_row = kp / 8;
-        for (int i = threadIdx.x; i < 8 * vec_per_row; i += kThreads) {
-            const int r = i / vec_per_row;
-            const int k = (i - r * vec_per_row) * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (r < M && k < K) v = *reinterpret_cast<const uint4 *>(X + static_cast<size_t>(r) * K + k);
-            sts_v4(xs + r * pitch + k * 2, v);
-        }
+        mbar_init(bar_x, 1);
+        mbar_init(bar_xzero, kConsumerWarps);
+        mbar_init(bar_red_full, kConsumerWarps);
+        mbar_init(bar_red_empty, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_wg);
+        tma_prefetch_desc(&tm_wu);
     }
     __syncthreads();
 
-    const uint32_t x_row = xs + grp * pitch + tig * 16;
-    for (; u < units; u += gridDim.x) {
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int cb = c_begin; cb < c_end; cb += kPrefetch) {
-#pragma unroll
-            for (int s = 0; s < kPrefetch; ++s) {
-                const int c = cb + s;
-                if (c < c_end) {
-                    const uint4 x = lds_v4(x_row + c * 64);
-                    // k order inside each 16-wide step: lane (grp, tig) holds
-                    // physical k 8*tig + {0..3} (first MMA) and 8*tig + {4..7}
-                    // (second MMA) of the chunk, for A and B alike.
-                    mma_m16n8k16_bf16(d, wg[s].x, wu[s].x, wg[s].y, wu[s].y, x.x, x.y);
-                    mma_m16n8k16_bf16(d, wg[s].z, wu[s].z, wg[s].w, wu[s].w, x.z, x.w);
-                    if (c + kPrefetch < c_end) load_slot(s, u, c + kPrefetch);
+    bool failed = false;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------- weight stream
+            mbar_arrive_expect_tx(bar_x, static_cast<uint32_t>(M * K * 2));
+            if (geo.kx == K) {
+                bulk_load(xs, X, static_cast<uint32_t>(M * K * 2), bar_x);
+            } else {
+                for (int m = 0; m < M; ++m)
+                    bulk_load(xs + m * x_pitch, X + static_cast<size_t>(m) * K,
+                              static_cast<uint32_t>(K * 2), bar_x);
+            }
+            const int kb_per_slice = geo.kc / geo.inner;
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int u = u_begin; u < u_end && !failed; ++u) {
+                for (int j = 0; j < geo.slices; ++j) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t st = sbase + stage * stage_bytes;
+                    mbar_arrive_expect_tx(fb, stage_bytes);
+                    // box: inner x (kc / inner) x 8 rows; k beyond K is zero-filled
+                    tma_load_3d(&tm_wg, fb, st, 0, j * kb_per_slice, u * 8);
+                    tma_load_3d(&tm_wu, fb, st + stage_bytes / 2, 0, j * kb_per_slice, u * 8);
+                    ++issued;
+                    if (++stage == geo.stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
-        }
-        // Cross-warp reduction in a fixed order.
-        float *mine = red + (warp * 32 + lane) * 4;
-        mine[0] = d[0];
-        mine[1] = d[1];
-        mine[2] = d[2];
-        mine[3] = d[3];
-        const int u_next = u + gridDim.x;
-        if (u_next < units) prologue(u_next);  // registers are free again
-        __syncthreads();
-        if (warp == 0) {
-            float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                const float *p = red + (w * 32 + lane) * 4;
-                s4[0] += p[0];
-                s4[1] += p[1];
-                s4[2] += p[2];
-                s4[3] += p[3];
+            // Never leave while a copy issued here may still write shared memory.
+            for (int s = 0; s < geo.stages; ++s) {
+                if (issued > s) {
+                    const long long uses = (issued - 1 - s) / geo.stages + 1;
+                    mbar_wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1));
+                }
             }
-            // s4[0], s4[1]: gate at m = 2*tig, 2*tig+1; s4[2], s4[3]: up.
-            const int n = u * 8 + grp;
-            const int m0 = 2 * tig;
-            if (m0 < M) H[static_cast<size_t>(m0) * N + n] = __float2bfloat16_rn(silu_mul_fast(s4[0], s4[2]));
-            if (m0 + 1 < M)
-                H[static_cast<size_t>(m0 + 1) * N + n] = __float2bfloat16_rn(silu_mul_fast(s4[1], s4[3]));
+            mbar_wait_drain(bar_x, 0);
         }
-        __syncthreads();
+    } else {
+        // ------------------------------------------------------ consumers
+        const int cw = warp - 1;
+        const int ct = threadIdx.x - 32;  // 0..127
+        const int grp = lane >> 2;
+        const int tig = lane & 3;
+        // Zero the X stage where the copies do not write: rows >= M, and the
+        // columns [K, kx) of rows < M (disjoint from the copies' bytes).
+        {
+            const int vec_per_row = static_cast<int>(x_pitch / 16);
+            for (int i = ct; i < 8 * vec_per_row; i += 32 * kConsumerWarps) {
+                const int r = i / vec_per_row;
+                const int byte = (i - r * vec_per_row) * 16;
+                if (r >= M || byte >= K * 2) sts_v4(xs + r * x_pitch + byte, make_uint4(0, 0, 0, 0));
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_xzero);
+        if (!mbar_wait(bar_xzero, 0, abort_flag) || !mbar_wait(bar_x, 0, abort_flag)) failed = true;
+
+        const uint32_t w_pitch = 2u * geo.kc;
+        const int chunks = (geo.kc + 31) / 32;
+        const uint32_t x_lane = xs + grp * x_pitch + tig * 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int u = u_begin; u < u_end && !failed; ++u) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < geo.slices; ++j) {
+                if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t st = sbase + stage * stage_bytes;
+                const uint32_t g_row = st + grp * w_pitch + tig * 16;
+                const uint32_t u_row = st + (8 + grp) * w_pitch + tig * 16;
+                const uint32_t x_row = x_lane + j * geo.kc * 2;
+#pragma unroll 2
+                for (int c = cw; c < chunks; c += kConsumerWarps) {
+                    uint4 wg = make_uint4(0, 0, 0, 0), wu = wg, x = wg;
+                    if (c * 32 + tig * 8 < geo.kc) {  // only a kc not divisible by 32 fails
+                        wg = lds_v4(g_row + c * 64);
+                        wu = lds_v4(u_row + c * 64);
+                        x = lds_v4(x_row + c * 64);
+                    }
+                    // lane (grp, tig) holds physical k 8*tig + {0..3} of the
+                    // chunk for the first MMA and 8*tig + {4..7} for the
+                    // second, in A and B alike.
+                    mma_m16n8k16_bf16(d, wg.x, wu.x, wg.y, wu.y, x.x, x.y);
+                    mma_m16n8k16_bf16(d, wg.z, wu.z, wg.w, wu.w, x.z, x.w);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
+                if (++stage == geo.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (failed) break;
+            // Cross-warp reduction in a fixed order.  red is free once the
+            // previous unit's epilogue has read it (red_empty).
+            const uint32_t par = static_cast<uint32_t>((u - u_begin) & 1);
+            if (u > u_begin && !mbar_wait(bar_red_empty, par ^ 1u, abort_flag)) {
+                failed = true;
+                break;
+            }
+            float *mine = red + (cw * 32 + lane) * 4;
+            mine[0] = d[0];
+            mine[1] = d[1];
+            mine[2] = d[2];
+            mine[3] = d[3];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_red_full);
+            if (cw == 0) {
+                if (!mbar_wait(bar_red_full, par, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float *p = red + (w * 32 + lane) * 4;
+                    s4[0] += p[0];
+                    s4[1] += p[1];
+                    s4[2] += p[2];
+                    s4[3] += p[3];
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_red_empty);
+                // s4[0], s4[1]: gate at m = 2*tig, 2*tig+1; s4[2], s4[3]: up.
+                const int n = u * 8 + grp;
+                const int m0 = 2 * tig;
+                if (m0 < M)
+                    H[static_cast<size_t>(m0) * N + n] = __float2bfloat16_rn(silu_mul_fast(s4[0], s4[2]));
+                if (m0 + 1 < M)
+                    H[static_cast<size_t>(m0 + 1) * N + n] =
+                        __float2bfloat16_rn(silu_mul_fast(s4[1], s4[3]));
+            }
+        }
     }
+    if (failed) atomicOr(&g_decode_status, 1u);
 }
 
 std::atomic<unsigned> g_attr_set_mask{0};
@@ -179,12 +317,25 @@ std::atomic<unsigned> g_attr_set_mask{0};
 }  // namespace
 
 bool decode_bf16_supported(int K) {
-    return K >= 0 && K <= (1 << 20) && decode_smem_bytes(K) <= kMaxSmem;
+    if (K < 8 || K % 8 != 0 || K > (1 << 16)) return false;
+    return geometry(K).ok;
 }
 
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
                                int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
-    const int smem = decode_smem_bytes(K);
+    const Geometry geo = geometry(K);
+    if (!geo.ok) return cudaErrorInvalidValue;
+    // 3-D view of each weight matrix: [N rows][K / inner blocks][inner]; a box
+    // is inner x (kc / inner) x 8 rows.
+    CUtensorMap tg, tu;
+    const uint64_t blocks = static_cast<uint64_t>(K / geo.inner);
+    const uint32_t kb = static_cast<uint32_t>(geo.kc / geo.inner);
+    if (!encode_tmap_3d(&tg, Wg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, geo.inner, blocks, N,
+                        2ull * geo.inner, 2ull * K, geo.inner, kb, 8) ||
+        !encode_tmap_3d(&tu, Wu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, geo.inner, blocks, N,
+                        2ull * geo.inner, 2ull * K, geo.inner, kb, 8)) {
+        return cudaErrorInvalidValue;
+    }
     const unsigned bit = 1u << (dev.device & 31);
     if (!(g_attr_set_mask.load() & bit)) {
         cudaError_t e = cudaFuncSetAttribute(swiglu_decode_bf16_kernel,
@@ -193,14 +344,21 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
         g_attr_set_mask.fetch_or(bit);
     }
     const int units = N / 8;
-    int per_sm = (200 * 1024) / smem;
-    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
-    const long long want = static_cast<long long>(dev.sm_count) * per_sm;
-    const int grid = static_cast<int>(units < want ? units : want);
-    swiglu_decode_bf16_kernel<<<grid, kThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(Wg),
-        static_cast<const __nv_bfloat16 *>(Wu), static_cast<__nv_bfloat16 *>(H), M, K, N);
+    const int grid = units < dev.sm_count ? units : dev.sm_count;
+    swiglu_decode_bf16_kernel<<<grid, kThreads, geo.smem, stream>>>(
+        tg, tu, static_cast<const __nv_bfloat16 *>(X), static_cast<__nv_bfloat16 *>(H), M, K, N);
     return cudaGetLastError();
+}
+
+cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host_out, g_decode_status, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_decode_status, &zero, sizeof(unsigned int), 0,
+                                cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
 }
 
 }  // namespace swiglu

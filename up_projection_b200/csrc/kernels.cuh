@@ -28,7 +28,7 @@ cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, vo
                                cudaStream_t stream);
 
 // bf16 forward for M <= 8: weight streaming with tensor-core dot products.
-// decode_bf16_supported: whether K fits the kernel's shared-memory X stage
+// decode_bf16_supported: whether K fits the kernel's shared-memory stages
 // (a pure function of K; larger K routes to the dual GEMM).
 bool decode_bf16_supported(int K);
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H,
@@ -49,6 +49,7 @@ cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void 
 // one into *host_out, reset it, and wait for the stream.
 cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool tensor_maps_available();

@@ -90,6 +90,27 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+// 3-D tiled load global -> shared (this CTA); x innermost, in elements.
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar, uint32_t dst,
+                                            int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// Non-tensor bulk copy global -> shared (this CTA); addresses 16-byte
+// aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 // 2-D tiled store shared -> global; elements outside the tensor are clipped.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src,
                                              int32_t x, int32_t y) {

@@ -16,4 +16,10 @@ bool encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtyp
                     uint64_t inner, uint64_t outer, uint64_t row_bytes,
                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// Encode a 3-D tensor: dims {d0, d1, d2} (d0 contiguous), byte strides of
+// dims 1 and 2, moved in boxes of {b0, b1, b2}, no swizzle.
+bool encode_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
+                    uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+                    uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+
 }  // namespace swiglu
