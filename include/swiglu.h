@@ -69,7 +69,18 @@ enum swiglu_status {
     SWIGLU_ERR_CUDA = 7,             /* a CUDA runtime/driver call failed   */
     SWIGLU_ERR_TIMEOUT = 8,          /* a device-side bounded wait gave up  */
     SWIGLU_ERR_OVERLAP = 9,          /* an output overlaps an input         */
-    SWIGLU_ERR_NO_DEVICE = 10        /* no CUDA device is usable            */
+    SWIGLU_ERR_NO_DEVICE = 10,       /* no CUDA device is usable            */
+    SWIGLU_ERR_BAD_FLAGS = 11        /* unknown bit in swiglu_fwd_ex flags  */
+};
+
+/* Flags of swiglu_fwd_ex. */
+enum swiglu_flags {
+    /* Wg and Wu are not written by work enqueued earlier on the stream, so
+     * the decode kernel may start streaming them before that work has
+     * finished (programmatic dependent launch).  X is still read, and H
+     * written, only after all earlier work on the stream has completed.
+     * Ignored by routes other than SWIGLU_ROUTE_DECODE_BF16. */
+    SWIGLU_FLAG_WEIGHTS_STABLE = 1
 };
 
 /* Kernel routes (which kernel a swiglu_fwd call enqueues). */
@@ -103,6 +114,16 @@ enum swiglu_route {
 SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu,
                           void *H, int64_t M, int64_t K, int64_t N, int dtype,
                           cudaStream_t stream);
+
+/*
+ * swiglu_fwd_ex -- swiglu_fwd with `flags`, a bitwise OR of swiglu_flags.
+ * flags == 0 is exactly swiglu_fwd; unknown bits return
+ * SWIGLU_ERR_BAD_FLAGS before anything is enqueued.
+ */
+SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu,
+                             void *H, int64_t M, int64_t K, int64_t N,
+                             int dtype, unsigned int flags,
+                             cudaStream_t stream);
 
 /*
  * dswiglu_bwd -- elementwise dSwiGLU, bf16.

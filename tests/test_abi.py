@@ -82,7 +82,14 @@ def test_no_device_is_an_error_not_a_fallback():
     assert st == _capi.SWIGLU_ERR_NO_DEVICE
 
 
+def test_unknown_flags_rejected():
+    lib = _capi.lib()
+    assert lib.swiglu_fwd_ex(16, 32, 48, 64, 4, 64, 64, 0, 2, None) == _capi.SWIGLU_ERR_BAD_FLAGS
+    assert lib.swiglu_fwd_ex(None, None, None, None, 4, 64, 64, 0, 1, None) == \
+        _capi.SWIGLU_ERR_NULL_POINTER
+
+
 def test_status_strings():
-    for code in range(11):
+    for code in range(12):
         assert _capi.status_string(code)
     assert _capi.status_string(999) == "unknown status"

@@ -150,3 +150,41 @@ def test_decode_astrai_full_size_rotated_copies():
             assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
             assert _capi.swiglu_last_route() == _capi.ROUTE_DECODE_BF16
             assert_bf16_close(f64(H), ref, f"astrai M={M} copy={r}")
+
+
+@pytest.mark.parametrize("K,N", [(1536, 6912), (4096, 11008), (256, 512)])
+def test_decode_weights_stable_path(K, N):
+    """The programmatic-dependent-launch path (weights prefetched before the
+    preceding kernel finishes) gives oracle-exact-within-tolerance results."""
+    for M in (1, 8):
+        X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M + 5)
+        Xd, Wgd, Wud = to_dev(X, Wg, Wu)
+        H = _capi.swiglu_fwd(Xd, Wgd, Wud, weights_stable=True)
+        assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+        assert _capi.swiglu_last_route() == _capi.ROUTE_DECODE_BF16
+        assert_bf16_close(f64(H), oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"], f"pdl M={M} K={K}")
+
+
+def test_decode_weights_stable_chain_reads_x_after_producer():
+    """A chain of dependent decode calls on one stream, each call's input X
+    being the previous call's output H, all with weights_stable: every X read
+    must see the finished output of the call before it."""
+    K = N = 1536
+    M, steps = 8, 12
+    X0, _, _ = synth.swiglu_inputs(M, K, N, "bf16", seed=21)
+    Ws = [synth.swiglu_inputs(1, K, N, "bf16", seed=100 + i)[1:] for i in range(steps)]
+    dev_ws = [(g.to(dev()), u.to(dev())) for g, u in Ws]
+    x = X0.to(dev())
+    outs = []
+    for g, u in dev_ws:
+        x = _capi.swiglu_fwd(x, g, u, weights_stable=True)
+        outs.append(x)
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+    # step by step on the host: each oracle step takes the GPU's previous
+    # (bf16) output, so errors do not compound across the chain
+    prev = X0
+    for i, (g, u) in enumerate(Ws):
+        ref = oracle.swiglu_fwd(prev, g, u, "bf16")["H"]
+        got = outs[i].cpu()
+        assert_bf16_close(f64(got), ref, f"chain step {i}")
+        prev = got

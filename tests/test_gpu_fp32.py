@@ -4,7 +4,9 @@ Bound per element (the pages' fp32 target is 1e-5 relative; a pure relative
 error is ill-posed where H ~ 0, so it is taken relative to the magnitude of
 the terms before cancellation):
     |gpu - ref| <= 1e-5 * (|H| + |silu(G)| * sum_k|x wu| + |U| * |silu'(G)| * sum_k|x wg|)
-test_fp32_tolerance.py (CPU) shows this bound rejects plain TF32."""
+test_fp32_tolerance.py (CPU) shows this bound rejects plain TF32.  The
+full-size tests also hold the stricter norm-wise reading,
+||gpu - ref||_2 / ||ref||_2 <= 1e-5."""
 import numpy as np
 import pytest
 import torch
@@ -86,4 +88,5 @@ def test_fp32_full_size_sampled(K, N):
     print(f"fp32 K={K} N={N}: max err/scale {np.max(err / scale):.2e}, "
           f"norm-wise {np.linalg.norm(err) / np.linalg.norm(ref['H']):.2e}, "
           f"max rel where |H| > 0.1 rms {np.max(err[away] / np.abs(ref['H'][away])):.2e}")
-    assert np.linalg.norm(err) / np.linalg.norm(ref["H"]) < 1e-3
+    # the stricter reading of "1e-5 relative": norm-wise over the samples
+    assert np.linalg.norm(err) / np.linalg.norm(ref["H"]) <= FP32_FWD_TOL

@@ -30,6 +30,9 @@ SWIGLU_ERR_CUDA = 7
 SWIGLU_ERR_TIMEOUT = 8
 SWIGLU_ERR_OVERLAP = 9
 SWIGLU_ERR_NO_DEVICE = 10
+SWIGLU_ERR_BAD_FLAGS = 11
+# enum swiglu_flags
+SWIGLU_FLAG_WEIGHTS_STABLE = 1
 # enum swiglu_route
 ROUTE_NONE = 0
 ROUTE_ZERO_K = 1
@@ -44,6 +47,7 @@ _I = ctypes.c_int
 # name -> (restype, argtypes), mirroring include/swiglu.h
 SIGNATURES = {
     "swiglu_fwd": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
+    "swiglu_fwd_ex": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, ctypes.c_uint, _P]),
     "dswiglu_bwd": (_I, [_P, _P, _P, _P, _P, _I64, _P]),
     "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
@@ -116,10 +120,15 @@ def _dev(t: torch.Tensor, name: str):
 
 
 def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
-               H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+               H: torch.Tensor | None = None, stream=None,
+               weights_stable: bool = False) -> torch.Tensor:
     """H = silu(X Wg^T) * (X Wu^T) through the C ABI.  X [..., K] (leading
     dims are flattened to M rows, as the TensorRT-LLM fused up-projection
-    does), Wg/Wu [N, K]; bf16 or fp32, all contiguous on one GPU."""
+    does), Wg/Wu [N, K]; bf16 or fp32, all contiguous on one GPU.
+
+    weights_stable=True promises that no earlier work on the stream writes
+    Wg or Wu (SWIGLU_FLAG_WEIGHTS_STABLE): the decode kernel may then start
+    streaming them while the preceding kernel finishes."""
     for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
         _dev(t, n)
     if not (X.dtype == Wg.dtype == Wu.dtype):
@@ -138,8 +147,9 @@ def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
         _dev(H, "H")
         if H.dtype != X.dtype or H.numel() != M * N:
             raise ValueError("H has the wrong dtype or size")
-    st = lib().swiglu_fwd(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
-                          M, K, N, _dtype_code(X), _stream(stream))
+    flags = SWIGLU_FLAG_WEIGHTS_STABLE if weights_stable else 0
+    st = lib().swiglu_fwd_ex(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
+                             M, K, N, _dtype_code(X), flags, _stream(stream))
     _check("swiglu_fwd", st)
     return H
 

@@ -145,6 +145,13 @@ SWIGLU_API int swiglu_route_for(int64_t M, int64_t K, int64_t N, int dtype) {
 
 SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu, void *H, int64_t M,
                           int64_t K, int64_t N, int dtype, cudaStream_t stream) {
+    return swiglu_fwd_ex(X, Wg, Wu, H, M, K, N, dtype, 0u, stream);
+}
+
+SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu, void *H, int64_t M,
+                             int64_t K, int64_t N, int dtype, unsigned int flags,
+                             cudaStream_t stream) {
+    if (flags & ~static_cast<unsigned int>(SWIGLU_FLAG_WEIGHTS_STABLE)) return SWIGLU_ERR_BAD_FLAGS;
     int route = SWIGLU_ROUTE_NONE;
     int st = check_fwd(X, Wg, Wu, H, M, K, N, dtype, &route);
     if (st != SWIGLU_OK) return st;
@@ -162,7 +169,8 @@ SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu, void *H
             e = cudaMemsetAsync(H, 0, static_cast<size_t>(M) * N * elem_size(dtype), stream);
             break;
         case SWIGLU_ROUTE_DECODE_BF16:
-            e = launch_decode_bf16(X, Wg, Wu, H, m, k, n, dev, stream);
+            e = launch_decode_bf16(X, Wg, Wu, H, m, k, n, (flags & SWIGLU_FLAG_WEIGHTS_STABLE) != 0,
+                                   dev, stream);
             break;
         case SWIGLU_ROUTE_GEMM_BF16:
             e = launch_gemm_bf16(X, Wg, Wu, H, m, k, n, dev, stream);
@@ -208,6 +216,7 @@ SWIGLU_API const char *swiglu_status_string(int status) {
         case SWIGLU_ERR_TIMEOUT: return "device-side bounded wait gave up";
         case SWIGLU_ERR_OVERLAP: return "output overlaps an input";
         case SWIGLU_ERR_NO_DEVICE: return "no usable CUDA device";
+        case SWIGLU_ERR_BAD_FLAGS: return "unknown flag bit";
         default: return "unknown status";
     }
 }

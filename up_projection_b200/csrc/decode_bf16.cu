@@ -52,7 +52,11 @@ using gemm::mbar_wait_drain;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
 constexpr int kMaxStages = 4;
-constexpr int kSmemBudget = 220 * 1024;  // stages + X stage
+constexpr int kSmemBudget = 220 * 1024;  // stages + X stage, one CTA per SM
+// With programmatic dependent launch, a footprint that lets the next call's
+// CTA share the SM (2 x ~100 KB) so its weight prefetch overlaps this call's
+// tail -- used when it still gives >= 3 stages of >= 512 k.
+constexpr int kPdlSmemBudget = 100 * 1024;
 constexpr int kMaxSmem = 227 * 1024;     // B200 opt-in limit per block
 constexpr int kNumBars = 2 * kMaxStages + 4;  // full, empty, x, x_zero, red_full, red_empty
 constexpr int kRedBytes = kConsumerWarps * 32 * 4 * 4;
@@ -67,7 +71,7 @@ struct Geometry {
     bool ok;
 };
 
-__host__ __device__ inline Geometry geometry(int K) {
+__host__ __device__ inline Geometry geometry(int K, int budget) {
     Geometry g{};
     g.inner = 8;
     for (int c = 256; c >= 8; c >>= 1)
@@ -88,9 +92,9 @@ __host__ __device__ inline Geometry geometry(int K) {
             if (kc / g.inner > 256) continue;
             const int stage = 32 * kc;  // 16 rows x kc bf16
             const int xbytes = 16 * s * kc;
-            int st = (kSmemBudget - xbytes) / stage;
+            int st = (budget - xbytes) / stage;
             if (st > kMaxStages) st = kMaxStages;
-            if (xbytes < kSmemBudget && st >= min_stages) {
+            if (xbytes < budget && st >= min_stages) {
                 g.slices = s;
                 g.kc = kc;
                 g.stages = st;
@@ -109,6 +113,24 @@ __host__ __device__ inline Geometry geometry(int K) {
     return g;
 }
 
+// Shared-memory budget of a launch: the small footprint only when it keeps
+// three or more stages of at least 512 k.
+__host__ __device__ inline int decode_budget(int K, bool weights_stable) {
+    if (weights_stable) {
+        const Geometry g = geometry(K, kPdlSmemBudget);
+        if (g.ok && g.stages >= 3 && g.kc >= 512) return kPdlSmemBudget;
+    }
+    return kSmemBudget;
+}
+
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], uint32_t a0, uint32_t a1,
                                                   uint32_t a2, uint32_t a3, uint32_t b0,
                                                   uint32_t b1) {
@@ -122,13 +144,18 @@ __device__ __forceinline__ float silu_mul_fast(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     swiglu_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_wg,
                               const __grid_constant__ CUtensorMap tm_wu,
                               const __nv_bfloat16 *__restrict__ X,
-                              __nv_bfloat16 *__restrict__ H, int M, int K, int N) {
+                              __nv_bfloat16 *__restrict__ H, int M, int K, int N,
+                              int weights_stable, int budget) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const Geometry geo = geometry(K);
+    const Geometry geo = geometry(K, budget);
+    // Under programmatic dependent launch the next call may be scheduled as
+    // soon as every CTA of this one is running: it only prefetches weights
+    // until this grid has completed (griddepcontrol.wait below).
+    if (weights_stable) griddep_launch_dependents();
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (sbase - raw);
@@ -170,20 +197,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------- weight stream
-            mbar_arrive_expect_tx(bar_x, static_cast<uint32_t>(M * K * 2));
-            if (geo.kx == K) {
-                bulk_load(xs, X, static_cast<uint32_t>(M * K * 2), bar_x);
-            } else {
-                for (int m = 0; m < M; ++m)
-                    bulk_load(xs + m * x_pitch, X + static_cast<size_t>(m) * K,
-                              static_cast<uint32_t>(K * 2), bar_x);
-            }
+            // X is produced by earlier work on the stream: with weights_stable
+            // the first weight stages are issued before waiting for it.
+            bool x_issued = false;
+            auto issue_x = [&]() {
+                if (weights_stable) griddep_wait();
+                mbar_arrive_expect_tx(bar_x, static_cast<uint32_t>(M * K * 2));
+                if (geo.kx == K) {
+                    bulk_load(xs, X, static_cast<uint32_t>(M * K * 2), bar_x);
+                } else {
+                    for (int m = 0; m < M; ++m)
+                        bulk_load(xs + m * x_pitch, X + static_cast<size_t>(m) * K,
+                                  static_cast<uint32_t>(K * 2), bar_x);
+                }
+                x_issued = true;
+            };
+            if (!weights_stable) issue_x();
             const int kb_per_slice = geo.kc / geo.inner;
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
             for (int u = u_begin; u < u_end && !failed; ++u) {
                 for (int j = 0; j < geo.slices; ++j) {
+                    if (!x_issued && issued >= geo.stages) issue_x();
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
@@ -201,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if (!x_issued) issue_x();
             // Never leave while a copy issued here may still write shared memory.
             for (int s = 0; s < geo.stages; ++s) {
                 if (issued > s) {
@@ -318,12 +355,14 @@ std::atomic<unsigned> g_attr_set_mask{0};
 
 bool decode_bf16_supported(int K) {
     if (K < 8 || K % 8 != 0 || K > (1 << 16)) return false;
-    return geometry(K).ok;
+    return geometry(K, kSmemBudget).ok;
 }
 
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
-                               int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
-    const Geometry geo = geometry(K);
+                               int K, int N, bool weights_stable, const DeviceInfo &dev,
+                               cudaStream_t stream) {
+    const int budget = decode_budget(K, weights_stable);
+    const Geometry geo = geometry(K, budget);
     if (!geo.ok) return cudaErrorInvalidValue;
     // 3-D view of each weight matrix: [N rows][K / inner blocks][inner]; a box
     // is inner x (kc / inner) x 8 rows.
@@ -343,10 +382,29 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
         if (e != cudaSuccess) return e;
         g_attr_set_mask.fetch_or(bit);
     }
+    // The small footprint fits two CTAs per SM: launch two per SM so each SM
+    // keeps twice the bytes in flight (and the next call's CTAs take over SMs
+    // as this call's CTAs finish).
+    const int per_sm = (budget == kPdlSmemBudget) ? 2 : 1;
     const int units = N / 8;
-    const int grid = units < dev.sm_count ? units : dev.sm_count;
-    swiglu_decode_bf16_kernel<<<grid, kThreads, geo.smem, stream>>>(
-        tg, tu, static_cast<const __nv_bfloat16 *>(X), static_cast<__nv_bfloat16 *>(H), M, K, N);
+    const int want = dev.sm_count * per_sm;
+    const int grid = units < want ? units : want;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(geo.smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = weights_stable ? 1 : 0;
+    const __nv_bfloat16 *xp = static_cast<const __nv_bfloat16 *>(X);
+    __nv_bfloat16 *hp = static_cast<__nv_bfloat16 *>(H);
+    const int ws = weights_stable ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_decode_bf16_kernel, tg, tu, xp, hp, M, K, N,
+                                       ws, budget);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

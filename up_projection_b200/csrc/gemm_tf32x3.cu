@@ -22,10 +22,18 @@
 //    lo copy is written to a parallel buffer with the same (swizzled) layout;
 //  * warp 1 (one thread): MMA issuer -- per 8-deep step three
 //    tcgen05.mma kind::tf32 (M=128, N=256): Xhi*[Wg;Wu]hi, Xhi*[Wg;Wu]lo,
-//    Xlo*[Wg;Wu]hi into a double-buffered accumulator (gate columns 0..127,
-//    up columns 128..255);
-//  * warps 6..9: epilogue -- h = g * sigmoid(g) * u in fp32 with expf and
-//    IEEE division, fp32 result staged (128-byte swizzle) and stored by TMA.
+//    Xlo*[Wg;Wu]hi into the chunk accumulator (gate columns 0..127, up
+//    columns 128..255);
+//  * warps 6..9: accumulation and epilogue.  The tensor cores' fp32
+//    accumulation loses up to about one unit in the last place of the running
+//    sum per accumulate step, an error that grows linearly with K.  So each
+//    tile's K range is cut into chunks of kChunkKB k-blocks (256 k): the MMAs
+//    of a chunk start from zero in the chunk accumulator (TMEM columns 0..255)
+//    and these warps fold every finished chunk into a running sum (TMEM
+//    columns 256..511) with round-to-nearest fp32 adds on the CUDA cores,
+//    releasing the chunk accumulator right after reading it.  After the last
+//    chunk: h = g * sigmoid(g) * u in fp32 with expf and IEEE division, staged
+//    (128-byte swizzle) and stored by TMA while the next tile's MMAs run.
 // All waits are bounded as in the bf16 kernel.
 #include <atomic>
 
@@ -50,8 +58,9 @@ constexpr int kBN = 128;                 // H columns per tile (gate, up each)
 constexpr int kBK = 16;                  // fp32 k per stage: one 64-byte row
 constexpr int kStages = 4;
 constexpr int kUmmaK = 8;                // k per tcgen05.mma, kind::tf32
-constexpr int kAccCols = 2 * kBN;
-constexpr int kTmemCols = 2 * kAccCols;  // 512
+constexpr int kAccCols = 2 * kBN;        // gate + up columns
+constexpr int kTmemCols = 2 * kAccCols;  // chunk accumulator + running sum
+constexpr int kChunkKB = 16;             // k-blocks per accumulation chunk
 constexpr int kSplitWarps = 4;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * (kSplitWarps + kEpiWarps);  // 320
@@ -67,7 +76,7 @@ constexpr uint32_t kEpiBufBytes = 32 * 128;            // 32 rows x 32 fp32
 constexpr uint32_t kOffStages = 0;
 constexpr uint32_t kOffEpi = kOffStages + kStages * kStageBytes;
 constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
-constexpr uint32_t kNumBars = 3 * kStages + 2 + 2 + 1;  // full, ready, empty, tfull, tempty, drain
+constexpr uint32_t kNumBars = 3 * kStages + 3;  // full, ready, empty, chunk_full, chunk_empty, drain
 constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
 constexpr uint32_t kSmemUsed = kOffAbort + 8;
@@ -121,9 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_full = base + kOffBar;
     const uint32_t bar_ready = bar_full + 8 * kStages;
     const uint32_t bar_empty = bar_ready + 8 * kStages;
-    const uint32_t bar_tfull = bar_empty + 8 * kStages;
-    const uint32_t bar_tempty = bar_tfull + 16;
-    const uint32_t bar_drain = bar_tempty + 16;
+    const uint32_t bar_cfull = bar_empty + 8 * kStages;
+    const uint32_t bar_cempty = bar_cfull + 8;
+    const uint32_t bar_drain = bar_cempty + 8;
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + kOffTmemPtr);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
 
@@ -131,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x % 32;
     const int num_tiles = num_m_tiles * num_n_tiles;
     const int num_kb = (K + kBK - 1) / kBK;
+    const int num_chunks = (num_kb + kChunkKB - 1) / kChunkKB;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -138,10 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_ready + 8 * s, kSplitWarps);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, kEpiWarps);
-        }
+        mbar_init(bar_cfull, 1);
+        mbar_init(bar_cempty, kEpiWarps);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -202,46 +210,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = make_idesc(2u, kBM, 2 * kBN);
             int stage = 0;
             uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
+            uint32_t chunk_phase = 0;  // parity of the chunk accumulator's uses
             for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
-                if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag)) {
-                    failed = true;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(bar_ready + 8 * stage, phase, abort_flag)) {
+                for (int q = 0; q < num_chunks && !failed; ++q) {
+                    // the epilogue warps must have read the previous chunk
+                    if (!mbar_wait(bar_cempty, chunk_phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t st = sst + stage * kStageBytes;
-                    const uint64_t a_hi = sw64_kmajor_desc(st);
-                    const uint64_t b_hi = sw64_kmajor_desc(st + kABytes);
-                    const uint64_t a_lo = sw64_kmajor_desc(st + kRawBytes);
-                    const uint64_t b_lo = sw64_kmajor_desc(st + kRawBytes + kABytes);
+                    const int kb_end = min(num_kb, (q + 1) * kChunkKB);
+                    for (int kb = q * kChunkKB; kb < kb_end; ++kb) {
+                        if (!mbar_wait(bar_ready + 8 * stage, phase, abort_flag)) {
+                            failed = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t st = sst + stage * kStageBytes;
+                        const uint64_t a_hi = sw64_kmajor_desc(st);
+                        const uint64_t b_hi = sw64_kmajor_desc(st + kABytes);
+                        const uint64_t a_lo = sw64_kmajor_desc(st + kRawBytes);
+                        const uint64_t b_lo = sw64_kmajor_desc(st + kRawBytes + kABytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        // +32 bytes along K inside the 64-byte swizzled row.
-                        const uint32_t o = 2u * kk;
-                        const uint32_t first = (kb == 0 && kk == 0) ? 0u : 1u;
-                        mma_tf32(d_tmem, a_lo + o, b_hi + o, idesc, first);
-                        mma_tf32(d_tmem, a_hi + o, b_lo + o, idesc, 1u);
-                        mma_tf32(d_tmem, a_hi + o, b_hi + o, idesc, 1u);
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            // +32 bytes along K inside the 64-byte swizzled row.
+                            const uint32_t o = 2u * kk;
+                            const uint32_t acc = (kb == q * kChunkKB && kk == 0) ? 0u : 1u;
+                            mma_tf32(tmem_base, a_lo + o, b_hi + o, idesc, acc);
+                            mma_tf32(tmem_base, a_hi + o, b_lo + o, idesc, 1u);
+                            mma_tf32(tmem_base, a_hi + o, b_hi + o, idesc, 1u);
+                        }
+                        mma_commit(bar_empty + 8 * stage);
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
-                    mma_commit(bar_empty + 8 * stage);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (failed) break;
-                mma_commit(bar_tfull + 8 * acc);
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
+                    if (failed) break;
+                    mma_commit(bar_cfull);
+                    chunk_phase ^= 1u;
                 }
             }
             mma_commit(bar_drain);
@@ -250,7 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kFirstEpiWarp) {
         // ---------------------------------------------------- hi/lo split
         const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
+        constexpr int kThreadsSplit = 32 * kSplitWarps;
         constexpr int kVecs = kRawBytes / 16;                  // 1536 per stage
+        constexpr int kPerThread = kVecs / kThreadsSplit;      // 12
+        static_assert(kVecs % kThreadsSplit == 0, "split work must divide evenly");
         int stage = 0;
         uint32_t phase = 0;
         for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
@@ -260,13 +270,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint32_t st = sst + stage * kStageBytes;
-#pragma unroll 4
-                for (int v = sidx; v < kVecs; v += 32 * kSplitWarps) {
-                    uint4 x = lds_v4(st + 16u * v);
+                // all loads first, then the splits and stores, so the shared-
+                // memory latency is paid once per stage
+                uint4 x[kPerThread];
+#pragma unroll
+                for (int i = 0; i < kPerThread; ++i)
+                    x[i] = lds_v4(st + 16u * (sidx + i * kThreadsSplit));
+#pragma unroll
+                for (int i = 0; i < kPerThread; ++i) {
                     uint4 lo;
-                    split4(x, lo);
-                    sts_v4(st + 16u * v, x);
-                    sts_v4(st + kRawBytes + 16u * v, lo);
+                    split4(x[i], lo);
+                    const uint32_t off = 16u * (sidx + i * kThreadsSplit);
+                    sts_v4(st + off, x[i]);
+                    sts_v4(st + kRawBytes + off, lo);
                 }
                 // make the generic-proxy writes visible to the tensor cores
                 fence_proxy_async_smem();
@@ -279,30 +295,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------- epilogue
+        // ------------------------------------------ accumulation + epilogue
         const int quad = warp & 3;
         const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t chunk_acc = tmem_base + row_off;             // cols 0..255
+        const uint32_t run_acc = tmem_base + row_off + kAccCols;    // cols 256..511
         const uint32_t buf = se + static_cast<uint32_t>(warp - kFirstEpiWarp) * kEpiBufBytes;
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        uint32_t chunk_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
             int mt, nt;
             tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
             const int m0 = mt * kBM, n0 = nt * kBN;
-            if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
-                failed = true;
-                break;
+            // fold every chunk into the running sum and release the chunk
+            // accumulator; the next tile's first chunk then overlaps the
+            // output below
+            for (int q = 0; q < num_chunks; ++q) {
+                if (!mbar_wait(bar_cfull, chunk_phase, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                chunk_phase ^= 1u;
+                tc_fence_after();
+#pragma unroll 1
+                for (int col = 0; col < kAccCols; col += 32) {
+                    uint32_t c[32], r[32];
+                    tmem_ld_32x32b_x32(chunk_acc + col, c);
+                    if (q > 0) tmem_ld_32x32b_x32(run_acc + col, r);
+                    tmem_ld_wait(c);
+                    if (q > 0) {
+                        tmem_ld_wait(r);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            c[i] = __float_as_uint(__fadd_rn(__uint_as_float(r[i]),
+                                                             __uint_as_float(c[i])));
+                    }
+                    tmem_st_32x32b_x32(run_acc + col, c);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_cempty);
             }
-            tc_fence_after();
-            const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kAccCols);
+            if (failed) break;
+            // output from the running sum
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 if (lane == 0) bulk_wait_read<0>();
                 __syncwarp();
                 uint32_t g[32], u[32];
-                tmem_ld_32x32b_x32(tacc + 32u * c, g);
-                tmem_ld_32x32b_x32(tacc + kBN + 32u * c, u);
+                tmem_ld_32x32b_x32(run_acc + 32u * c, g);
+                tmem_ld_32x32b_x32(run_acc + kBN + 32u * c, u);
                 tmem_ld_wait(g);
                 tmem_ld_wait(u);
 #pragma unroll
@@ -326,13 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bulk_commit();
                     }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
             }
         }
         if (lane == 0) bulk_wait<0>();

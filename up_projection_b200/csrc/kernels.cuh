@@ -31,9 +31,12 @@ cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, vo
 // decode_bf16_supported: whether K fits the kernel's shared-memory stages
 // (a pure function of K; larger K routes to the dual GEMM).
 bool decode_bf16_supported(int K);
+// weights_stable: launch with programmatic dependent launch and prefetch the
+// first weight stages before waiting for the preceding grid (see
+// SWIGLU_FLAG_WEIGHTS_STABLE).
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H,
-                               int M, int K, int N, const DeviceInfo &dev,
-                               cudaStream_t stream);
+                               int M, int K, int N, bool weights_stable,
+                               const DeviceInfo &dev, cudaStream_t stream);
 
 // Elementwise dSwiGLU; dtype 0 = bf16, 1 = fp32.
 cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG,
