@@ -17,8 +17,9 @@ decode shape (GB/s), each with its roofline fraction.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and cuda synchronize, CUDA events on the launching stream, max over ranks.
-The step is replayed from CUDA graphs (one per group of 4 rotated copies) so
-host launch overhead does not starve the GPU.  Multi-GPU (torchrun): every
+The steps are replayed from CUDA graphs holding one full rotation of the
+copies (4 steps, 16 calls) so host launch overhead does not starve the GPU
+and consecutive calls overlap under programmatic dependent launch.  Multi-GPU (torchrun): every
 rank runs the same per-GPU workload on its own GPU (independent problems, no
 data-path collective): weak scaling, value = all ranks' bytes / max time.
 
@@ -56,11 +57,12 @@ DECODE_COPIES = 16
 # DRAM traffic of the decode kernel per launch from one ncu capture, keyed by
 # the sha256 of the kernel source it was measured on; reported as null when
 # the source has changed since.
-DECODE_TRAFFIC = {"src_sha256": "75a1d6a990d619b7277d4f0adcf7dd69036f86b7799f0159159836affecf108a",
-                  # one ncu capture of this kernel at M = 8 (AstrAI-1B shape);
-                  # X and H add < 0.3 % per M, so it stands for every M.
-                  "bytes_per_launch_by_M": {"1": 42526720, "2": 42526720, "4": 42526720,
-                                            "8": 42526720}}
+DECODE_TRAFFIC = {"src_sha256": "abf674ca452f48cf26473f03aaa655244986f43d84c2448c917910274ffc02be",
+                  # one ncu capture of this kernel at M = 8 (AstrAI-1B shape,
+                  # weights-stable launch); X and H add < 0.3 % per M, so it
+                  # stands for every M.
+                  "bytes_per_launch_by_M": {"1": 42532864, "2": 42532864, "4": 42532864,
+                                            "8": 42532864}}
 
 
 def peaks():
@@ -205,43 +207,49 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
     Xd = {M: Xs_host[M].to(dev) for M in Ms}
     Hd = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
     per_step = len(Ms)
-    groups = copies // per_step   # one graph per group of per_step copies
+    groups = copies // per_step   # steps per full rotation of the copies
 
     def step_calls(g):
         for i, M in enumerate(Ms):
             c = g * per_step + i
             up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream, weights_stable=True)
 
-    # eager warm-up (tensor maps, function attributes), then capture
+    # eager warm-up (tensor maps, function attributes), then capture: one graph
+    # per full rotation (groups steps, so consecutive calls overlap under
+    # programmatic dependent launch across the whole rotation), plus graphs of
+    # the first r steps for a remainder, so that exactly K steps are timed.
     with torch.cuda.stream(stream):
         for g in range(groups):
             step_calls(g)
     torch.cuda.synchronize()
     assert up.swiglu_sync_status(stream) == 0
-    graphs = []
-    for g in range(groups):
+
+    def capture(nsteps):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            step_calls(g)
-        graphs.append(gr)
+            for g in range(nsteps):
+                step_calls(g)
+        return gr
+
+    full = capture(groups)
+    partial = {r: capture(r) for r in range(1, groups)}
     torch.cuda.synchronize()
 
-    state = {"i": 0}
-
-    def one_step():
-        graphs[state["i"] % groups].replay()
-        state["i"] += 1
+    def run_steps(k):
+        for _ in range(k // groups):
+            full.replay()
+        if k % groups:
+            partial[k % groups].replay()
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            one_step()
+        run_steps(args.warmup)
     torch.cuda.synchronize()
     barrier(world)
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(torch.cuda.current_device())
     with ClockSampler(gpu_id) as clk:
         with torch.cuda.stream(stream):
-            ms = timed_events(one_step, args.steps, stream)
+            ms = timed_events(lambda: run_steps(args.steps), 1, stream)
     torch.cuda.synchronize()
     barrier(world)
     st = up.swiglu_sync_status(stream)
@@ -303,8 +311,7 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
         barrier(world)
         e_ms = max_over_ranks(e_ms, world)
         out["e2e"] = {"ms": e_ms, "steps": e_steps, "h2d": h2d, "d2h": d2h}
-    for g in graphs:
-        del g
+    del full, partial
     del Wg_all, Wu_all
     torch.cuda.empty_cache()
     return out

@@ -51,7 +51,7 @@ using gemm::mbar_wait_drain;
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kSmemBudget = 220 * 1024;  // stages + X stage, one CTA per SM
 // With programmatic dependent launch, a footprint that lets the next call's
 // CTA share the SM (2 x ~100 KB) so its weight prefetch overlaps this call's

@@ -29,6 +29,8 @@ def main(argv=None):
     ap.add_argument("--n", type=int, default=8192 * 14336)
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--weights-stable", action="store_true",
+                    help="decode: SWIGLU_FLAG_WEIGHTS_STABLE (programmatic dependent launch)")
     a = ap.parse_args(argv)
 
     import up_projection_b200 as up
@@ -47,7 +49,7 @@ def main(argv=None):
         for i in range(L):
             c = i % a.copies
             if a.case == "decode":
-                up.swiglu_fwd(X, Wg[c], Wu[c], H)
+                up.swiglu_fwd(X, Wg[c], Wu[c], H, weights_stable=a.weights_stable)
             else:
                 up.swiglu_read_floor(Wg[c], Wu[c], sink)
     elif a.case in ("prefill", "fp32"):
