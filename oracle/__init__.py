@@ -84,10 +84,23 @@ class Oracle:
 
     def __init__(self, lib_path: str):
         lib = ctypes.CDLL(lib_path)
-        for name in ("oracle_sigmoid", "oracle_silu", "oracle_dsilu"):
+        for name in ("oracle_sigmoid", "oracle_silu", "oracle_dsilu", "oracle_gelu_tanh",
+                     "oracle_dgelu_tanh"):
             f = getattr(lib, name)
             f.restype = _D
             f.argtypes = [_D]
+        for name in ("oracle_act", "oracle_dact"):
+            f = getattr(lib, name)
+            f.restype = _D
+            f.argtypes = [_D, ctypes.c_int]
+        lib.oracle_swiglu_fwd_act_f64.restype = None
+        lib.oracle_swiglu_fwd_act_f64.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _D,
+                                                  _P, _P, _P, _P, _P]
+        lib.oracle_swiglu_fwd_points_act.restype = ctypes.c_int
+        lib.oracle_swiglu_fwd_points_act.argtypes = [ctypes.c_int, _P, _P, _P, _I64, _P, _P, _I64,
+                                                     ctypes.c_int, _D, _P, _P, _P, _P, _P]
+        lib.oracle_dswiglu_act_f64.restype = None
+        lib.oracle_dswiglu_act_f64.argtypes = [_P, _P, _P, _I64, ctypes.c_int, _D, _P, _P]
         for name in ("oracle_bf16_to_f64", "oracle_f32_to_f64"):
             f = getattr(lib, name)
             f.restype = None
@@ -121,6 +134,19 @@ class Oracle:
     def dsilu(self, x: float) -> float:
         return self.lib.oracle_dsilu(float(x))
 
+    def gelu_tanh(self, x: float) -> float:
+        return self.lib.oracle_gelu_tanh(float(x))
+
+    def dgelu_tanh(self, x: float) -> float:
+        return self.lib.oracle_dgelu_tanh(float(x))
+
+    def act(self, x: float, act: int) -> float:
+        """Activation code 0 = SiLU, 1 = GELU(tanh)."""
+        return self.lib.oracle_act(float(x), int(act))
+
+    def dact(self, x: float, act: int) -> float:
+        return self.lib.oracle_dact(float(x), int(act))
+
     # ---- decoding ------------------------------------------------------------
     def decode_bf16(self, a) -> np.ndarray:
         """Exact float64 values of bf16 bit patterns (the oracle's decoder)."""
@@ -140,8 +166,10 @@ class Oracle:
         return out
 
     # ---- forward ---------------------------------------------------------------
-    def swiglu_fwd_f64(self, X, Wg, Wu, want_magnitudes: bool = False):
-        """Full forward on float64 operands X [M,K], Wg/Wu [N,K].
+    def swiglu_fwd_f64(self, X, Wg, Wu, want_magnitudes: bool = False, act: int = 0,
+                       alpha: float = 1.0):
+        """Full forward on float64 operands X [M,K], Wg/Wu [N,K]:
+        H = act(alpha * G) * U (act 0 = SiLU, 1 = GELU(tanh)).
 
         Returns a dict with G, U, H (float64 [M,N]) and, if asked,
         AG = sum_k |x wg| and AU = sum_k |x wu| (error-bound magnitudes)."""
@@ -155,20 +183,21 @@ class Oracle:
         if want_magnitudes:
             out["AG"] = np.empty((M, N), dtype=np.float64)
             out["AU"] = np.empty((M, N), dtype=np.float64)
-        self.lib.oracle_swiglu_fwd_f64(
-            _ptr(X), _ptr(Wg), _ptr(Wu), M, K, N, _ptr(out["G"]),
+        self.lib.oracle_swiglu_fwd_act_f64(
+            _ptr(X), _ptr(Wg), _ptr(Wu), M, K, N, int(act), float(alpha), _ptr(out["G"]),
             _ptr(out["U"]), _ptr(out["H"]),
             _ptr(out["AG"]) if want_magnitudes else None,
             _ptr(out["AU"]) if want_magnitudes else None)
         return out
 
     def swiglu_fwd(self, X, Wg, Wu, dtype: str = "bf16",
-                   want_magnitudes: bool = False):
+                   want_magnitudes: bool = False, act: int = 0, alpha: float = 1.0):
         """Full forward from bf16 (uint16 bits / torch.bfloat16) or fp32."""
         return self.swiglu_fwd_f64(self.decode(X, dtype), self.decode(Wg, dtype),
-                                   self.decode(Wu, dtype), want_magnitudes)
+                                   self.decode(Wu, dtype), want_magnitudes, act, alpha)
 
-    def swiglu_fwd_points(self, X, Wg, Wu, idx_m, idx_n, dtype: str = "bf16"):
+    def swiglu_fwd_points(self, X, Wg, Wu, idx_m, idx_n, dtype: str = "bf16",
+                          act: int = 0, alpha: float = 1.0):
         """Forward at the sampled outputs (idx_m[i], idx_n[i]) only, straight
         from the stored operands.  Returns float64 vectors G, U, H, AG, AU."""
         idx_m = np.ascontiguousarray(idx_m, dtype=np.int64)
@@ -190,28 +219,38 @@ class Oracle:
                               and 0 <= idx_n.min() and idx_n.max() < N)
         out = {k: np.empty(count, dtype=np.float64)
                for k in ("G", "U", "H", "AG", "AU")}
-        rc = fn(_ptr(Xa), _ptr(Wga), _ptr(Wua), K, _ptr(idx_m), _ptr(idx_n),
-                count, _ptr(out["G"]), _ptr(out["U"]), _ptr(out["H"]),
-                _ptr(out["AG"]), _ptr(out["AU"]))
+        if act == 0 and alpha == 1.0:
+            rc = fn(_ptr(Xa), _ptr(Wga), _ptr(Wua), K, _ptr(idx_m), _ptr(idx_n),
+                    count, _ptr(out["G"]), _ptr(out["U"]), _ptr(out["H"]),
+                    _ptr(out["AG"]), _ptr(out["AU"]))
+        else:
+            rc = self.lib.oracle_swiglu_fwd_points_act(
+                0 if dtype == "bf16" else 1, _ptr(Xa), _ptr(Wga), _ptr(Wua), K, _ptr(idx_m),
+                _ptr(idx_n), count, int(act), float(alpha), _ptr(out["G"]), _ptr(out["U"]),
+                _ptr(out["H"]), _ptr(out["AG"]), _ptr(out["AU"]))
         if rc != 0:
             raise MemoryError("oracle: row buffer allocation failed")
         return out
 
     # ---- backward --------------------------------------------------------------
-    def dswiglu_f64(self, dH, G, U):
-        """Elementwise dSwiGLU on float64 arrays of equal shape -> (dG, dU)."""
+    def dswiglu_f64(self, dH, G, U, act: int = 0, alpha: float = 1.0):
+        """Elementwise backward of h = act(alpha g) u on float64 arrays of
+        equal shape -> (dG, dU); act 0 = SiLU (dSwiGLU), 1 = GELU(tanh)."""
         dH = np.ascontiguousarray(dH, dtype=np.float64)
         G = np.ascontiguousarray(G, dtype=np.float64)
         U = np.ascontiguousarray(U, dtype=np.float64)
         assert dH.shape == G.shape == U.shape
         dG = np.empty(G.shape, dtype=np.float64)
         dU = np.empty(G.shape, dtype=np.float64)
-        self.lib.oracle_dswiglu_f64(_ptr(dH), _ptr(G), _ptr(U), G.size,
-                                    _ptr(dG), _ptr(dU))
+        self.lib.oracle_dswiglu_act_f64(_ptr(dH), _ptr(G), _ptr(U), G.size, int(act),
+                                        float(alpha), _ptr(dG), _ptr(dU))
         return dG, dU
 
-    def dswiglu(self, dH, G, U, dtype: str = "bf16"):
+    def dswiglu(self, dH, G, U, dtype: str = "bf16", act: int = 0, alpha: float = 1.0):
         """dSwiGLU straight from bf16 (bits / torch.bfloat16) or fp32."""
+        if act != 0 or alpha != 1.0:
+            return self.dswiglu_f64(self.decode(dH, dtype), self.decode(G, dtype),
+                                    self.decode(U, dtype), act, alpha)
         if dtype == "bf16":
             a, b, c = _as_bits(dH), _as_bits(G), _as_bits(U)
             fn = self.lib.oracle_dswiglu_bf16
@@ -238,7 +277,8 @@ def default() -> Oracle:
 
 def __getattr__(name):
     # Module-level convenience: oracle.swiglu_fwd(...) etc. use default().
-    if name in {"sigmoid", "silu", "dsilu", "decode_bf16", "decode",
+    if name in {"sigmoid", "silu", "dsilu", "gelu_tanh", "dgelu_tanh", "act", "dact",
+                "decode_bf16", "decode",
                 "swiglu_fwd_f64", "swiglu_fwd", "swiglu_fwd_points",
                 "dswiglu_f64", "dswiglu"}:
         return getattr(default(), name)

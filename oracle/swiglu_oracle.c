@@ -33,6 +33,10 @@
  * textbook definitions: sigmoid(x) = 1/(1+exp(-x)), silu(x) = x*sigmoid(x),
  * silu'(x) = sigmoid(x) * (1 + x*(1 - sigmoid(x))).
  *
+ * Epilogue variants (the _act entry points): h = act(alpha * g) * u with
+ * act = SiLU or GELU(tanh) and alpha the scalar gate multiplier; the plain
+ * entry points are act = SiLU, alpha = 1.
+ *
  * bf16 inputs arrive as their 16-bit patterns and are decoded here by a bit
  * shift into the top half of an IEEE float (exact), then widened to double.
  */
@@ -67,6 +71,40 @@ ORACLE_API double oracle_dsilu(double x)
     return s * (1.0 + x * (1.0 - s));
 }
 
+/*
+ * GELU with the tanh approximation, the "GELU(tanh)" of the GEGLU variant
+ * (TensorRT-LLM PR #17693 fuses GELU(tanh) into the up projection; Liger-
+ * Kernel issue #937 lists swiglu/geglu): gelu(x) = x/2 (1 + tanh(c (x + a x^3)))
+ * with c = sqrt(2/pi), a = 0.044715.  Derivative by differentiation.
+ */
+#define ORACLE_GELU_C 0.79788456080286535587989211986876 /* sqrt(2/pi) */
+#define ORACLE_GELU_A 0.044715
+
+ORACLE_API double oracle_gelu_tanh(double x)
+{
+    double t = tanh(ORACLE_GELU_C * (x + ORACLE_GELU_A * x * x * x));
+    return 0.5 * x * (1.0 + t);
+}
+
+ORACLE_API double oracle_dgelu_tanh(double x)
+{
+    double y = ORACLE_GELU_C * (x + ORACLE_GELU_A * x * x * x);
+    double t = tanh(y);
+    double dy = ORACLE_GELU_C * (1.0 + 3.0 * ORACLE_GELU_A * x * x);
+    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * dy;
+}
+
+/* Activation codes: 0 = SiLU, 1 = GELU(tanh). */
+ORACLE_API double oracle_act(double x, int act)
+{
+    return act == 1 ? oracle_gelu_tanh(x) : oracle_silu(x);
+}
+
+ORACLE_API double oracle_dact(double x, int act)
+{
+    return act == 1 ? oracle_dgelu_tanh(x) : oracle_dsilu(x);
+}
+
 /* ---- input decoding ---------------------------------------------------- */
 
 static double bf16_bits_to_double(uint16_t b)
@@ -97,9 +135,16 @@ ORACLE_API void oracle_f32_to_f64(const float *src, double *dst, int64_t n)
  * sum_k |x*wg| and sum_k |x*wu| that bound the rounding error of any
  * summation order (used by the fp32-mode tolerance).
  */
+/*
+ * The epilogue variants: h = act(alpha * g) * u, where alpha is the scalar
+ * gate multiplier of Liger-Kernel issue #937 (its "multiplier", for
+ * Falcon-H1) applied to the gate pre-activation, and act is SiLU (SwiGLU)
+ * or GELU(tanh) (GEGLU).  alpha = 1 and SiLU give the plain op.
+ */
 static void one_output(const double *x, const double *wg, const double *wu,
-                       int64_t K, double *g_out, double *u_out, double *h_out,
-                       double *ag_out, double *au_out)
+                       int64_t K, int act, double alpha, double *g_out,
+                       double *u_out, double *h_out, double *ag_out,
+                       double *au_out)
 {
     double g = 0.0, u = 0.0, ag = 0.0, au = 0.0;
     for (int64_t k = 0; k < K; ++k) {
@@ -112,7 +157,7 @@ static void one_output(const double *x, const double *wg, const double *wu,
     }
     if (g_out) *g_out = g;
     if (u_out) *u_out = u;
-    if (h_out) *h_out = oracle_silu(g) * u;
+    if (h_out) *h_out = oracle_act(alpha * g, act) * u;
     if (ag_out) *ag_out = ag;
     if (au_out) *au_out = au;
 }
@@ -123,20 +168,30 @@ static void one_output(const double *x, const double *wg, const double *wu,
  * OpenMP threads; each element's sum order does not depend on the thread
  * count.
  */
-ORACLE_API void oracle_swiglu_fwd_f64(const double *X, const double *Wg,
-                                      const double *Wu, int64_t M, int64_t K,
-                                      int64_t N, double *G, double *U,
-                                      double *H, double *AG, double *AU)
+ORACLE_API void oracle_swiglu_fwd_act_f64(const double *X, const double *Wg,
+                                          const double *Wu, int64_t M,
+                                          int64_t K, int64_t N, int act,
+                                          double alpha, double *G, double *U,
+                                          double *H, double *AG, double *AU)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
             int64_t o = m * N + n;
-            one_output(X + m * K, Wg + n * K, Wu + n * K, K,
+            one_output(X + m * K, Wg + n * K, Wu + n * K, K, act, alpha,
                        G ? G + o : 0, U ? U + o : 0, H ? H + o : 0,
                        AG ? AG + o : 0, AU ? AU + o : 0);
         }
     }
+}
+
+/* The plain op: SiLU, no gate multiplier. */
+ORACLE_API void oracle_swiglu_fwd_f64(const double *X, const double *Wg,
+                                      const double *Wu, int64_t M, int64_t K,
+                                      int64_t N, double *G, double *U,
+                                      double *H, double *AG, double *AU)
+{
+    oracle_swiglu_fwd_act_f64(X, Wg, Wu, M, K, N, 0, 1.0, G, U, H, AG, AU);
 }
 
 /*
@@ -155,7 +210,7 @@ ORACLE_API void oracle_swiglu_fwd_points_f64(const double *X, const double *Wg,
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < count; ++i) {
         one_output(X + idx_m[i] * K, Wg + idx_n[i] * K, Wu + idx_n[i] * K, K,
-                   G ? G + i : 0, U ? U + i : 0, H ? H + i : 0,
+                   0, 1.0, G ? G + i : 0, U ? U + i : 0, H ? H + i : 0,
                    AG ? AG + i : 0, AU ? AU + i : 0);
     }
 }
@@ -186,8 +241,9 @@ static void decode_f32_rows(const void *src, int64_t offset, double *dst,
 
 static int fwd_points(decode_fn dec, const void *X, const void *Wg,
                       const void *Wu, int64_t K, const int64_t *idx_m,
-                      const int64_t *idx_n, int64_t count, double *G,
-                      double *U, double *H, double *AG, double *AU)
+                      const int64_t *idx_n, int64_t count, int act,
+                      double alpha, double *G, double *U, double *H,
+                      double *AG, double *AU)
 {
     int failed = 0;
 #pragma omp parallel reduction(| : failed)
@@ -202,13 +258,27 @@ static int fwd_points(decode_fn dec, const void *X, const void *Wg,
             dec(X, idx_m[i] * K, buf, K);
             dec(Wg, idx_n[i] * K, buf + K, K);
             dec(Wu, idx_n[i] * K, buf + 2 * K, K);
-            one_output(buf, buf + K, buf + 2 * K, K, G ? G + i : 0,
+            one_output(buf, buf + K, buf + 2 * K, K, act, alpha, G ? G + i : 0,
                        U ? U + i : 0, H ? H + i : 0, AG ? AG + i : 0,
                        AU ? AU + i : 0);
         }
         free(buf);
     }
     return failed ? -1 : 0;
+}
+
+ORACLE_API int oracle_swiglu_fwd_points_act(int storage, const void *X,
+                                            const void *Wg, const void *Wu,
+                                            int64_t K, const int64_t *idx_m,
+                                            const int64_t *idx_n,
+                                            int64_t count, int act,
+                                            double alpha, double *G,
+                                            double *U, double *H, double *AG,
+                                            double *AU)
+{
+    /* storage: 0 = bf16 bit patterns, 1 = fp32 */
+    return fwd_points(storage == 0 ? decode_bf16_rows : decode_f32_rows, X, Wg,
+                      Wu, K, idx_m, idx_n, count, act, alpha, G, U, H, AG, AU);
 }
 
 ORACLE_API int oracle_swiglu_fwd_points_bf16(const uint16_t *X,
@@ -220,8 +290,8 @@ ORACLE_API int oracle_swiglu_fwd_points_bf16(const uint16_t *X,
                                              double *U, double *H, double *AG,
                                              double *AU)
 {
-    return fwd_points(decode_bf16_rows, X, Wg, Wu, K, idx_m, idx_n, count, G,
-                      U, H, AG, AU);
+    return fwd_points(decode_bf16_rows, X, Wg, Wu, K, idx_m, idx_n, count, 0,
+                      1.0, G, U, H, AG, AU);
 }
 
 ORACLE_API int oracle_swiglu_fwd_points_f32(const float *X, const float *Wg,
@@ -232,32 +302,41 @@ ORACLE_API int oracle_swiglu_fwd_points_f32(const float *X, const float *Wg,
                                             double *U, double *H, double *AG,
                                             double *AU)
 {
-    return fwd_points(decode_f32_rows, X, Wg, Wu, K, idx_m, idx_n, count, G,
-                      U, H, AG, AU);
+    return fwd_points(decode_f32_rows, X, Wg, Wu, K, idx_m, idx_n, count, 0,
+                      1.0, G, U, H, AG, AU);
 }
 
 /* ---- dSwiGLU backward -------------------------------------------------- */
 
 /*
- * Elementwise backward of h = silu(g) * u with upstream gradient dh:
- *   dU = dh * silu(g)
- *   dG = dh * u * silu'(g)
- * (the "dSwiGLU" of Liger-Kernel issue #1383).
+ * Elementwise backward of h = act(alpha * g) * u with upstream gradient dh:
+ *   dU = dh * act(alpha g)
+ *   dG = dh * u * alpha * act'(alpha g)
+ * (the "dSwiGLU" of Liger-Kernel issue #1383 for act = SiLU, alpha = 1).
  */
-static void dswiglu_one(double dh, double g, double u, double *dg, double *du)
+static void dswiglu_one(double dh, double g, double u, int act, double alpha,
+                        double *dg, double *du)
 {
-    *du = dh * oracle_silu(g);
-    *dg = dh * u * oracle_dsilu(g);
+    *du = dh * oracle_act(alpha * g, act);
+    *dg = dh * u * alpha * oracle_dact(alpha * g, act);
 }
 
-/* n contiguous elements, double operands. */
+/* n contiguous elements, double operands, any activation / multiplier. */
+ORACLE_API void oracle_dswiglu_act_f64(const double *dH, const double *G,
+                                       const double *U, int64_t n, int act,
+                                       double alpha, double *dG, double *dU)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        dswiglu_one(dH[i], G[i], U[i], act, alpha, dG + i, dU + i);
+}
+
+/* The plain dSwiGLU, double operands. */
 ORACLE_API void oracle_dswiglu_f64(const double *dH, const double *G,
                                    const double *U, int64_t n, double *dG,
                                    double *dU)
 {
-#pragma omp parallel for schedule(static)
-    for (int64_t i = 0; i < n; ++i)
-        dswiglu_one(dH[i], G[i], U[i], dG + i, dU + i);
+    oracle_dswiglu_act_f64(dH, G, U, n, 0, 1.0, dG, dU);
 }
 
 /* Same, straight from bf16 bit patterns (full-size n is large). */
@@ -268,7 +347,7 @@ ORACLE_API void oracle_dswiglu_bf16(const uint16_t *dH, const uint16_t *G,
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i)
         dswiglu_one(bf16_bits_to_double(dH[i]), bf16_bits_to_double(G[i]),
-                    bf16_bits_to_double(U[i]), dG + i, dU + i);
+                    bf16_bits_to_double(U[i]), 0, 1.0, dG + i, dU + i);
 }
 
 /* Same, fp32 operands. */
@@ -278,5 +357,6 @@ ORACLE_API void oracle_dswiglu_f32(const float *dH, const float *G,
 {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i)
-        dswiglu_one((double)dH[i], (double)G[i], (double)U[i], dG + i, dU + i);
+        dswiglu_one((double)dH[i], (double)G[i], (double)U[i], 0, 1.0, dG + i,
+                    dU + i);
 }

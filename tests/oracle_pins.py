@@ -33,6 +33,16 @@ What pins what:
   dswiglu_special       dh = 0, u = 0, g = 0, g = +-40, g = x*.
   dswiglu_storage       the bf16 and fp32 entry points agree with the double
                         one on the decoded values.
+  gelu_closed_forms     GELU(tanh): value and slope at 0, the identity
+                        gelu(x) - gelu(-x) = x, the limits, torch's
+                        gelu(approximate="tanh") in float64 (an independent
+                        library routine), and gelu' against central differences.
+  variants_fwd          act(alpha g) u: G, U do not depend on the variant;
+                        H(Wg) - H(-Wg) = G U for GELU too (from its identity);
+                        H(alpha, Wg) = H(1, alpha Wg) for alpha a power of two
+                        (the multiplier acts on the gate pre-activation).
+  variants_bwd          dG, dU of the variants against central differences of
+                        the variant forward, and dU = dh act(alpha g).
 """
 from __future__ import annotations
 
@@ -280,7 +290,72 @@ def dswiglu_storage(o):
         assert np.array_equal(dG, dG2) and np.array_equal(dU, dU2), dtype
 
 
+def gelu_closed_forms(o):
+    assert o.gelu_tanh(0.0) == 0.0
+    assert o.dgelu_tanh(0.0) == 0.5
+    assert o.act(1.3, 1) == o.gelu_tanh(1.3) and o.act(1.3, 0) == o.silu(1.3)
+    assert abs(o.gelu_tanh(10.0) - 10.0) < 1e-15
+    assert abs(o.gelu_tanh(-10.0)) < 1e-15
+    xs = np.linspace(-8.0, 8.0, 161)
+    ref = torch.nn.functional.gelu(torch.from_numpy(xs), approximate="tanh").numpy()
+    for x, r in zip(xs, ref):
+        x = float(x)
+        assert abs(o.gelu_tanh(x) - r) <= 1e-15 * max(1.0, abs(x)), (x, o.gelu_tanh(x), r)
+        # gelu(x) - gelu(-x) = x  (the tanh factor is odd)
+        assert abs(o.gelu_tanh(x) - o.gelu_tanh(-x) - x) <= 1e-14 * max(1.0, abs(x)), x
+        h = 1e-5
+        fd = (o.gelu_tanh(x + h) - o.gelu_tanh(x - h)) / (2.0 * h)
+        assert abs(o.dgelu_tanh(x) - fd) < 1e-8, (x, o.dgelu_tanh(x), fd)
+        assert o.dact(x, 1) == o.dgelu_tanh(x) and o.dact(x, 0) == o.dsilu(x)
+
+
+def variants_fwd(o):
+    X, Wg, Wu = _random_problem(5, 64, 40, 90, scale_w=0.4)
+    base = o.swiglu_fwd_f64(X, Wg, Wu)
+    GU = (X @ Wg.T) * (X @ Wu.T)
+    scale = np.abs(X) @ np.abs(Wg).T * np.abs(X @ Wu.T) + 1e-300
+    for act in (0, 1):
+        v = o.swiglu_fwd_f64(X, Wg, Wu, act=act, alpha=1.0)
+        assert np.array_equal(v["G"], base["G"]) and np.array_equal(v["U"], base["U"])
+        if act == 0:
+            assert np.array_equal(v["H"], base["H"])
+        # act(g) - act(-g) = g for both activations
+        vn = o.swiglu_fwd_f64(X, -Wg, Wu, act=act)
+        assert np.all(np.abs((v["H"] - vn["H"]) - GU) <= 1e-12 * scale), act
+        for alpha in (2.0, 0.5, -4.0):
+            a = o.swiglu_fwd_f64(X, Wg, Wu, act=act, alpha=alpha)
+            b = o.swiglu_fwd_f64(X, alpha * Wg, Wu, act=act)
+            assert np.array_equal(a["H"], b["H"]), (act, alpha)
+            assert np.array_equal(a["G"], v["G"])   # G is stored before the multiplier
+    # a multiplier really changes H (it is not applied after the activation)
+    a = o.swiglu_fwd_f64(X, Wg, Wu, alpha=2.0)["H"]
+    assert np.max(np.abs(a - 2.0 * base["H"])) > 1e-3
+
+
+def variants_bwd(o):
+    r = _rng(95)
+    g = r.standard_normal(30) * 2.0
+    u = r.standard_normal(30)
+    dh = r.standard_normal(30)
+    d = 1e-6
+    for act in (0, 1):
+        for alpha in (1.0, 1.7, -0.6):
+            dG, dU = o.dswiglu_f64(dh, g, u, act=act, alpha=alpha)
+
+            def h(gg, uu):
+                return float(o.swiglu_fwd_f64(np.array([[1.0]]), np.array([[gg]]),
+                                              np.array([[uu]]), act=act, alpha=alpha)["H"][0, 0])
+            for i in range(g.size):
+                fdg = (h(g[i] + d, u[i]) - h(g[i] - d, u[i])) / (2 * d)
+                fdu = (h(g[i], u[i] + d) - h(g[i], u[i] - d)) / (2 * d)
+                sg = abs(dh[i]) * (abs(u[i]) + 1.0) * (abs(alpha) + 1.0)
+                assert abs(dG[i] - dh[i] * fdg) <= 3e-8 * sg, (act, alpha, i)
+                assert abs(dU[i] - dh[i] * fdu) <= 3e-8 * abs(dh[i]) * (abs(g[i] * alpha) + 1.0)
+                assert dU[i] == dh[i] * o.act(alpha * g[i], act)
+
+
 ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
             fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
             fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
-            dswiglu_special, dswiglu_storage]
+            dswiglu_special, dswiglu_storage, gelu_closed_forms, variants_fwd,
+            variants_bwd]

@@ -44,7 +44,8 @@ def test_tiny_config():
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
-@pytest.mark.parametrize("K,N", [(256, 512), (264, 72), (8, 8), (1536, 6912), (40, 1032)])
+@pytest.mark.parametrize("K,N", [(256, 512), (264, 72), (8, 8), (1536, 6912), (40, 1032),
+                                 (5000, 264)])
 def test_decode_shapes(M, K, N):
     X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 1000 + K)
     check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"decode M={M} K={K} N={N}")
@@ -152,7 +153,8 @@ def test_decode_astrai_full_size_rotated_copies():
             assert_bf16_close(f64(H), ref, f"astrai M={M} copy={r}")
 
 
-@pytest.mark.parametrize("K,N", [(1536, 6912), (4096, 11008), (256, 512)])
+@pytest.mark.parametrize("K,N", [(1536, 6912), (4096, 11008), (256, 512), (5000, 264),
+                                 (8, 8), (264, 72)])
 def test_decode_weights_stable_path(K, N):
     """The programmatic-dependent-launch path (weights prefetched before the
     preceding kernel finishes) gives oracle-exact-within-tolerance results."""

@@ -18,14 +18,25 @@ MUTANTS = [
     ("reversed_weight_index",
      "double pg = x[k] * wg[k];", "double pg = x[k] * wg[K - 1 - k];"),
     ("gate_up_swapped",
-     "if (h_out) *h_out = oracle_silu(g) * u;",
-     "if (h_out) *h_out = oracle_silu(u) * g;"),
+     "if (h_out) *h_out = oracle_act(alpha * g, act) * u;",
+     "if (h_out) *h_out = oracle_act(alpha * u, act) * g;"),
+    ("multiplier_after_activation",
+     "if (h_out) *h_out = oracle_act(alpha * g, act) * u;",
+     "if (h_out) *h_out = alpha * oracle_act(g, act) * u;"),
+    ("gelu_sign",
+     "return 0.5 * x * (1.0 + t);", "return 0.5 * x * (1.0 - t);"),
+    ("gelu_slope_cubic_term",
+     "double dy = ORACLE_GELU_C * (1.0 + 3.0 * ORACLE_GELU_A * x * x);",
+     "double dy = ORACLE_GELU_C * (1.0 + ORACLE_GELU_A * x * x);"),
+    ("dG_missing_multiplier",
+     "*dg = dh * u * alpha * oracle_dact(alpha * g, act);",
+     "*dg = dh * u * oracle_dact(alpha * g, act);"),
     ("sigmoid_sign",
      "return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
     ("dsilu_sign",
      "return s * (1.0 + x * (1.0 - s));", "return s * (1.0 - x * (1.0 - s));"),
     ("dU_uses_up_operand",
-     "*du = dh * oracle_silu(g);", "*du = dh * oracle_silu(u);"),
+     "*du = dh * oracle_act(alpha * g, act);", "*du = dh * oracle_act(alpha * u, act);"),
     ("wrong_weight_row",
      "one_output(X + m * K, Wg + n * K, Wu + n * K, K,",
      "one_output(X + m * K, Wg + ((n + 1) % N) * K, Wu + n * K, K,"),
