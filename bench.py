@@ -319,7 +319,10 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
 
 def run_extras(stream, pk):
     """Single-GPU extra measurements (rank 0 only)."""
+    import ctypes
+
     import up_projection_b200 as up
+    from up_projection_b200 import _capi as up_capi
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
     gen.manual_seed(1)
@@ -347,7 +350,29 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
-    del X, Wg, Wu, H
+    # training forward: the same call also storing G and U for the backward
+    Gs = torch.empty_like(H)
+    Us = torch.empty_like(H)
+    ms = time_op(lambda: up.lib().swiglu_fwd_epilogue(
+        X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(), M, K, N, 0,
+        ctypes.byref(up_capi.Epilogue(0, 1.0, Gs.data_ptr(), Us.data_ptr())), 0,
+        stream.cuda_stream))
+    tf = fl / (ms * 1e-3) / 1e12
+    res.append({"workload": "prefill training forward (also stores G, U) LLaMA-3 8B bf16",
+                "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(tf / pk["bf16_tflops"], 4)}})
+    # GEGLU (GELU-tanh) epilogue with a gate multiplier
+    ms = time_op(lambda: up.swiglu_fwd(X, Wg, Wu, H, stream=stream,
+                                       activation=up.SWIGLU_ACT_GELU_TANH, gate_multiplier=1.5))
+    tf = fl / (ms * 1e-3) / 1e12
+    res.append({"workload": "prefill GEGLU (GELU-tanh, gate multiplier 1.5) LLaMA-3 8B bf16",
+                "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(tf / pk["bf16_tflops"], 4)}})
+    del X, Wg, Wu, H, Gs, Us
     # dSwiGLU on [8192, 14336] bf16
     n = 8192 * 14336
     dH = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)

@@ -70,8 +70,32 @@ enum swiglu_status {
     SWIGLU_ERR_TIMEOUT = 8,          /* a device-side bounded wait gave up  */
     SWIGLU_ERR_OVERLAP = 9,          /* an output overlaps an input         */
     SWIGLU_ERR_NO_DEVICE = 10,       /* no CUDA device is usable            */
-    SWIGLU_ERR_BAD_FLAGS = 11        /* unknown bit in swiglu_fwd_ex flags  */
+    SWIGLU_ERR_BAD_FLAGS = 11,       /* unknown bit in swiglu_fwd_ex flags  */
+    SWIGLU_ERR_BAD_EPILOGUE = 12     /* unknown activation, non-finite gate
+                                        multiplier, or only one of G/U     */
 };
+
+/* Gate activations of the epilogue variants, h = act(alpha * g) * u. */
+enum swiglu_activation {
+    SWIGLU_ACT_SILU = 0,      /* SwiGLU: silu(x) = x * sigmoid(x)            */
+    SWIGLU_ACT_GELU_TANH = 1  /* GEGLU: x/2 (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3))) */
+};
+
+/*
+ * Epilogue variant of swiglu_fwd_epilogue (Liger-Kernel issue #937: the
+ * swiglu/geglu activations and the scalar gate multiplier fused into the
+ * GEMM epilogue; TensorRT-LLM PR #17693: GELU(tanh) on the fp32
+ * accumulator).  The multiplier scales the gate pre-activation.
+ */
+typedef struct swiglu_epilogue {
+    int activation;        /* swiglu_activation                            */
+    float gate_multiplier; /* alpha; 1.0f for none                         */
+    void *G;               /* NULL, or [M, N] device output, dtype: the
+                              gate projection X Wg^T (before alpha)        */
+    void *U;               /* NULL, or [M, N] device output: X Wu^T.  G and
+                              U are given together (training forward: the
+                              backward needs them) or not at all           */
+} swiglu_epilogue;
 
 /* Flags of swiglu_fwd_ex. */
 enum swiglu_flags {
@@ -126,6 +150,18 @@ SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu,
                              cudaStream_t stream);
 
 /*
+ * swiglu_fwd_epilogue -- H = act(alpha * (X Wg^T)) (.) (X Wu^T), optionally
+ * also storing G = X Wg^T and U = X Wu^T (each rounded once to dtype from
+ * the fp32 accumulator).  `epi` may be NULL (SiLU, alpha = 1, no G/U, i.e.
+ * swiglu_fwd_ex).  G and U follow H's rules: 16-byte aligned, no overlap
+ * with any input, with H or with each other.  Same routes as swiglu_fwd.
+ */
+SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu,
+                                   void *H, int64_t M, int64_t K, int64_t N,
+                                   int dtype, const swiglu_epilogue *epi,
+                                   unsigned int flags, cudaStream_t stream);
+
+/*
  * dswiglu_bwd -- elementwise dSwiGLU, bf16.
  *
  *  dH, G, U  [n] device bf16 inputs, 16-byte aligned.
@@ -141,6 +177,17 @@ SWIGLU_API int dswiglu_bwd(const void *dH, const void *G, const void *U,
 SWIGLU_API int dswiglu_bwd_dtype(const void *dH, const void *G, const void *U,
                                  void *dG, void *dU, int64_t n, int dtype,
                                  cudaStream_t stream);
+
+/*
+ * dswiglu_bwd_epilogue -- backward of the epilogue variants:
+ *   dU = dH (.) act(alpha G),   dG = dH (.) U (.) alpha act'(alpha G).
+ * activation SWIGLU_ACT_SILU with gate_multiplier 1 is dswiglu_bwd_dtype.
+ * Same buffer rules as dswiglu_bwd.
+ */
+SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U,
+                                    void *dG, void *dU, int64_t n, int dtype,
+                                    int activation, float gate_multiplier,
+                                    cudaStream_t stream);
 
 /* Route swiglu_fwd takes for these arguments (pure host function; returns a
  * swiglu_route, or -1 for arguments swiglu_fwd would reject). */

@@ -89,7 +89,33 @@ def test_unknown_flags_rejected():
         _capi.SWIGLU_ERR_NULL_POINTER
 
 
+def test_epilogue_validation():
+    import ctypes
+    lib = _capi.lib()
+    args = (1 << 20, 1 << 21, 1 << 22, 1 << 23, 4, 64, 64, 0)
+    bad_act = _capi.Epilogue(7, 1.0, None, None)
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(bad_act), 0, None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+    nan_mult = _capi.Epilogue(0, float("nan"), None, None)
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(nan_mult), 0, None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+    only_g = _capi.Epilogue(0, 1.0, 1 << 24, None)
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(only_g), 0, None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+    misaligned = _capi.Epilogue(0, 1.0, (1 << 24) + 8, 1 << 25)
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(misaligned), 0, None) == \
+        _capi.SWIGLU_ERR_MISALIGNED_PTR
+    g_on_h = _capi.Epilogue(0, 1.0, 1 << 23, 1 << 25)   # G == H
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(g_on_h), 0, None) == _capi.SWIGLU_ERR_OVERLAP
+    g_on_x = _capi.Epilogue(0, 1.0, 1 << 20, 1 << 25)   # G == X
+    assert lib.swiglu_fwd_epilogue(*args, ctypes.byref(g_on_x), 0, None) == _capi.SWIGLU_ERR_OVERLAP
+    assert lib.dswiglu_bwd_epilogue(16, 32, 48, 64, 80, 10, 0, 5, 1.0, None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+    assert lib.dswiglu_bwd_epilogue(16, 32, 48, 64, 80, 10, 0, 1, float("inf"), None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+
+
 def test_status_strings():
-    for code in range(12):
+    for code in range(13):
         assert _capi.status_string(code)
     assert _capi.status_string(999) == "unknown status"

@@ -31,6 +31,10 @@ SWIGLU_ERR_TIMEOUT = 8
 SWIGLU_ERR_OVERLAP = 9
 SWIGLU_ERR_NO_DEVICE = 10
 SWIGLU_ERR_BAD_FLAGS = 11
+SWIGLU_ERR_BAD_EPILOGUE = 12
+# enum swiglu_activation
+SWIGLU_ACT_SILU = 0
+SWIGLU_ACT_GELU_TANH = 1
 # enum swiglu_flags
 SWIGLU_FLAG_WEIGHTS_STABLE = 1
 # enum swiglu_route
@@ -44,10 +48,20 @@ _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I = ctypes.c_int
 
+
+class Epilogue(ctypes.Structure):
+    """struct swiglu_epilogue."""
+    _fields_ = [("activation", ctypes.c_int), ("gate_multiplier", ctypes.c_float),
+                ("G", ctypes.c_void_p), ("U", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes), mirroring include/swiglu.h
 SIGNATURES = {
     "swiglu_fwd": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_fwd_ex": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, ctypes.c_uint, _P]),
+    "swiglu_fwd_epilogue": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, ctypes.POINTER(Epilogue),
+                                 ctypes.c_uint, _P]),
+    "dswiglu_bwd_epilogue": (_I, [_P, _P, _P, _P, _P, _I64, _I, _I, ctypes.c_float, _P]),
     "dswiglu_bwd": (_I, [_P, _P, _P, _P, _P, _I64, _P]),
     "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
@@ -121,14 +135,20 @@ def _dev(t: torch.Tensor, name: str):
 
 def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
                H: torch.Tensor | None = None, stream=None,
-               weights_stable: bool = False) -> torch.Tensor:
+               weights_stable: bool = False, activation: int = SWIGLU_ACT_SILU,
+               gate_multiplier: float = 1.0, return_gu: bool = False):
     """H = silu(X Wg^T) * (X Wu^T) through the C ABI.  X [..., K] (leading
     dims are flattened to M rows, as the TensorRT-LLM fused up-projection
     does), Wg/Wu [N, K]; bf16 or fp32, all contiguous on one GPU.
 
     weights_stable=True promises that no earlier work on the stream writes
     Wg or Wu (SWIGLU_FLAG_WEIGHTS_STABLE): the decode kernel may then start
-    streaming them while the preceding kernel finishes."""
+    streaming them while the preceding kernel finishes.
+
+    activation / gate_multiplier select the epilogue variant
+    H = act(gate_multiplier * G) * U (SWIGLU_ACT_SILU or
+    SWIGLU_ACT_GELU_TANH).  return_gu=True also stores G = X Wg^T and
+    U = X Wu^T (training forward) and returns (H, G, U)."""
     for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
         _dev(t, n)
     if not (X.dtype == Wg.dtype == Wu.dtype):
@@ -148,16 +168,29 @@ def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
         if H.dtype != X.dtype or H.numel() != M * N:
             raise ValueError("H has the wrong dtype or size")
     flags = SWIGLU_FLAG_WEIGHTS_STABLE if weights_stable else 0
-    st = lib().swiglu_fwd_ex(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
-                             M, K, N, _dtype_code(X), flags, _stream(stream))
+    G = U = None
+    if return_gu:
+        G = torch.empty_like(H)
+        U = torch.empty_like(H)
+    if activation == SWIGLU_ACT_SILU and gate_multiplier == 1.0 and not return_gu:
+        st = lib().swiglu_fwd_ex(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
+                                 M, K, N, _dtype_code(X), flags, _stream(stream))
+    else:
+        epi = Epilogue(int(activation), float(gate_multiplier),
+                       G.data_ptr() if G is not None else None,
+                       U.data_ptr() if U is not None else None)
+        st = lib().swiglu_fwd_epilogue(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
+                                       M, K, N, _dtype_code(X), ctypes.byref(epi), flags,
+                                       _stream(stream))
     _check("swiglu_fwd", st)
-    return H
+    return (H, G, U) if return_gu else H
 
 
 def dswiglu_bwd(dH: torch.Tensor, G: torch.Tensor, U: torch.Tensor,
                 dG: torch.Tensor | None = None, dU: torch.Tensor | None = None,
-                stream=None):
-    """(dG, dU) of h = silu(g) * u through the C ABI (bf16 or fp32)."""
+                stream=None, activation: int = SWIGLU_ACT_SILU, gate_multiplier: float = 1.0):
+    """(dG, dU) of h = act(gate_multiplier g) * u through the C ABI (bf16 or
+    fp32); the defaults are the plain dSwiGLU."""
     for t, n in ((dH, "dH"), (G, "G"), (U, "U")):
         _dev(t, n)
     if not (dH.dtype == G.dtype == U.dtype) or dH.shape != G.shape or G.shape != U.shape:
@@ -166,8 +199,9 @@ def dswiglu_bwd(dH: torch.Tensor, G: torch.Tensor, U: torch.Tensor,
     dU = torch.empty_like(U) if dU is None else dU
     _dev(dG, "dG")
     _dev(dU, "dU")
-    st = lib().dswiglu_bwd_dtype(dH.data_ptr(), G.data_ptr(), U.data_ptr(), dG.data_ptr(),
-                                 dU.data_ptr(), G.numel(), _dtype_code(G), _stream(stream))
+    st = lib().dswiglu_bwd_epilogue(dH.data_ptr(), G.data_ptr(), U.data_ptr(), dG.data_ptr(),
+                                    dU.data_ptr(), G.numel(), _dtype_code(G), int(activation),
+                                    float(gate_multiplier), _stream(stream))
     _check("dswiglu_bwd", st)
     return dG, dU
 

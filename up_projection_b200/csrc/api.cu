@@ -6,6 +6,7 @@
 // fallback: when no usable sm_100 device is current, calls fail with
 // SWIGLU_ERR_NO_DEVICE / SWIGLU_ERR_UNSUPPORTED_DEVICE.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -105,6 +106,30 @@ int check_fwd(const void *X, const void *Wg, const void *Wu, const void *H, int6
     return SWIGLU_OK;
 }
 
+// Epilogue checks (G/U buffers against the forward's buffers).
+int check_epilogue(const swiglu_epilogue *epi, const void *X, const void *Wg, const void *Wu,
+                   const void *H, int64_t M, int64_t K, int64_t N, int dtype, int route) {
+    if (!epi) return SWIGLU_OK;
+    if (epi->activation != SWIGLU_ACT_SILU && epi->activation != SWIGLU_ACT_GELU_TANH)
+        return SWIGLU_ERR_BAD_EPILOGUE;
+    if (!isfinite(epi->gate_multiplier)) return SWIGLU_ERR_BAD_EPILOGUE;
+    if ((epi->G == nullptr) != (epi->U == nullptr)) return SWIGLU_ERR_BAD_EPILOGUE;
+    if (!epi->G || route == SWIGLU_ROUTE_NONE) return SWIGLU_OK;
+    if (!aligned16(epi->G) || !aligned16(epi->U)) return SWIGLU_ERR_MISALIGNED_PTR;
+    const int es = elem_size(dtype);
+    const int64_t ob = M * N * es;
+    if (overlaps(epi->G, ob, epi->U, ob) || overlaps(epi->G, ob, H, ob) || overlaps(epi->U, ob, H, ob))
+        return SWIGLU_ERR_OVERLAP;
+    if (route != SWIGLU_ROUTE_ZERO_K) {
+        const int64_t xb = M * K * es, wb = N * K * es;
+        const void *outs[2] = {epi->G, epi->U};
+        for (const void *o : outs)
+            if (overlaps(o, ob, X, xb) || overlaps(o, ob, Wg, wb) || overlaps(o, ob, Wu, wb))
+                return SWIGLU_ERR_OVERLAP;
+    }
+    return SWIGLU_OK;
+}
+
 int check_bwd(const void *dH, const void *G, const void *U, const void *dG, const void *dU,
               int64_t n, int dtype) {
     if (dtype != SWIGLU_BF16 && dtype != SWIGLU_FP32) return SWIGLU_ERR_BAD_DTYPE;
@@ -151,10 +176,26 @@ SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu, void *H
 SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu, void *H, int64_t M,
                              int64_t K, int64_t N, int dtype, unsigned int flags,
                              cudaStream_t stream) {
+    return swiglu_fwd_epilogue(X, Wg, Wu, H, M, K, N, dtype, nullptr, flags, stream);
+}
+
+SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu, void *H,
+                                   int64_t M, int64_t K, int64_t N, int dtype,
+                                   const swiglu_epilogue *epi, unsigned int flags,
+                                   cudaStream_t stream) {
     if (flags & ~static_cast<unsigned int>(SWIGLU_FLAG_WEIGHTS_STABLE)) return SWIGLU_ERR_BAD_FLAGS;
     int route = SWIGLU_ROUTE_NONE;
     int st = check_fwd(X, Wg, Wu, H, M, K, N, dtype, &route);
     if (st != SWIGLU_OK) return st;
+    st = check_epilogue(epi, X, Wg, Wu, H, M, K, N, dtype, route);
+    if (st != SWIGLU_OK) return st;
+    Epilogue ep;
+    if (epi) {
+        ep.activation = epi->activation;
+        ep.gate_multiplier = epi->gate_multiplier;
+        ep.G = epi->G;
+        ep.U = epi->U;
+    }
     if (route == SWIGLU_ROUTE_NONE) {
         t_last_route = route;
         return SWIGLU_OK;
@@ -165,18 +206,23 @@ SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu, void
     const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
     cudaError_t e = cudaSuccess;
     switch (route) {
-        case SWIGLU_ROUTE_ZERO_K:
-            e = cudaMemsetAsync(H, 0, static_cast<size_t>(M) * N * elem_size(dtype), stream);
+        case SWIGLU_ROUTE_ZERO_K: {
+            // G = U = 0 and act(0) = 0 for both activations, so H = 0.
+            const size_t bytes = static_cast<size_t>(M) * N * elem_size(dtype);
+            e = cudaMemsetAsync(H, 0, bytes, stream);
+            if (e == cudaSuccess && ep.G) e = cudaMemsetAsync(ep.G, 0, bytes, stream);
+            if (e == cudaSuccess && ep.U) e = cudaMemsetAsync(ep.U, 0, bytes, stream);
             break;
+        }
         case SWIGLU_ROUTE_DECODE_BF16:
-            e = launch_decode_bf16(X, Wg, Wu, H, m, k, n, (flags & SWIGLU_FLAG_WEIGHTS_STABLE) != 0,
-                                   dev, stream);
+            e = launch_decode_bf16(X, Wg, Wu, H, m, k, n, ep,
+                                   (flags & SWIGLU_FLAG_WEIGHTS_STABLE) != 0, dev, stream);
             break;
         case SWIGLU_ROUTE_GEMM_BF16:
-            e = launch_gemm_bf16(X, Wg, Wu, H, m, k, n, dev, stream);
+            e = launch_gemm_bf16(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             break;
         case SWIGLU_ROUTE_GEMM_TF32X3:
-            e = launch_gemm_tf32x3(X, Wg, Wu, H, m, k, n, dev, stream);
+            e = launch_gemm_tf32x3(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             break;
         default:
             return SWIGLU_ERR_BAD_DTYPE;
@@ -186,14 +232,24 @@ SWIGLU_API int swiglu_fwd_ex(const void *X, const void *Wg, const void *Wu, void
     return st;
 }
 
-SWIGLU_API int dswiglu_bwd_dtype(const void *dH, const void *G, const void *U, void *dG,
-                                 void *dU, int64_t n, int dtype, cudaStream_t stream) {
+SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U, void *dG,
+                                    void *dU, int64_t n, int dtype, int activation,
+                                    float gate_multiplier, cudaStream_t stream) {
+    if (activation != SWIGLU_ACT_SILU && activation != SWIGLU_ACT_GELU_TANH)
+        return SWIGLU_ERR_BAD_EPILOGUE;
+    if (!isfinite(gate_multiplier)) return SWIGLU_ERR_BAD_EPILOGUE;
     int st = check_bwd(dH, G, U, dG, dU, n, dtype);
     if (st != SWIGLU_OK || n == 0) return st;
     DeviceInfo dev;
     st = current_device(dev);
     if (st != SWIGLU_OK) return st;
-    return from_cuda(launch_dswiglu(dH, G, U, dG, dU, n, dtype == SWIGLU_BF16 ? 0 : 1, dev, stream));
+    return from_cuda(launch_dswiglu(dH, G, U, dG, dU, n, dtype == SWIGLU_BF16 ? 0 : 1, activation,
+                                    gate_multiplier, dev, stream));
+}
+
+SWIGLU_API int dswiglu_bwd_dtype(const void *dH, const void *G, const void *U, void *dG,
+                                 void *dU, int64_t n, int dtype, cudaStream_t stream) {
+    return dswiglu_bwd_epilogue(dH, G, U, dG, dU, n, dtype, SWIGLU_ACT_SILU, 1.0f, stream);
 }
 
 SWIGLU_API int dswiglu_bwd(const void *dH, const void *G, const void *U, void *dG, void *dU,
@@ -217,6 +273,7 @@ SWIGLU_API const char *swiglu_status_string(int status) {
         case SWIGLU_ERR_OVERLAP: return "output overlaps an input";
         case SWIGLU_ERR_NO_DEVICE: return "no usable CUDA device";
         case SWIGLU_ERR_BAD_FLAGS: return "unknown flag bit";
+        case SWIGLU_ERR_BAD_EPILOGUE: return "bad epilogue (activation, multiplier or G/U pair)";
         default: return "unknown status";
     }
 }

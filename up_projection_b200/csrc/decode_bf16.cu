@@ -34,6 +34,7 @@
 
 #include <atomic>
 
+#include "activation.cuh"
 #include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -140,16 +141,15 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], uint32_t a0, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float silu_mul_fast(float g, float u) {
-    return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
 
 __global__ void __launch_bounds__(kThreads, 2)
     swiglu_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_wg,
                               const __grid_constant__ CUtensorMap tm_wu,
                               const __nv_bfloat16 *__restrict__ X,
                               __nv_bfloat16 *__restrict__ H, int M, int K, int N,
-                              int weights_stable, int budget) {
+                              int weights_stable, int budget, int which_act, float alpha,
+                              __nv_bfloat16 *__restrict__ Gout,
+                              __nv_bfloat16 *__restrict__ Uout) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Geometry geo = geometry(K, budget);
     // Under programmatic dependent launch the next call may be scheduled as
@@ -337,12 +337,18 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (lane == 0) mbar_arrive(bar_red_empty);
                 // s4[0], s4[1]: gate at m = 2*tig, 2*tig+1; s4[2], s4[3]: up.
                 const int n = u * 8 + grp;
-                const int m0 = 2 * tig;
-                if (m0 < M)
-                    H[static_cast<size_t>(m0) * N + n] = __float2bfloat16_rn(silu_mul_fast(s4[0], s4[2]));
-                if (m0 + 1 < M)
-                    H[static_cast<size_t>(m0 + 1) * N + n] =
-                        __float2bfloat16_rn(silu_mul_fast(s4[1], s4[3]));
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int m = 2 * tig + q;
+                    if (m < M) {
+                        const size_t o = static_cast<size_t>(m) * N + n;
+                        H[o] = __float2bfloat16_rn(act::gated<false>(which_act, alpha, s4[q], s4[2 + q]));
+                        if (Gout) {
+                            Gout[o] = __float2bfloat16_rn(s4[q]);
+                            Uout[o] = __float2bfloat16_rn(s4[2 + q]);
+                        }
+                    }
+                }
             }
         }
     }
@@ -359,8 +365,8 @@ bool decode_bf16_supported(int K) {
 }
 
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
-                               int K, int N, bool weights_stable, const DeviceInfo &dev,
-                               cudaStream_t stream) {
+                               int K, int N, const Epilogue &epi, bool weights_stable,
+                               const DeviceInfo &dev, cudaStream_t stream) {
     const int budget = decode_budget(K, weights_stable);
     const Geometry geo = geometry(K, budget);
     if (!geo.ok) return cudaErrorInvalidValue;
@@ -402,8 +408,12 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
     const __nv_bfloat16 *xp = static_cast<const __nv_bfloat16 *>(X);
     __nv_bfloat16 *hp = static_cast<__nv_bfloat16 *>(H);
     const int ws = weights_stable ? 1 : 0;
+    const int which_act = epi.activation;
+    const float alpha = epi.gate_multiplier;
+    __nv_bfloat16 *gp = static_cast<__nv_bfloat16 *>(epi.G);
+    __nv_bfloat16 *up = static_cast<__nv_bfloat16 *>(epi.U);
     cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_decode_bf16_kernel, tg, tu, xp, hp, M, K, N,
-                                       ws, budget);
+                                       ws, budget, which_act, alpha, gp, up);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -2,7 +2,9 @@
 // issue #1383) and the bench-only read-floor probe.
 //
 //   dU = dH * silu(G),   dG = dH * U * silu'(G),
-//   silu(g) = g s,  silu'(g) = s (1 + g (1 - s)),  s = sigmoid(g).
+//   silu(g) = g s,  silu'(g) = s (1 + g (1 - s)),  s = sigmoid(g);
+// and for the epilogue variants h = act(alpha g) u (GELU(tanh), a gate
+// multiplier): dU = dH act(alpha G), dG = dH U alpha act'(alpha G).
 //
 // HBM-bound (3 loads + 2 stores per element): 128-bit vector accesses,
 // L1-bypassing loads, streaming stores, a grid of a few CTAs per SM looping
@@ -13,6 +15,7 @@
 // hardware approximations, far below the bf16 output rounding.
 #include <cuda_bf16.h>
 
+#include "activation.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -25,25 +28,16 @@ constexpr int kThreads = 256;
 constexpr int kBlocksPerSm = 8;
 constexpr int kUnroll = 2;
 
+// dU = dh * act(alpha g),  dG = dh * u * alpha * act'(alpha g).  `which` is
+// a compile-time constant at every call (the kernel is instantiated per
+// activation), so the other activation's code folds away.
 template <bool kFast>
-__device__ __forceinline__ void dswiglu_elem(float dh, float g, float u, float &dg, float &du) {
-    const float a = fabsf(g);
-    float t, r;
-    if (kFast) {
-        t = __expf(-a);
-        r = __frcp_rn(1.0f + t);
-    } else {
-        t = expf(-a);
-        r = 1.0f / (1.0f + t);
-    }
-    const float tr = t * r;
-    const bool pos = g >= 0.0f;
-    const float s = pos ? r : tr;      // sigmoid(g)
-    const float oms = pos ? tr : r;    // 1 - sigmoid(g)
-    const float silu = g * s;
-    const float dsilu = s * (1.0f + g * oms);
-    du = dh * silu;
-    dg = dh * u * dsilu;
+__device__ __forceinline__ void dswiglu_elem(int which, float alpha, float dh, float g, float u,
+                                             float &dg, float &du) {
+    float a, da;
+    act::value_and_slope<!kFast>(which, alpha * g, a, da);
+    du = dh * a;
+    dg = dh * u * alpha * da;
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -55,40 +49,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // One 16-byte vector of each operand: 8 bf16 elements.
-__device__ __forceinline__ void vec_bf16(const uint4 &dh, const uint4 &g, const uint4 &u,
-                                         uint4 &dg, uint4 &du) {
+__device__ __forceinline__ void vec_bf16(int which, float alpha, const uint4 &dh, const uint4 &g,
+                                         const uint4 &u, uint4 &dg, uint4 &du) {
     const uint32_t *pdh = &dh.x, *pg = &g.x, *pu = &u.x;
     uint32_t *pdg = &dg.x, *pdu = &du.x;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float g0, u0, g1, u1;
-        dswiglu_elem<true>(bf_lo(pdh[i]), bf_lo(pg[i]), bf_lo(pu[i]), g0, u0);
-        dswiglu_elem<true>(bf_hi(pdh[i]), bf_hi(pg[i]), bf_hi(pu[i]), g1, u1);
+        dswiglu_elem<true>(which, alpha, bf_lo(pdh[i]), bf_lo(pg[i]), bf_lo(pu[i]), g0, u0);
+        dswiglu_elem<true>(which, alpha, bf_hi(pdh[i]), bf_hi(pg[i]), bf_hi(pu[i]), g1, u1);
         pdg[i] = pack_bf16x2(g0, g1);
         pdu[i] = pack_bf16x2(u0, u1);
     }
 }
 
 // 4 fp32 elements.
-__device__ __forceinline__ void vec_f32(const uint4 &dh, const uint4 &g, const uint4 &u,
-                                        uint4 &dg, uint4 &du) {
+__device__ __forceinline__ void vec_f32(int which, float alpha, const uint4 &dh, const uint4 &g,
+                                        const uint4 &u, uint4 &dg, uint4 &du) {
     const uint32_t *pdh = &dh.x, *pg = &g.x, *pu = &u.x;
     uint32_t *pdg = &dg.x, *pdu = &du.x;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float a, b;
-        dswiglu_elem<false>(__uint_as_float(pdh[i]), __uint_as_float(pg[i]),
+        dswiglu_elem<false>(which, alpha, __uint_as_float(pdh[i]), __uint_as_float(pg[i]),
                             __uint_as_float(pu[i]), a, b);
         pdg[i] = __float_as_uint(a);
         pdu[i] = __float_as_uint(b);
     }
 }
 
-template <bool kBf16>
+template <bool kBf16, int kAct>
 __global__ void __launch_bounds__(kThreads)
     dswiglu_kernel(const uint4 *dH, const uint4 *G, const uint4 *U, uint4 *dG, uint4 *dU,
                    int64_t nvec, const void *dH_tail, const void *G_tail, const void *U_tail,
-                   void *dG_tail, void *dU_tail, int tail) {
+                   void *dG_tail, void *dU_tail, int tail, float alpha) {
+    constexpr int which = kAct;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     for (; i + (kUnroll - 1) * stride < nvec; i += kUnroll * stride) {
@@ -102,8 +97,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int j = 0; j < kUnroll; ++j) {
             uint4 og, ou;
-            if (kBf16) vec_bf16(a[j], b[j], c[j], og, ou);
-            else vec_f32(a[j], b[j], c[j], og, ou);
+            if (kBf16) vec_bf16(which, alpha, a[j], b[j], c[j], og, ou);
+            else vec_f32(which, alpha, a[j], b[j], c[j], og, ou);
             st_stream_v4(dG + i + j * stride, og);
             st_stream_v4(dU + i + j * stride, ou);
         }
@@ -111,8 +106,8 @@ __global__ void __launch_bounds__(kThreads)
     for (; i < nvec; i += stride) {
         const uint4 a = ld_stream_v4(dH + i), b = ld_stream_v4(G + i), c = ld_stream_v4(U + i);
         uint4 og, ou;
-        if (kBf16) vec_bf16(a, b, c, og, ou);
-        else vec_f32(a, b, c, og, ou);
+        if (kBf16) vec_bf16(which, alpha, a, b, c, og, ou);
+        else vec_f32(which, alpha, a, b, c, og, ou);
         st_stream_v4(dG + i, og);
         st_stream_v4(dU + i, ou);
     }
@@ -124,7 +119,7 @@ __global__ void __launch_bounds__(kThreads)
             const __nv_bfloat16 *pg = static_cast<const __nv_bfloat16 *>(G_tail);
             const __nv_bfloat16 *pu = static_cast<const __nv_bfloat16 *>(U_tail);
             float og, ou;
-            dswiglu_elem<true>(__bfloat162float(pdh[j]), __bfloat162float(pg[j]),
+            dswiglu_elem<true>(which, alpha, __bfloat162float(pdh[j]), __bfloat162float(pg[j]),
                                __bfloat162float(pu[j]), og, ou);
             static_cast<__nv_bfloat16 *>(dG_tail)[j] = __float2bfloat16_rn(og);
             static_cast<__nv_bfloat16 *>(dU_tail)[j] = __float2bfloat16_rn(ou);
@@ -133,7 +128,7 @@ __global__ void __launch_bounds__(kThreads)
             const float *pg = static_cast<const float *>(G_tail);
             const float *pu = static_cast<const float *>(U_tail);
             float og, ou;
-            dswiglu_elem<false>(pdh[j], pg[j], pu[j], og, ou);
+            dswiglu_elem<false>(which, alpha, pdh[j], pg[j], pu[j], og, ou);
             static_cast<float *>(dG_tail)[j] = og;
             static_cast<float *>(dU_tail)[j] = ou;
         }
@@ -181,7 +176,8 @@ __global__ void __launch_bounds__(kProbeThreads)
 }  // namespace
 
 cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG, void *dU,
-                           int64_t n, int dtype, const DeviceInfo &dev, cudaStream_t stream) {
+                           int64_t n, int dtype, int activation, float alpha,
+                           const DeviceInfo &dev, cudaStream_t stream) {
     const int per_vec = dtype == 0 ? 8 : 4;
     const int esize = dtype == 0 ? 2 : 4;
     const int64_t nvec = n / per_vec;
@@ -196,17 +192,23 @@ cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *d
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * kBlocksPerSm;
     int grid = static_cast<int>(want_blocks < cap ? want_blocks : cap);
     if (grid < 1) grid = 1;
-    if (dtype == 0) {
-        dswiglu_kernel<true><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint4 *>(dH), static_cast<const uint4 *>(G),
-            static_cast<const uint4 *>(U), static_cast<uint4 *>(dG), static_cast<uint4 *>(dU), nvec,
-            tdh, tg, tu, tdg, tdu, tail);
-    } else {
-        dswiglu_kernel<false><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint4 *>(dH), static_cast<const uint4 *>(G),
-            static_cast<const uint4 *>(U), static_cast<uint4 *>(dG), static_cast<uint4 *>(dU), nvec,
-            tdh, tg, tu, tdg, tdu, tail);
-    }
+    const uint4 *a = static_cast<const uint4 *>(dH);
+    const uint4 *b = static_cast<const uint4 *>(G);
+    const uint4 *c = static_cast<const uint4 *>(U);
+    uint4 *og = static_cast<uint4 *>(dG);
+    uint4 *ou = static_cast<uint4 *>(dU);
+    if (dtype == 0 && activation == act::kGeluTanh)
+        dswiglu_kernel<true, act::kGeluTanh><<<grid, kThreads, 0, stream>>>(
+            a, b, c, og, ou, nvec, tdh, tg, tu, tdg, tdu, tail, alpha);
+    else if (dtype == 0)
+        dswiglu_kernel<true, act::kSilu><<<grid, kThreads, 0, stream>>>(
+            a, b, c, og, ou, nvec, tdh, tg, tu, tdg, tdu, tail, alpha);
+    else if (activation == act::kGeluTanh)
+        dswiglu_kernel<false, act::kGeluTanh><<<grid, kThreads, 0, stream>>>(
+            a, b, c, og, ou, nvec, tdh, tg, tu, tdg, tdu, tail, alpha);
+    else
+        dswiglu_kernel<false, act::kSilu><<<grid, kThreads, 0, stream>>>(
+            a, b, c, og, ou, nvec, tdh, tg, tu, tdg, tdu, tail, alpha);
     return cudaGetLastError();
 }
 

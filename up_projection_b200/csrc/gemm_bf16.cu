@@ -30,6 +30,7 @@
 
 #include <atomic>
 
+#include "activation.cuh"
 #include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -74,10 +75,9 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;       // slack for 1024-B alig
 static_assert(kBN % 64 == 0, "epilogue works in 64-column chunks");
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
 
-__device__ __forceinline__ float silu_mul_fast(uint32_t gbits, uint32_t ubits) {
-    const float g = __uint_as_float(gbits);
-    const float u = __uint_as_float(ubits);
-    return __fdividef(g, 1.0f + __expf(-g)) * u;
+__device__ __forceinline__ float gated_fast(int which, float alpha, uint32_t gbits,
+                                            uint32_t ubits) {
+    return act::gated<false>(which, alpha, __uint_as_float(gbits), __uint_as_float(ubits));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -89,8 +89,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     swiglu_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_x,
                             const __grid_constant__ CUtensorMap tm_wg,
                             const __grid_constant__ CUtensorMap tm_wu,
-                            const __grid_constant__ CUtensorMap tm_h, int M, int N, int K,
-                            int num_m_tiles, int num_n_tiles) {
+                            const __grid_constant__ CUtensorMap tm_h,
+                            const __grid_constant__ CUtensorMap tm_g,
+                            const __grid_constant__ CUtensorMap tm_u, int M, int N, int K,
+                            int num_m_tiles, int num_n_tiles, int which_act, float alpha,
+                            int store_gu) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -128,6 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_wg);
         tma_prefetch_desc(&tm_wu);
         tma_prefetch_desc(&tm_h);
+        if (store_gu) {
+            tma_prefetch_desc(&tm_g);
+            tma_prefetch_desc(&tm_u);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
@@ -242,44 +249,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kAccCols);
+            // Per 64-column chunk: H = act(alpha g) u, then (training
+            // forward) G and U themselves, each staged and stored by TMA.
+            const int outputs = store_gu ? 3 : 1;
 #pragma unroll 1
             for (int c = 0; c < kBN / 64; ++c) {
-                // The previous store from this buffer must have read it.
-                if (lane == 0) bulk_wait_read<0>();
-                __syncwarp();
+#pragma unroll 1
+                for (int what = 0; what < outputs; ++what) {
+                    // The previous store from this buffer must have read it.
+                    if (lane == 0) bulk_wait_read<0>();
+                    __syncwarp();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t g[32], u[32];
-                    const uint32_t col = static_cast<uint32_t>(c * 64 + h * 32);
-                    tmem_ld_32x32b_x32(tacc + col, g);
-                    tmem_ld_32x32b_x32(tacc + kBN + col, u);
-                    tmem_ld_wait(g);
-                    tmem_ld_wait(u);
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t g[32], u[32];
+                        const uint32_t col = static_cast<uint32_t>(c * 64 + h * 32);
+                        if (what != 2) tmem_ld_32x32b_x32(tacc + col, g);
+                        if (what != 1) tmem_ld_32x32b_x32(tacc + kBN + col, u);
+                        tmem_ld_wait(g);
+                        tmem_ld_wait(u);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint4 v;
-                        v.x = pack_bf16x2(silu_mul_fast(g[8 * j + 0], u[8 * j + 0]),
-                                          silu_mul_fast(g[8 * j + 1], u[8 * j + 1]));
-                        v.y = pack_bf16x2(silu_mul_fast(g[8 * j + 2], u[8 * j + 2]),
-                                          silu_mul_fast(g[8 * j + 3], u[8 * j + 3]));
-                        v.z = pack_bf16x2(silu_mul_fast(g[8 * j + 4], u[8 * j + 4]),
-                                          silu_mul_fast(g[8 * j + 5], u[8 * j + 5]));
-                        v.w = pack_bf16x2(silu_mul_fast(g[8 * j + 6], u[8 * j + 6]),
-                                          silu_mul_fast(g[8 * j + 7], u[8 * j + 7]));
-                        // 16-byte chunk (h*4 + j) of this lane's 128-byte row,
-                        // placed where the TMA 128-byte swizzle expects it.
-                        const uint32_t chunk = static_cast<uint32_t>(h * 4 + j);
-                        sts_v4(buf + static_cast<uint32_t>(lane) * 128u + ((chunk ^ swz) << 4), v);
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 v;
+                            uint32_t *pv = &v.x;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int e = 8 * j + 2 * q;
+                                if (what == 0)
+                                    pv[q] = pack_bf16x2(gated_fast(which_act, alpha, g[e], u[e]),
+                                                        gated_fast(which_act, alpha, g[e + 1], u[e + 1]));
+                                else if (what == 1)
+                                    pv[q] = pack_bf16x2(__uint_as_float(g[e]), __uint_as_float(g[e + 1]));
+                                else
+                                    pv[q] = pack_bf16x2(__uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+                            }
+                            // 16-byte chunk (h*4 + j) of this lane's 128-byte row,
+                            // placed where the TMA 128-byte swizzle expects it.
+                            const uint32_t chunk = static_cast<uint32_t>(h * 4 + j);
+                            sts_v4(buf + static_cast<uint32_t>(lane) * 128u + ((chunk ^ swz) << 4), v);
+                        }
                     }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const int x = n0 + c * 64;
-                    const int y = m0 + quad * 32;
-                    if (x < N && y < M) {
-                        tma_store_2d(&tm_h, buf, x, y);
-                        bulk_commit();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int x = n0 + c * 64;
+                        const int y = m0 + quad * 32;
+                        if (x < N && y < M) {
+                            const CUtensorMap *dst = what == 0 ? &tm_h : (what == 1 ? &tm_g : &tm_u);
+                            tma_store_2d(dst, buf, x, y);
+                            bulk_commit();
+                        }
                     }
                 }
             }
@@ -311,14 +329,20 @@ std::atomic<unsigned> g_attr_set_mask{0};
 }  // namespace
 
 cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
-                             int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
-    CUtensorMap tx, twg, twu, th;
+                             int K, int N, const Epilogue &epi, const DeviceInfo &dev,
+                             cudaStream_t stream) {
+    CUtensorMap tx, twg, twu, th, tg, tu;
     const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const bool store_gu = epi.G != nullptr;
     if (!encode_tmap_2d(&tx, X, bf16, K, M, static_cast<uint64_t>(K) * 2, kBK, kBM, sw) ||
         !encode_tmap_2d(&twg, Wg, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
         !encode_tmap_2d(&twu, Wu, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
-        !encode_tmap_2d(&th, H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32, sw)) {
+        !encode_tmap_2d(&th, H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32, sw) ||
+        !encode_tmap_2d(&tg, store_gu ? epi.G : H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32,
+                        sw) ||
+        !encode_tmap_2d(&tu, store_gu ? epi.U : H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32,
+                        sw)) {
         return cudaErrorInvalidValue;
     }
     const unsigned bit = 1u << (dev.device & 31);
@@ -333,8 +357,9 @@ cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void
     const int num_n = (N + kBN - 1) / kBN;
     const long long tiles = static_cast<long long>(num_m) * num_n;
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    swiglu_gemm_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tx, twg, twu, th, M, N, K,
-                                                                   num_m, num_n);
+    swiglu_gemm_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+        tx, twg, twu, th, tg, tu, M, N, K, num_m, num_n, epi.activation, epi.gate_multiplier,
+        store_gu ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -37,6 +37,7 @@
 // All waits are bounded as in the bf16 kernel.
 #include <atomic>
 
+#include "activation.cuh"
 #include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -103,23 +104,22 @@ __device__ __forceinline__ void split4(uint4 &v, uint4 &lo) {
     }
 }
 
-// h = silu(g) * u in fp32: sigmoid from t = exp(-|g|) without cancellation,
-// expf and an IEEE division (a few ulp in total).
-__device__ __forceinline__ float silu_mul_accurate(uint32_t gbits, uint32_t ubits) {
-    const float g = __uint_as_float(gbits);
-    const float u = __uint_as_float(ubits);
-    const float t = expf(-fabsf(g));
-    const float r = 1.0f / (1.0f + t);
-    const float s = g >= 0.0f ? r : t * r;
-    return g * s * u;
+// h = act(alpha g) * u in fp32 with expf / tanhf and IEEE division (a few
+// ulp in total).
+__device__ __forceinline__ float gated_accurate(int which, float alpha, uint32_t gbits,
+                                                uint32_t ubits) {
+    return act::gated<true>(which, alpha, __uint_as_float(gbits), __uint_as_float(ubits));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     swiglu_gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_x,
                               const __grid_constant__ CUtensorMap tm_wg,
                               const __grid_constant__ CUtensorMap tm_wu,
-                              const __grid_constant__ CUtensorMap tm_h, int M, int N, int K,
-                              int num_m_tiles, int num_n_tiles) {
+                              const __grid_constant__ CUtensorMap tm_h,
+                              const __grid_constant__ CUtensorMap tm_g,
+                              const __grid_constant__ CUtensorMap tm_u, int M, int N, int K,
+                              int num_m_tiles, int num_n_tiles, int which_act, float alpha,
+                              int store_gu) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -157,6 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_wg);
         tma_prefetch_desc(&tm_wu);
         tma_prefetch_desc(&tm_h);
+        if (store_gu) {
+            tma_prefetch_desc(&tm_g);
+            tma_prefetch_desc(&tm_u);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
@@ -338,35 +342,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(bar_cempty);
             }
             if (failed) break;
-            // output from the running sum
+            // output from the running sum: H = act(alpha g) u, then (training
+            // forward) G and U themselves
+            const int outputs = store_gu ? 3 : 1;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
-                if (lane == 0) bulk_wait_read<0>();
-                __syncwarp();
-                uint32_t g[32], u[32];
-                tmem_ld_32x32b_x32(run_acc + 32u * c, g);
-                tmem_ld_32x32b_x32(run_acc + kBN + 32u * c, u);
-                tmem_ld_wait(g);
-                tmem_ld_wait(u);
+#pragma unroll 1
+                for (int what = 0; what < outputs; ++what) {
+                    if (lane == 0) bulk_wait_read<0>();
+                    __syncwarp();
+                    uint32_t g[32], u[32];
+                    if (what != 2) tmem_ld_32x32b_x32(run_acc + 32u * c, g);
+                    if (what != 1) tmem_ld_32x32b_x32(run_acc + kBN + 32u * c, u);
+                    tmem_ld_wait(g);
+                    tmem_ld_wait(u);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint4 v;
-                    v.x = __float_as_uint(silu_mul_accurate(g[4 * j + 0], u[4 * j + 0]));
-                    v.y = __float_as_uint(silu_mul_accurate(g[4 * j + 1], u[4 * j + 1]));
-                    v.z = __float_as_uint(silu_mul_accurate(g[4 * j + 2], u[4 * j + 2]));
-                    v.w = __float_as_uint(silu_mul_accurate(g[4 * j + 3], u[4 * j + 3]));
-                    sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
-                               ((static_cast<uint32_t>(j) ^ swz) << 4),
-                           v);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const int x = n0 + c * 32;
-                    const int y = m0 + quad * 32;
-                    if (x < N && y < M) {
-                        tma_store_2d(&tm_h, buf, x, y);
-                        bulk_commit();
+                    for (int j = 0; j < 8; ++j) {
+                        uint4 v;
+                        uint32_t *pv = &v.x;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int e = 4 * j + q;
+                            pv[q] = what == 0 ? __float_as_uint(gated_accurate(which_act, alpha, g[e], u[e]))
+                                              : (what == 1 ? g[e] : u[e]);
+                        }
+                        sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
+                                   ((static_cast<uint32_t>(j) ^ swz) << 4),
+                               v);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int x = n0 + c * 32;
+                        const int y = m0 + quad * 32;
+                        if (x < N && y < M) {
+                            const CUtensorMap *dst = what == 0 ? &tm_h : (what == 1 ? &tm_g : &tm_u);
+                            tma_store_2d(dst, buf, x, y);
+                            bulk_commit();
+                        }
                     }
                 }
             }
@@ -390,15 +403,20 @@ std::atomic<unsigned> g_attr_set_mask{0};
 }  // namespace
 
 cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, void *H, int M,
-                               int K, int N, const DeviceInfo &dev, cudaStream_t stream) {
-    CUtensorMap tx, twg, twu, th;
+                               int K, int N, const Epilogue &epi, const DeviceInfo &dev,
+                               cudaStream_t stream) {
+    CUtensorMap tx, twg, twu, th, tg, tu;
     const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const bool store_gu = epi.G != nullptr;
+    const uint64_t hrow = static_cast<uint64_t>(N) * 4;
     if (!encode_tmap_2d(&tx, X, f32, K, M, static_cast<uint64_t>(K) * 4, kBK, kBM, sw64) ||
         !encode_tmap_2d(&twg, Wg, f32, K, N, static_cast<uint64_t>(K) * 4, kBK, kBN, sw64) ||
         !encode_tmap_2d(&twu, Wu, f32, K, N, static_cast<uint64_t>(K) * 4, kBK, kBN, sw64) ||
-        !encode_tmap_2d(&th, H, f32, N, M, static_cast<uint64_t>(N) * 4, 32, 32,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) {
+        !encode_tmap_2d(&th, H, f32, N, M, hrow, 32, 32, sw128) ||
+        !encode_tmap_2d(&tg, store_gu ? epi.G : H, f32, N, M, hrow, 32, 32, sw128) ||
+        !encode_tmap_2d(&tu, store_gu ? epi.U : H, f32, N, M, hrow, 32, 32, sw128)) {
         return cudaErrorInvalidValue;
     }
     const unsigned bit = 1u << (dev.device & 31);
@@ -413,8 +431,9 @@ cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, vo
     const int num_n = (N + kBN - 1) / kBN;
     const long long tiles = static_cast<long long>(num_m) * num_n;
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    swiglu_gemm_tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tx, twg, twu, th, M, N, K,
-                                                                     num_m, num_n);
+    swiglu_gemm_tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+        tx, twg, twu, th, tg, tu, M, N, K, num_m, num_n, epi.activation, epi.gate_multiplier,
+        store_gu ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -9,6 +9,16 @@
 
 namespace swiglu {
 
+// Epilogue variant of a forward call: H = act(gate_multiplier * G) * U with
+// act 0 = SiLU, 1 = GELU(tanh); G and U (same dtype as H) are also stored
+// when G != nullptr (then U != nullptr too).
+struct Epilogue {
+    int activation = 0;
+    float gate_multiplier = 1.0f;
+    void *G = nullptr;
+    void *U = nullptr;
+};
+
 struct DeviceInfo {
     int device;
     int sm_count;
@@ -19,13 +29,13 @@ struct DeviceInfo {
 
 // bf16 forward, tcgen05 dual GEMM (any M >= 1, K >= 1, N >= 1).
 cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void *H,
-                             int M, int K, int N, const DeviceInfo &dev,
-                             cudaStream_t stream);
+                             int M, int K, int N, const Epilogue &epi,
+                             const DeviceInfo &dev, cudaStream_t stream);
 
 // fp32 forward, 3xTF32 tcgen05 dual GEMM.
 cudaError_t launch_gemm_tf32x3(const void *X, const void *Wg, const void *Wu, void *H,
-                               int M, int K, int N, const DeviceInfo &dev,
-                               cudaStream_t stream);
+                               int M, int K, int N, const Epilogue &epi,
+                               const DeviceInfo &dev, cudaStream_t stream);
 
 // bf16 forward for M <= 8: weight streaming with tensor-core dot products.
 // decode_bf16_supported: whether K fits the kernel's shared-memory stages
@@ -35,13 +45,13 @@ bool decode_bf16_supported(int K);
 // first weight stages before waiting for the preceding grid (see
 // SWIGLU_FLAG_WEIGHTS_STABLE).
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H,
-                               int M, int K, int N, bool weights_stable,
+                               int M, int K, int N, const Epilogue &epi, bool weights_stable,
                                const DeviceInfo &dev, cudaStream_t stream);
 
-// Elementwise dSwiGLU; dtype 0 = bf16, 1 = fp32.
+// Elementwise backward of h = act(alpha g) u; dtype 0 = bf16, 1 = fp32.
 cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG,
-                           void *dU, int64_t n, int dtype, const DeviceInfo &dev,
-                           cudaStream_t stream);
+                           void *dU, int64_t n, int dtype, int activation, float alpha,
+                           const DeviceInfo &dev, cudaStream_t stream);
 
 // Pure streaming read of two buffers (bench-only floor probe).
 int read_floor_grid(const DeviceInfo &dev);
