@@ -101,6 +101,10 @@ class Oracle:
                                                      ctypes.c_int, _D, _P, _P, _P, _P, _P]
         lib.oracle_dswiglu_act_f64.restype = None
         lib.oracle_dswiglu_act_f64.argtypes = [_P, _P, _P, _I64, ctypes.c_int, _D, _P, _P]
+        lib.oracle_bwd_dx_f64.restype = None
+        lib.oracle_bwd_dx_f64.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P]
+        lib.oracle_bwd_dw_f64.restype = None
+        lib.oracle_bwd_dw_f64.argtypes = [_P, _P, _P, _I64, _I64, _I64, _P, _P]
         for name in ("oracle_bf16_to_f64", "oracle_f32_to_f64"):
             f = getattr(lib, name)
             f.restype = None
@@ -232,6 +236,28 @@ class Oracle:
             raise MemoryError("oracle: row buffer allocation failed")
         return out
 
+    # ---- backward GEMMs -------------------------------------------------------
+    def bwd_dx_f64(self, dG, dU, Wg, Wu):
+        """dX [M,K] = dG Wg + dU Wu for dG, dU [M,N] and Wg, Wu [N,K]."""
+        dG, dU, Wg, Wu = (np.ascontiguousarray(a, dtype=np.float64) for a in (dG, dU, Wg, Wu))
+        M, N = dG.shape
+        K = Wg.shape[1]
+        assert dU.shape == (M, N) and Wg.shape == (N, K) and Wu.shape == (N, K)
+        dX = np.empty((M, K), dtype=np.float64)
+        self.lib.oracle_bwd_dx_f64(_ptr(dG), _ptr(dU), _ptr(Wg), _ptr(Wu), M, K, N, _ptr(dX))
+        return dX
+
+    def bwd_dw_f64(self, dG, dU, X):
+        """(dWg, dWu) [N,K] = (dG^T X, dU^T X) for dG, dU [M,N] and X [M,K]."""
+        dG, dU, X = (np.ascontiguousarray(a, dtype=np.float64) for a in (dG, dU, X))
+        M, N = dG.shape
+        K = X.shape[1]
+        assert dU.shape == (M, N) and X.shape == (M, K)
+        dWg = np.empty((N, K), dtype=np.float64)
+        dWu = np.empty((N, K), dtype=np.float64)
+        self.lib.oracle_bwd_dw_f64(_ptr(dG), _ptr(dU), _ptr(X), M, K, N, _ptr(dWg), _ptr(dWu))
+        return dWg, dWu
+
     # ---- backward --------------------------------------------------------------
     def dswiglu_f64(self, dH, G, U, act: int = 0, alpha: float = 1.0):
         """Elementwise backward of h = act(alpha g) u on float64 arrays of
@@ -280,6 +306,6 @@ def __getattr__(name):
     if name in {"sigmoid", "silu", "dsilu", "gelu_tanh", "dgelu_tanh", "act", "dact",
                 "decode_bf16", "decode",
                 "swiglu_fwd_f64", "swiglu_fwd", "swiglu_fwd_points",
-                "dswiglu_f64", "dswiglu"}:
+                "dswiglu_f64", "dswiglu", "bwd_dx_f64", "bwd_dw_f64"}:
         return getattr(default(), name)
     raise AttributeError(name)

@@ -360,3 +360,48 @@ ORACLE_API void oracle_dswiglu_f32(const float *dH, const float *G,
         dswiglu_one((double)dH[i], (double)G[i], (double)U[i], 0, 1.0, dG + i,
                     dU + i);
 }
+
+/* ---- backward GEMMs of the projection ----------------------------------- */
+
+/*
+ * With G = X Wg^T and U = X Wu^T, and dG, dU the gradients of the loss with
+ * respect to G and U (the output of dSwiGLU), the chain rule gives
+ *   dX[m,k]  = sum_n dG[m,n] Wg[n,k] + dU[m,n] Wu[n,k]
+ *   dWg[n,k] = sum_m dG[m,n] X[m,k],   dWu[n,k] = sum_m dU[m,n] X[m,k]
+ * (the backward half of the fused MLP's forward/backward dataflow, page
+ * "[RFC] Testing Methodology for FP32 Convergence Tests on Fused
+ * SwiGLU/dSwiGLU Kernels", Background).  Plain loops, ascending summation
+ * index.
+ */
+ORACLE_API void oracle_bwd_dx_f64(const double *dG, const double *dU,
+                                  const double *Wg, const double *Wu,
+                                  int64_t M, int64_t K, int64_t N, double *dX)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                acc += dG[m * N + n] * Wg[n * K + k] + dU[m * N + n] * Wu[n * K + k];
+            dX[m * K + k] = acc;
+        }
+    }
+}
+
+ORACLE_API void oracle_bwd_dw_f64(const double *dG, const double *dU,
+                                  const double *X, int64_t M, int64_t K,
+                                  int64_t N, double *dWg, double *dWu)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double ag = 0.0, au = 0.0;
+            for (int64_t m = 0; m < M; ++m) {
+                ag += dG[m * N + n] * X[m * K + k];
+                au += dU[m * N + n] * X[m * K + k];
+            }
+            dWg[n * K + k] = ag;
+            dWu[n * K + k] = au;
+        }
+    }
+}

@@ -43,6 +43,9 @@ What pins what:
                         (the multiplier acts on the gate pre-activation).
   variants_bwd          dG, dU of the variants against central differences of
                         the variant forward, and dU = dh act(alpha g).
+  backward_gemms        dX, dWg, dWu against numpy matmul, and the whole chain
+                        (forward, dSwiGLU, backward GEMMs) against central
+                        differences of the scalar loss sum(dH * H) in X, Wg, Wu.
 """
 from __future__ import annotations
 
@@ -354,8 +357,39 @@ def variants_bwd(o):
                 assert dU[i] == dh[i] * o.act(alpha * g[i], act)
 
 
+def backward_gemms(o):
+    r = _rng(120)
+    M, K, N = 5, 12, 9
+    X = r.standard_normal((M, K))
+    Wg = r.standard_normal((N, K)) * 0.4
+    Wu = r.standard_normal((N, K)) * 0.4
+    dH = r.standard_normal((M, N))
+    f = o.swiglu_fwd_f64(X, Wg, Wu)
+    dG, dU = o.dswiglu_f64(dH, f["G"], f["U"])
+    dX = o.bwd_dx_f64(dG, dU, Wg, Wu)
+    dWg, dWu = o.bwd_dw_f64(dG, dU, X)
+    assert np.allclose(dX, dG @ Wg + dU @ Wu, rtol=1e-12, atol=1e-14)
+    assert np.allclose(dWg, dG.T @ X, rtol=1e-12, atol=1e-14)
+    assert np.allclose(dWu, dU.T @ X, rtol=1e-12, atol=1e-14)
+
+    def loss(X_, Wg_, Wu_):
+        return float(np.sum(dH * o.swiglu_fwd_f64(X_, Wg_, Wu_)["H"]))
+    d = 1e-6
+    for (arr, grad, name) in ((X, dX, "X"), (Wg, dWg, "Wg"), (Wu, dWu, "Wu")):
+        for idx in [(0, 0), (arr.shape[0] - 1, arr.shape[1] - 1), (2, 5), (1, 7)]:
+            p, q = arr.copy(), arr.copy()
+            p[idx] += d
+            q[idx] -= d
+            args_p = [X, Wg, Wu]
+            args_q = [X, Wg, Wu]
+            i = {"X": 0, "Wg": 1, "Wu": 2}[name]
+            args_p[i], args_q[i] = p, q
+            fd = (loss(*args_p) - loss(*args_q)) / (2 * d)
+            assert abs(fd - grad[idx]) <= 1e-7 * (1 + abs(fd)), (name, idx, fd, grad[idx])
+
+
 ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
             fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
             fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
             dswiglu_special, dswiglu_storage, gelu_closed_forms, variants_fwd,
-            variants_bwd]
+            variants_bwd, backward_gemms]

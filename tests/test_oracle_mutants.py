@@ -40,6 +40,11 @@ MUTANTS = [
     ("wrong_weight_row",
      "one_output(X + m * K, Wg + n * K, Wu + n * K, K,",
      "one_output(X + m * K, Wg + ((n + 1) % N) * K, Wu + n * K, K,"),
+    ("dx_wrong_weight",
+     "acc += dG[m * N + n] * Wg[n * K + k] + dU[m * N + n] * Wu[n * K + k];",
+     "acc += dG[m * N + n] * Wu[n * K + k] + dU[m * N + n] * Wg[n * K + k];"),
+    ("dw_transposed_index",
+     "ag += dG[m * N + n] * X[m * K + k];", "ag += dG[m * N + n] * X[m * K + (K - 1 - k)];"),
     ("bf16_decode_shift",
      "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
     ("magnitude_missing_abs",
