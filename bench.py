@@ -372,7 +372,27 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
-    del X, Wg, Wu, H, Gs, Us
+    # backward GEMMs at the same size: dX = dG Wg + dU Wu and dWg, dWu
+    dGb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)
+    dUb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    ms = time_op(lambda: up.swiglu_bwd_dx(dGb, dUb, Wg, Wu, dX, stream=stream))
+    tf = fl / (ms * 1e-3) / 1e12
+    res.append({"workload": "backward dX = dG Wg + dU Wu, LLaMA-3 8B M=8192 bf16",
+                "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(tf / pk["bf16_tflops"], 4)}})
+    dWg = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    dWu = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    ms = time_op(lambda: up.swiglu_bwd_dw(dGb, dUb, X, dWg, dWu, stream=stream))
+    tf = fl / (ms * 1e-3) / 1e12
+    res.append({"workload": "backward dWg = dG^T X, dWu = dU^T X, LLaMA-3 8B M=8192 bf16",
+                "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": round(tf / pk["bf16_tflops"], 4)}})
+    del X, Wg, Wu, H, Gs, Us, dGb, dUb, dX, dWg, dWu
     # dSwiGLU on [8192, 14336] bf16
     n = 8192 * 14336
     dH = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)

@@ -113,7 +113,8 @@ enum swiglu_route {
     SWIGLU_ROUTE_ZERO_K = 1,      /* K == 0: H is filled with zeros         */
     SWIGLU_ROUTE_DECODE_BF16 = 2, /* bf16, M <= 8: weight-streaming kernel  */
     SWIGLU_ROUTE_GEMM_BF16 = 3,   /* bf16, M > 8: tcgen05 dual GEMM         */
-    SWIGLU_ROUTE_GEMM_TF32X3 = 4  /* fp32: 3xTF32 tcgen05 dual GEMM         */
+    SWIGLU_ROUTE_GEMM_TF32X3 = 4, /* fp32: 3xTF32 tcgen05 dual GEMM         */
+    SWIGLU_ROUTE_BWD_GEMM_BF16 = 5 /* bf16 backward GEMM (swiglu_bwd_dx/_dw) */
 };
 
 /*
@@ -189,12 +190,55 @@ SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U
                                     int activation, float gate_multiplier,
                                     cudaStream_t stream);
 
+/*
+ * swiglu_bwd_dx -- input gradient of the projection:
+ *   dX = dG Wg + dU Wu,   dX[m,k] = sum_n dG[m,n] Wg[n,k] + dU[m,n] Wu[n,k]
+ * (chain rule through G = X Wg^T and U = X Wu^T; the backward half of the
+ * fused MLP's forward/backward dataflow, page "[RFC] Testing Methodology for
+ * FP32 Convergence Tests on Fused SwiGLU/dSwiGLU Kernels", Background).
+ *
+ *  dG, dU  [M, N] device bf16 (the outputs of dswiglu_bwd), 16-byte aligned.
+ *  Wg, Wu  [N, K] device bf16, the forward's weights, 16-byte aligned.
+ *  dX      [M, K] device bf16 output, 16-byte aligned; written, never read.
+ *  M, K, N >= 0; K and N multiples of 8.  dtype must be SWIGLU_BF16 (any
+ *  other value: SWIGLU_ERR_BAD_DTYPE).
+ *
+ *  Both products accumulate in ONE fp32 accumulator (tcgen05, TMEM); dX is
+ *  rounded once to bf16 (RNE).  M == 0 or K == 0: nothing enqueued.  N == 0:
+ *  dX is set to +0.  dX must not overlap an input (SWIGLU_ERR_OVERLAP).
+ *  Allocates no device memory.
+ */
+SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
+                             const void *Wu, void *dX, int64_t M, int64_t K,
+                             int64_t N, int dtype, cudaStream_t stream);
+
+/*
+ * swiglu_bwd_dw -- weight gradients of the projection:
+ *   dWg = dG^T X,  dWu = dU^T X,  dWg[n,k] = sum_m dG[m,n] X[m,k]
+ * (same passage as swiglu_bwd_dx).
+ *
+ *  dG, dU    [M, N] device bf16, 16-byte aligned.
+ *  X         [M, K] device bf16, the forward's input, 16-byte aligned.
+ *  dWg, dWu  [N, K] device bf16 outputs, 16-byte aligned; written, never
+ *            read (not accumulated into).
+ *  M, K, N >= 0; K and N multiples of 8.  dtype must be SWIGLU_BF16.
+ *
+ *  fp32 accumulation over all M rows in TMEM, one RNE rounding per output.
+ *  N == 0 or K == 0: nothing enqueued.  M == 0: dWg and dWu are set to +0.
+ *  Outputs must not overlap each other or an input (SWIGLU_ERR_OVERLAP).
+ *  Allocates no device memory.
+ */
+SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X,
+                             void *dWg, void *dWu, int64_t M, int64_t K,
+                             int64_t N, int dtype, cudaStream_t stream);
+
 /* Route swiglu_fwd takes for these arguments (pure host function; returns a
  * swiglu_route, or -1 for arguments swiglu_fwd would reject). */
 SWIGLU_API int swiglu_route_for(int64_t M, int64_t K, int64_t N, int dtype);
 
-/* Route of the last swiglu_fwd call on this host thread that returned
- * SWIGLU_OK (SWIGLU_ROUTE_NONE before the first).  Lets tests assert that
+/* Route of the last swiglu_fwd* or swiglu_bwd_dx/_dw call on this host
+ * thread that returned SWIGLU_OK (SWIGLU_ROUTE_NONE before the first; an
+ * empty reduction reports SWIGLU_ROUTE_ZERO_K).  Lets tests assert that
  * the fused kernel actually ran. */
 SWIGLU_API int swiglu_last_route(void);
 

@@ -119,3 +119,54 @@ def test_status_strings():
     for code in range(13):
         assert _capi.status_string(code)
     assert _capi.status_string(999) == "unknown status"
+
+
+# swiglu_bwd_dx(dG, dU, Wg, Wu, dX, M, K, N, dtype)
+@pytest.mark.parametrize("args,code", [
+    ((16, 32, 48, 64, None, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((None, 32, 48, 64, 80, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((16, 32, 48, 64, 88, 4, 64, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_PTR),
+    ((16, 32, 48, 64, 80, 4, 64, 64, 1), _capi.SWIGLU_ERR_BAD_DTYPE),   # bf16 only
+    ((16, 32, 48, 64, 80, 4, 60, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, 80, 4, 64, 68, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, 80, -1, 64, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
+    ((16, 32, 48, 64, 80, 1 << 31, 64, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
+    # dX [4,64] at 1 MiB overlaps Wg [64,64] placed 16 bytes before it
+    ((1 << 22, 1 << 23, (1 << 20) - 16, 1 << 24, 1 << 20, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),
+    ((1 << 20, 1 << 23, 1 << 22, 1 << 24, 1 << 20, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),
+    ((None, None, None, None, None, 0, 64, 64, 0), _capi.SWIGLU_OK),   # M == 0
+    ((None, None, None, None, None, 4, 0, 64, 0), _capi.SWIGLU_OK),    # K == 0
+])
+def test_bwd_dx_host_validation(args, code):
+    assert _capi.lib().swiglu_bwd_dx(*args, None) == code
+
+
+# swiglu_bwd_dw(dG, dU, X, dWg, dWu, M, K, N, dtype)
+@pytest.mark.parametrize("args,code", [
+    ((16, 32, 48, None, 80, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((16, None, 48, 1 << 20, 1 << 21, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
+    ((16, 32, 48, 1 << 20, (1 << 21) + 4, 4, 64, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_PTR),
+    ((16, 32, 48, 64, 80, 4, 64, 64, 1), _capi.SWIGLU_ERR_BAD_DTYPE),
+    ((16, 32, 48, 64, 80, 4, 64, 12, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, 80, 4, -8, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
+    # dWu [64,64] bf16 = 8 KiB starts inside dWg
+    ((1 << 22, 1 << 23, 1 << 24, 1 << 20, (1 << 20) + 4096, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),
+    # dWg on top of X
+    ((1 << 22, 1 << 23, 1 << 20, 1 << 20, 1 << 24, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),
+    ((None, None, None, None, None, 4, 64, 0, 0), _capi.SWIGLU_OK),    # N == 0
+    ((None, None, None, None, None, 4, 0, 64, 0), _capi.SWIGLU_OK),    # K == 0
+])
+def test_bwd_dw_host_validation(args, code):
+    assert _capi.lib().swiglu_bwd_dw(*args, None) == code
+
+
+def test_bwd_gemm_no_device_is_an_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    lib = _capi.lib()
+    assert lib.swiglu_bwd_dx(1 << 20, 1 << 21, 1 << 22, 1 << 23, 1 << 24, 4, 64, 64, 0,
+                             None) == _capi.SWIGLU_ERR_NO_DEVICE
+    # empty reduction still needs the device (it writes zeros)
+    assert lib.swiglu_bwd_dw(None, None, None, 1 << 20, 1 << 21, 0, 64, 64, 0,
+                             None) == _capi.SWIGLU_ERR_NO_DEVICE

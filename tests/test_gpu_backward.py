@@ -1,0 +1,194 @@
+"""Backward GEMMs of the projection (dX = dG Wg + dU Wu; dWg = dG^T X,
+dWu = dU^T X -- the backward half of the fused MLP's forward/backward
+dataflow, page "[RFC] Testing Methodology for FP32 Convergence Tests on
+Fused SwiGLU/dSwiGLU Kernels", Background) through the C ABI, against the
+fp64 oracle on the same bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_bf16_close, assert_guards_intact, dev, f64, guarded_empty,
+                      to_dev)
+from up_projection_b200 import _capi, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _grads(M, N, seed):
+    return synth.normal((M, N), seed + 10), synth.normal((M, N), seed + 11)
+
+
+def run_dx(dG, dU, Wg, Wu):
+    M, N = dG.shape
+    K = Wg.shape[1]
+    dGd, dUd, Wgd, Wud = to_dev(dG, dU, Wg, Wu)
+    full, dX = guarded_empty(M * K, torch.bfloat16)
+    st = _capi.lib().swiglu_bwd_dx(dGd.data_ptr(), dUd.data_ptr(), Wgd.data_ptr(),
+                                   Wud.data_ptr(), dX.data_ptr(), M, K, N, _capi.SWIGLU_BF16,
+                                   torch.cuda.current_stream().cuda_stream)
+    assert st == 0, _capi.status_string(st)
+    assert _capi.swiglu_sync_status() == 0
+    assert_guards_intact(full)
+    return dX.view(M, K)
+
+
+def run_dw(dG, dU, X):
+    M, N = dG.shape
+    K = X.shape[1]
+    dGd, dUd, Xd = to_dev(dG, dU, X)
+    fg, dWg = guarded_empty(N * K, torch.bfloat16)
+    fu, dWu = guarded_empty(N * K, torch.bfloat16)
+    st = _capi.lib().swiglu_bwd_dw(dGd.data_ptr(), dUd.data_ptr(), Xd.data_ptr(),
+                                   dWg.data_ptr(), dWu.data_ptr(), M, K, N, _capi.SWIGLU_BF16,
+                                   torch.cuda.current_stream().cuda_stream)
+    assert st == 0, _capi.status_string(st)
+    assert _capi.swiglu_sync_status() == 0
+    assert_guards_intact(fg)
+    assert_guards_intact(fu)
+    return dWg.view(N, K), dWu.view(N, K)
+
+
+# (M, K, N): single tile, ragged tails in every dimension (K not a multiple of
+# 64, N not a multiple of 64 or 128), several tiles each way.  With 148 SMs
+# the tile-width model picks 256-wide tiles for dX of (1300, 2560, 136) and
+# dW of (200, 2048, 1032), 192-wide ones for dX of (4800, 448, 72) and dW of
+# (100, 448, 2376), and 128-wide ones elsewhere, so all three are covered.
+SHAPES = [(1, 8, 8), (130, 264, 200), (300, 520, 136), (257, 1032, 72), (64, 128, 64),
+          (1300, 2560, 136), (200, 2048, 1032), (9, 64, 1544), (4800, 448, 72),
+          (100, 448, 2376)]
+
+
+@pytest.mark.parametrize("M,K,N", SHAPES)
+def test_bwd_dx_matches_oracle(M, K, N):
+    _, Wg, Wu = synth.swiglu_inputs(M, K, N, seed=M + K)
+    dG, dU = _grads(M, N, seed=N)
+    dX = run_dx(dG, dU, Wg, Wu)
+    assert _capi.swiglu_last_route() == _capi.ROUTE_BWD_GEMM_BF16
+    ref = oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu))
+    assert_bf16_close(f64(dX), ref, f"dX {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M,K,N", SHAPES)
+def test_bwd_dw_matches_oracle(M, K, N):
+    X, _, _ = synth.swiglu_inputs(M, K, N, seed=M + K)
+    dG, dU = _grads(M, N, seed=N)
+    dWg, dWu = run_dw(dG, dU, X)
+    assert _capi.swiglu_last_route() == _capi.ROUTE_BWD_GEMM_BF16
+    rg, ru = oracle.bwd_dw_f64(f64(dG), f64(dU), f64(X))
+    assert_bf16_close(f64(dWg), rg, f"dWg {M}x{K}x{N}")
+    assert_bf16_close(f64(dWu), ru, f"dWu {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 264, 200), (130, 1032, 1544)])
+def test_bwd_integer_exact(M, K, N):
+    """Ternary operands: every sum is a small integer, exact in fp32 in any
+    order and, below 256 in magnitude, exact in bf16 -- so the outputs must
+    match the oracle bit for bit (a wrong index, operand or tail fails)."""
+    X = synth.ternary((M, K), 1, 0.5)
+    Wg = synth.ternary((N, K), 2, 0.05)
+    Wu = synth.ternary((N, K), 3, 0.05)
+    dG = synth.ternary((M, N), 4, 0.05)
+    dU = synth.ternary((M, N), 5, 0.05)
+    rdx = oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu))
+    rg, ru = oracle.bwd_dw_f64(f64(dG), f64(dU), f64(X))
+    for r in (rdx, rg, ru):
+        assert np.abs(r).max() <= 256 and np.abs(r).max() >= 2
+    np.testing.assert_array_equal(f64(run_dx(dG, dU, Wg, Wu)), rdx)
+    dWg, dWu = run_dw(dG, dU, X)
+    np.testing.assert_array_equal(f64(dWg), rg)
+    np.testing.assert_array_equal(f64(dWu), ru)
+
+
+def test_bwd_pairs_are_not_swapped():
+    """dU = 0: dX must equal dG Wg alone (and dWu must be exactly zero)."""
+    M, K, N = 200, 264, 136
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, seed=5)
+    dG, _ = _grads(M, N, seed=7)
+    dU = torch.zeros_like(dG)
+    dX = run_dx(dG, dU, Wg, Wu)
+    assert_bf16_close(f64(dX), f64(dG) @ f64(Wg), "dX with dU = 0")
+    dWg, dWu = run_dw(dG, dU, X)
+    assert not bool(dWu.any())
+    assert_bf16_close(f64(dWg), f64(dG).T @ f64(X), "dWg")
+
+
+def test_bwd_empty_and_degenerate():
+    s = torch.cuda.current_stream().cuda_stream
+    lib = _capi.lib()
+    # N == 0: dX = 0 (the empty reduction), dW untouched-and-empty.
+    full, dX = guarded_empty(5 * 64, torch.bfloat16)
+    assert lib.swiglu_bwd_dx(None, None, None, None, dX.data_ptr(), 5, 64, 0, 0, s) == 0
+    assert _capi.swiglu_last_route() == _capi.ROUTE_ZERO_K
+    torch.cuda.synchronize()
+    assert not bool(dX.any()) and not bool(torch.signbit(dX).any())
+    assert_guards_intact(full)
+    # M == 0: dWg = dWu = 0.
+    fg, dWg = guarded_empty(16 * 64, torch.bfloat16)
+    fu, dWu = guarded_empty(16 * 64, torch.bfloat16)
+    assert lib.swiglu_bwd_dw(None, None, None, dWg.data_ptr(), dWu.data_ptr(), 0, 64, 16, 0,
+                             s) == 0
+    torch.cuda.synchronize()
+    assert not bool(dWg.any()) and not bool(dWu.any())
+    assert_guards_intact(fg)
+    assert_guards_intact(fu)
+    # M == 0 for dX / N == 0 for dW: nothing to write, nothing enqueued.
+    assert lib.swiglu_bwd_dx(None, None, None, None, None, 0, 64, 64, 0, s) == 0
+    assert _capi.swiglu_last_route() == _capi.ROUTE_NONE
+    assert lib.swiglu_bwd_dw(None, None, None, None, None, 7, 64, 0, 0, s) == 0
+
+
+def test_bwd_deterministic():
+    M, K, N = 520, 1032, 264
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, seed=3)
+    dG, dU = _grads(M, N, seed=4)
+    a = run_dx(dG, dU, Wg, Wu).clone()
+    b = run_dx(dG, dU, Wg, Wu)
+    assert torch.equal(a, b)
+    g1, u1 = run_dw(dG, dU, X)
+    g1, u1 = g1.clone(), u1.clone()
+    g2, u2 = run_dw(dG, dU, X)
+    assert torch.equal(g1, g2) and torch.equal(u1, u2)
+
+
+def test_bwd_python_binding_shapes():
+    M, K, N = 3 * 70, 264, 136
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, seed=9)
+    dG, dU = _grads(M, N, seed=9)
+    Xd, Wgd, Wud, dGd, dUd = to_dev(X, Wg, Wu, dG, dU)
+    dX = _capi.swiglu_bwd_dx(dGd.view(3, 70, N), dUd.view(3, 70, N), Wgd, Wud)
+    assert dX.shape == (3, 70, K)
+    dWg, dWu = _capi.swiglu_bwd_dw(dGd.view(3, 70, N), dUd.view(3, 70, N), Xd.view(3, 70, K))
+    assert dWg.shape == (N, K) and dWu.shape == (N, K)
+    assert_bf16_close(f64(dX).reshape(M, K), oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu)),
+                      "dX via binding")
+    with pytest.raises(TypeError):
+        _capi.swiglu_bwd_dx(dGd.float(), dUd.float(), Wgd.float(), Wud.float())
+
+
+def test_training_step_full_size_sampled():
+    """The whole training step at the prefill size (M=4096 tokens, K=4096,
+    N=14336): forward storing G and U, dSwiGLU, dX and dW -- each stage
+    checked on sampled outputs against the oracle fed that stage's GPU
+    inputs."""
+    M, K, N = 4096, 4096, 14336
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, seed=21)
+    dH = synth.normal((M, N), 22)
+    Xd, Wgd, Wud, dHd = to_dev(X, Wg, Wu, dH)
+    H, G, U = _capi.swiglu_fwd(Xd, Wgd, Wud, return_gu=True)
+    dG, dU = _capi.dswiglu_bwd(dHd, G, U)
+    dX = _capi.swiglu_bwd_dx(dG, dU, Wgd, Wud)
+    dWg, dWu = _capi.swiglu_bwd_dw(dG, dU, Xd)
+    assert _capi.swiglu_sync_status() == 0
+    r = np.random.Generator(np.random.PCG64(5))
+    rows = np.concatenate([r.integers(0, M, 6), [0, M - 1]])
+    cols = np.concatenate([r.integers(0, N, 6), [0, N - 1]])
+    dGc, dUc = dG.cpu(), dU.cpu()
+    ref_dx = oracle.bwd_dx_f64(f64(dGc[rows]), f64(dUc[rows]), f64(Wg), f64(Wu))
+    assert_bf16_close(f64(dX.cpu()[rows]), ref_dx, "dX rows (full size)")
+    rg, ru = oracle.bwd_dw_f64(f64(dGc[:, cols]), f64(dUc[:, cols]), f64(X))
+    assert_bf16_close(f64(dWg.cpu()[cols]), rg, "dWg rows (full size)")
+    assert_bf16_close(f64(dWu.cpu()[cols]), ru, "dWu rows (full size)")
+    rdg, rdu = oracle.dswiglu_f64(f64(dH[rows]), f64(G.cpu()[rows]), f64(U.cpu()[rows]))
+    assert_bf16_close(f64(dGc[rows]), rdg, "dG rows")
+    assert_bf16_close(f64(dUc[rows]), rdu, "dU rows")

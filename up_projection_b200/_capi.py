@@ -43,6 +43,7 @@ ROUTE_ZERO_K = 1
 ROUTE_DECODE_BF16 = 2
 ROUTE_GEMM_BF16 = 3
 ROUTE_GEMM_TF32X3 = 4
+ROUTE_BWD_GEMM_BF16 = 5
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -64,6 +65,8 @@ SIGNATURES = {
     "dswiglu_bwd_epilogue": (_I, [_P, _P, _P, _P, _P, _I64, _I, _I, ctypes.c_float, _P]),
     "dswiglu_bwd": (_I, [_P, _P, _P, _P, _P, _I64, _P]),
     "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
+    "swiglu_bwd_dx": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
+    "swiglu_bwd_dw": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
     "swiglu_last_route": (_I, []),
     "swiglu_status_string": (ctypes.c_char_p, [_I]),
@@ -204,6 +207,60 @@ def dswiglu_bwd(dH: torch.Tensor, G: torch.Tensor, U: torch.Tensor,
                                     float(gate_multiplier), _stream(stream))
     _check("dswiglu_bwd", st)
     return dG, dU
+
+
+def _bwd_shapes(dG, dU, name_w, W):
+    for t, n in ((dG, "dG"), (dU, "dU"), (W, name_w)):
+        _dev(t, n)
+    if not (dG.dtype == dU.dtype == W.dtype == torch.bfloat16):
+        raise TypeError("the backward GEMMs take bfloat16 tensors")
+    if dG.shape != dU.shape:
+        raise ValueError("dG and dU must have the same shape")
+    N = dG.shape[-1]
+    M = dG.numel() // N if N else 0
+    return M, N
+
+
+def swiglu_bwd_dx(dG: torch.Tensor, dU: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
+                  dX: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dX = dG Wg + dU Wu through the C ABI (bf16).  dG, dU [..., N] (leading
+    dims flattened to M rows), Wg, Wu [N, K]; dX has dG's leading dims."""
+    M, N = _bwd_shapes(dG, dU, "Wg", Wg)
+    _dev(Wu, "Wu")
+    K = Wg.shape[-1]
+    if Wg.shape != (N, K) or Wu.shape != (N, K) or Wu.dtype != Wg.dtype:
+        raise ValueError(f"weights must be bf16 [N, K] = [{N}, {K}]")
+    if dX is None:
+        dX = torch.empty((*dG.shape[:-1], K), dtype=dG.dtype, device=dG.device)
+    else:
+        _dev(dX, "dX")
+        if dX.dtype != dG.dtype or dX.numel() != M * K:
+            raise ValueError("dX has the wrong dtype or size")
+    st = lib().swiglu_bwd_dx(dG.data_ptr(), dU.data_ptr(), Wg.data_ptr(), Wu.data_ptr(),
+                             dX.data_ptr(), M, K, N, SWIGLU_BF16, _stream(stream))
+    _check("swiglu_bwd_dx", st)
+    return dX
+
+
+def swiglu_bwd_dw(dG: torch.Tensor, dU: torch.Tensor, X: torch.Tensor,
+                  dWg: torch.Tensor | None = None, dWu: torch.Tensor | None = None,
+                  stream=None):
+    """(dWg, dWu) = (dG^T X, dU^T X) through the C ABI (bf16).  dG, dU
+    [..., N] and X [..., K] with the same leading dims (M rows)."""
+    M, N = _bwd_shapes(dG, dU, "X", X)
+    K = X.shape[-1]
+    if X.numel() != M * K:
+        raise ValueError("X must have dG's leading dims")
+    dWg = torch.empty((N, K), dtype=X.dtype, device=X.device) if dWg is None else dWg
+    dWu = torch.empty((N, K), dtype=X.dtype, device=X.device) if dWu is None else dWu
+    for t, n in ((dWg, "dWg"), (dWu, "dWu")):
+        _dev(t, n)
+        if t.dtype != X.dtype or t.numel() != N * K:
+            raise ValueError(f"{n} has the wrong dtype or size")
+    st = lib().swiglu_bwd_dw(dG.data_ptr(), dU.data_ptr(), X.data_ptr(), dWg.data_ptr(),
+                             dWu.data_ptr(), M, K, N, SWIGLU_BF16, _stream(stream))
+    _check("swiglu_bwd_dw", st)
+    return dWg, dWu
 
 
 def swiglu_route_for(M: int, K: int, N: int, dtype: int) -> int:

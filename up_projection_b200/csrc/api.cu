@@ -150,6 +150,62 @@ int check_bwd(const void *dH, const void *G, const void *U, const void *dG, cons
     return SWIGLU_OK;
 }
 
+// Shape rules shared by the backward GEMMs (bf16 only).
+int check_bwd_shape(int64_t M, int64_t K, int64_t N, int dtype) {
+    if (dtype != SWIGLU_BF16) return SWIGLU_ERR_BAD_DTYPE;
+    if (M < 0 || K < 0 || N < 0) return SWIGLU_ERR_BAD_DIM;
+    if (M > kMaxDim || K > kMaxDim || N > kMaxDim) return SWIGLU_ERR_BAD_DIM;
+    if (K % 8 != 0 || N % 8 != 0) return SWIGLU_ERR_MISALIGNED_DIM;
+    return SWIGLU_OK;
+}
+
+// swiglu_bwd_dx: route NONE (nothing to write), ZERO_K (N == 0) or the GEMM.
+int check_bwd_dx(const void *dG, const void *dU, const void *Wg, const void *Wu, const void *dX,
+                 int64_t M, int64_t K, int64_t N, int dtype, int *route) {
+    int st = check_bwd_shape(M, K, N, dtype);
+    if (st != SWIGLU_OK) return st;
+    *route = SWIGLU_ROUTE_NONE;
+    if (M == 0 || K == 0) return SWIGLU_OK;
+    if (!dX) return SWIGLU_ERR_NULL_POINTER;
+    if (!aligned16(dX)) return SWIGLU_ERR_MISALIGNED_PTR;
+    *route = SWIGLU_ROUTE_ZERO_K;
+    if (N == 0) return SWIGLU_OK;
+    *route = SWIGLU_ROUTE_BWD_GEMM_BF16;
+    if (!dG || !dU || !Wg || !Wu) return SWIGLU_ERR_NULL_POINTER;
+    if (!aligned16(dG) || !aligned16(dU) || !aligned16(Wg) || !aligned16(Wu))
+        return SWIGLU_ERR_MISALIGNED_PTR;
+    const int64_t xb = M * K * 2, gb = M * N * 2, wb = N * K * 2;
+    if (overlaps(dX, xb, dG, gb) || overlaps(dX, xb, dU, gb) || overlaps(dX, xb, Wg, wb) ||
+        overlaps(dX, xb, Wu, wb))
+        return SWIGLU_ERR_OVERLAP;
+    return SWIGLU_OK;
+}
+
+// swiglu_bwd_dw: route NONE, ZERO_K (M == 0) or the GEMM.
+int check_bwd_dw(const void *dG, const void *dU, const void *X, const void *dWg,
+                 const void *dWu, int64_t M, int64_t K, int64_t N, int dtype, int *route) {
+    int st = check_bwd_shape(M, K, N, dtype);
+    if (st != SWIGLU_OK) return st;
+    *route = SWIGLU_ROUTE_NONE;
+    if (N == 0 || K == 0) return SWIGLU_OK;
+    if (!dWg || !dWu) return SWIGLU_ERR_NULL_POINTER;
+    if (!aligned16(dWg) || !aligned16(dWu)) return SWIGLU_ERR_MISALIGNED_PTR;
+    const int64_t wb = N * K * 2;
+    if (overlaps(dWg, wb, dWu, wb)) return SWIGLU_ERR_OVERLAP;
+    *route = SWIGLU_ROUTE_ZERO_K;
+    if (M == 0) return SWIGLU_OK;
+    *route = SWIGLU_ROUTE_BWD_GEMM_BF16;
+    if (!dG || !dU || !X) return SWIGLU_ERR_NULL_POINTER;
+    if (!aligned16(dG) || !aligned16(dU) || !aligned16(X)) return SWIGLU_ERR_MISALIGNED_PTR;
+    const int64_t gb = M * N * 2, xb = M * K * 2;
+    const void *outs[2] = {dWg, dWu};
+    for (const void *o : outs) {
+        if (overlaps(o, wb, dG, gb) || overlaps(o, wb, dU, gb) || overlaps(o, wb, X, xb))
+            return SWIGLU_ERR_OVERLAP;
+    }
+    return SWIGLU_OK;
+}
+
 int from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return SWIGLU_OK;
     (void)cudaGetLastError();
@@ -257,6 +313,57 @@ SWIGLU_API int dswiglu_bwd(const void *dH, const void *G, const void *U, void *d
     return dswiglu_bwd_dtype(dH, G, U, dG, dU, n, SWIGLU_BF16, stream);
 }
 
+SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                             void *dX, int64_t M, int64_t K, int64_t N, int dtype,
+                             cudaStream_t stream) {
+    int route = SWIGLU_ROUTE_NONE;
+    int st = check_bwd_dx(dG, dU, Wg, Wu, dX, M, K, N, dtype, &route);
+    if (st != SWIGLU_OK) return st;
+    if (route == SWIGLU_ROUTE_NONE) {
+        t_last_route = route;
+        return SWIGLU_OK;
+    }
+    DeviceInfo dev;
+    st = current_device(dev);
+    if (st != SWIGLU_OK) return st;
+    cudaError_t e;
+    if (route == SWIGLU_ROUTE_ZERO_K)
+        e = cudaMemsetAsync(dX, 0, static_cast<size_t>(M) * K * 2, stream);
+    else
+        e = launch_bwd_dx_bf16(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
+                               static_cast<int>(N), dev, stream);
+    st = from_cuda(e);
+    if (st == SWIGLU_OK) t_last_route = route;
+    return st;
+}
+
+SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X, void *dWg,
+                             void *dWu, int64_t M, int64_t K, int64_t N, int dtype,
+                             cudaStream_t stream) {
+    int route = SWIGLU_ROUTE_NONE;
+    int st = check_bwd_dw(dG, dU, X, dWg, dWu, M, K, N, dtype, &route);
+    if (st != SWIGLU_OK) return st;
+    if (route == SWIGLU_ROUTE_NONE) {
+        t_last_route = route;
+        return SWIGLU_OK;
+    }
+    DeviceInfo dev;
+    st = current_device(dev);
+    if (st != SWIGLU_OK) return st;
+    cudaError_t e;
+    if (route == SWIGLU_ROUTE_ZERO_K) {
+        const size_t bytes = static_cast<size_t>(N) * K * 2;
+        e = cudaMemsetAsync(dWg, 0, bytes, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dWu, 0, bytes, stream);
+    } else {
+        e = launch_bwd_dw_bf16(dG, dU, X, dWg, dWu, static_cast<int>(M), static_cast<int>(K),
+                               static_cast<int>(N), dev, stream);
+    }
+    st = from_cuda(e);
+    if (st == SWIGLU_OK) t_last_route = route;
+    return st;
+}
+
 SWIGLU_API int swiglu_last_route(void) { return t_last_route; }
 
 SWIGLU_API const char *swiglu_status_string(int status) {
@@ -284,14 +391,16 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0, w3 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = decode_status_fetch_and_clear(&w3, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2 | w3) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = gemm_bwd_status_fetch_and_clear(&w4, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3 | w4) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
 }
 
 SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes, void *sink,

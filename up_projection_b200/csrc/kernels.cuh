@@ -53,6 +53,18 @@ cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *d
                            void *dU, int64_t n, int dtype, int activation, float alpha,
                            const DeviceInfo &dev, cudaStream_t stream);
 
+// Backward GEMMs, bf16 (M, K, N >= 1; K, N multiples of 8):
+//   dX = dG Wg + dU Wu  (one accumulator),  dWg = dG^T X,  dWu = dU^T X.
+cudaError_t launch_bwd_dx_bf16(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                               void *dX, int M, int K, int N, const DeviceInfo &dev,
+                               cudaStream_t stream);
+cudaError_t launch_bwd_dw_bf16(const void *dG, const void *dU, const void *X, void *dWg,
+                               void *dWu, int M, int K, int N, const DeviceInfo &dev,
+                               cudaStream_t stream);
+// Output tile width (128, 192 or 256 columns) the backward GEMMs use for a raster
+// of `row_tiles_total` 128-row tiles by `cols` columns.
+int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
+
 // Pure streaming read of two buffers (bench-only floor probe).
 int read_floor_grid(const DeviceInfo &dev);
 cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
@@ -63,6 +75,7 @@ cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void 
 cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool tensor_maps_available();

@@ -216,6 +216,27 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
     return d;
 }
 
+// Descriptor for an MN-major operand (the M or N index contiguous in memory)
+// in the 128-byte swizzle.  The tile is a row of atoms, each 64 bf16 along MN
+// (one 128-byte swizzled row) by R reduction rows, as a TMA box {64, R}
+// writes it; groups of 8 reduction rows are 1024 B apart (stride byte
+// offset) and consecutive 64-wide MN atoms `atom_bytes` apart (leading byte
+// offset).  Atoms must start on 1024-byte boundaries.  16 reduction rows
+// further on = +2048 B = +128 in the start-address field.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t atom_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((atom_bytes >> 4) & 0x3FFFu) << 16;  // LBO: next MN atom
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;                   // SBO: next 8 rows
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
+// Instruction-descriptor bits that mark A (bit 15) or B (bit 16) as MN-major.
+constexpr uint32_t kIdescAMnMajor = 1u << 15;
+constexpr uint32_t kIdescBMnMajor = 1u << 16;
+
 // Same for a 64-byte swizzle (rows of 64 B, 8-row core groups 512 B apart);
 // the tile must start on a 512-byte boundary.
 __device__ __forceinline__ uint64_t sw64_kmajor_desc(uint32_t smem_addr) {

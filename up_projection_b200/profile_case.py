@@ -5,6 +5,8 @@
     python -m up_projection_b200.profile_case dswiglu --n 117440512 --launches 3
     python -m up_projection_b200.profile_case fp32    --M 2048 --K 5120 --N 13824 --launches 2
     python -m up_projection_b200.profile_case floor   --K 1536 --N 6912 --copies 4 --launches 3
+    python -m up_projection_b200.profile_case bwd_dx  --M 4096 --K 4096 --N 14336 --launches 2
+    python -m up_projection_b200.profile_case bwd_dw  --M 4096 --K 4096 --N 14336 --launches 2
 
 Each launch of the profiled kernel is preceded by nothing else of this
 library, so `ncu -k regex:<name> -s <skip> -c <count>` selects launches by
@@ -22,7 +24,8 @@ import torch
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "prefill", "dswiglu", "fp32", "floor"])
+    ap.add_argument("case", choices=["decode", "prefill", "dswiglu", "fp32", "floor", "bwd_dx",
+                                       "bwd_dw"])
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--K", type=int, default=1536)
     ap.add_argument("--N", type=int, default=6912)
@@ -60,6 +63,22 @@ def main(argv=None):
         H = torch.empty((a.M, a.N), dtype=dt, device=dev)
         for _ in range(L):
             up.swiglu_fwd(X, Wg, Wu, H)
+    elif a.case in ("bwd_dx", "bwd_dw"):
+        bf = torch.bfloat16
+        dG = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
+        dU = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
+        if a.case == "bwd_dx":
+            Wg = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+            Wu = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+            dX = torch.empty((a.M, a.K), dtype=bf, device=dev)
+            for _ in range(L):
+                up.swiglu_bwd_dx(dG, dU, Wg, Wu, dX)
+        else:
+            X = torch.randn((a.M, a.K), generator=g, device=dev).to(bf)
+            dWg = torch.empty((a.N, a.K), dtype=bf, device=dev)
+            dWu = torch.empty((a.N, a.K), dtype=bf, device=dev)
+            for _ in range(L):
+                up.swiglu_bwd_dw(dG, dU, X, dWg, dWu)
     else:
         dH, G, U = (torch.randn(a.n, generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
         dG, dU = torch.empty_like(G), torch.empty_like(U)

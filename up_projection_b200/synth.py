@@ -74,3 +74,15 @@ def integer_inputs(M: int, K: int, N: int, seed: int = 0, dtype: str = "bf16"):
     conv = (lambda a: torch.from_numpy(a).to(DTYPES[dtype])) if dtype != "f32" \
         else torch.from_numpy
     return conv(X), conv(Wg), conv(Wu)
+
+
+def ternary(shape, seed: int, density: float = 0.5, dtype: str = "bf16") -> torch.Tensor:
+    """Entries in {-1, 0, +1}: nonzero with probability `density`, either
+    sign equally likely.  For bit-exact checks of sums: every partial sum of
+    such entries (and of their products) is a small integer, exact in fp32
+    whatever the summation order."""
+    rng = np.random.Generator(np.random.PCG64(seed + 200))
+    mag = (rng.random(size=tuple(shape)) < density).astype(np.float32)
+    sign = np.where(rng.random(size=tuple(shape)) < 0.5, -1.0, 1.0).astype(np.float32)
+    t = torch.from_numpy(mag * sign)
+    return t.to(DTYPES[dtype]) if dtype != "f32" else t
