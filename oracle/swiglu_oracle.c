@@ -74,24 +74,32 @@ ORACLE_API double oracle_dsilu(double x)
 /*
  * GELU with the tanh approximation, the "GELU(tanh)" of the GEGLU variant
  * (TensorRT-LLM PR #17693 fuses GELU(tanh) into the up projection; Liger-
- * Kernel issue #937 lists swiglu/geglu): gelu(x) = x/2 (1 + tanh(c (x + a x^3)))
- * with c = sqrt(2/pi), a = 0.044715.  Derivative by differentiation.
+ * Kernel issue #937 lists swiglu/geglu): gelu(x) = x/2 (1 + tanh(y)),
+ * y = c (x + a x^3), c = sqrt(2/pi), a = 0.044715.
+ *
+ * Evaluated through the exact identities 1 + tanh(y) = 2 sigmoid(2y) and
+ * 1 - tanh(y)^2 = 4 sigmoid(2y) sigmoid(-2y): the same function, without
+ * the cancellation of 1 + tanh(y) for negative y (in double, tanh(y) rounds
+ * to -1 below y = -19, where gelu(x) ~ x e^(2y) would come out as 0, and
+ * loses ~13 bits already at y = -15).  Derivative by differentiation:
+ * gelu'(x) = s + 2 x s (1 - s) y',  s = sigmoid(2y),  y' = c (1 + 3 a x^2).
  */
 #define ORACLE_GELU_C 0.79788456080286535587989211986876 /* sqrt(2/pi) */
 #define ORACLE_GELU_A 0.044715
 
 ORACLE_API double oracle_gelu_tanh(double x)
 {
-    double t = tanh(ORACLE_GELU_C * (x + ORACLE_GELU_A * x * x * x));
-    return 0.5 * x * (1.0 + t);
+    double y = ORACLE_GELU_C * (x + ORACLE_GELU_A * x * x * x);
+    return x * oracle_sigmoid(2.0 * y);
 }
 
 ORACLE_API double oracle_dgelu_tanh(double x)
 {
     double y = ORACLE_GELU_C * (x + ORACLE_GELU_A * x * x * x);
-    double t = tanh(y);
+    double s = oracle_sigmoid(2.0 * y);
+    double oms = oracle_sigmoid(-2.0 * y);
     double dy = ORACLE_GELU_C * (1.0 + 3.0 * ORACLE_GELU_A * x * x);
-    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * dy;
+    return s + 2.0 * x * s * oms * dy;
 }
 
 /* Activation codes: 0 = SiLU, 1 = GELU(tanh). */

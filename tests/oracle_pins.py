@@ -43,6 +43,8 @@ What pins what:
                         (the multiplier acts on the gate pre-activation).
   variants_bwd          dG, dU of the variants against central differences of
                         the variant forward, and dU = dh act(alpha g).
+  gelu_high_precision   gelu, gelu' against the tanh definition in 120-digit
+                        mpmath arithmetic, x in [-12, 8].
   backward_gemms        dX, dWg, dWu against numpy matmul, and the whole chain
                         (forward, dSwiGLU, backward GEMMs) against central
                         differences of the scalar loss sum(dH * H) in X, Wg, Wu.
@@ -312,6 +314,39 @@ def gelu_closed_forms(o):
         assert o.dact(x, 1) == o.dgelu_tanh(x) and o.dact(x, 0) == o.dsilu(x)
 
 
+def gelu_high_precision(o):
+    """gelu and gelu' against the definition x/2 (1 + tanh(c(x + a x^3)))
+    evaluated in 120-digit arithmetic (mpmath), where 1 + tanh(y) does not
+    cancel: relative agreement over the whole range, including x < -5 where
+    a double-precision tanh form loses its digits."""
+    import mpmath
+    mpmath.mp.dps = 120
+    c = mpmath.sqrt(2 / mpmath.pi)
+    a = mpmath.mpf("0.044715")
+
+    def g(x):
+        return x / 2 * (1 + mpmath.tanh(c * (x + a * x ** 3)))
+    for xf in list(np.linspace(-12.0, 8.0, 81)) + [-6.578, -7.3, -9.5, 1e-3, -1e-3]:
+        x = mpmath.mpf(float(xf))
+        ref = g(x)
+        dref = mpmath.diff(g, x)
+        v, dv = o.gelu_tanh(float(xf)), o.dgelu_tanh(float(xf))
+        # e^(2y) turns the rounding of its double argument (a few ulp of
+        # |2y|) into a relative error of about |2y| ulp: the bound scales
+        # with |2y| (about 10 ulp at x = 0, 2.6e-13 at x = -12).
+        z = abs(2 * float(c) * (float(xf) + 0.044715 * float(xf) ** 3))
+        tol = 2.2e-16 * (20.0 + 8.0 * z)
+        assert abs(mpmath.mpf(v) - ref) <= tol * abs(ref), (xf, v, ref)
+        # gelu' = s + 2 x s (1 - s) y' cancels near the minimum of gelu
+        # (x ~ -0.75): relative to the size of its two terms there.
+        xv = float(xf)
+        sd = float(1 / (1 + mpmath.exp(-2 * c * (x + a * x ** 3))))
+        terms = abs(sd) + abs(2 * xv * sd * (1 - sd) * float(c) * (1 + 3 * 0.044715 * xv * xv))
+        assert abs(mpmath.mpf(dv) - dref) <= 2 * tol * max(abs(float(dref)), terms) + 1e-300, \
+            (xf, dv, dref)
+    assert o.gelu_tanh(-10.0) < 0.0 and o.dgelu_tanh(-10.0) != 0.0
+
+
 def variants_fwd(o):
     X, Wg, Wu = _random_problem(5, 64, 40, 90, scale_w=0.4)
     base = o.swiglu_fwd_f64(X, Wg, Wu)
@@ -392,4 +427,4 @@ ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
             fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
             fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
             dswiglu_special, dswiglu_storage, gelu_closed_forms, variants_fwd,
-            variants_bwd, backward_gemms]
+            variants_bwd, backward_gemms, gelu_high_precision]

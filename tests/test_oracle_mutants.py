@@ -24,7 +24,9 @@ MUTANTS = [
      "if (h_out) *h_out = oracle_act(alpha * g, act) * u;",
      "if (h_out) *h_out = alpha * oracle_act(g, act) * u;"),
     ("gelu_sign",
-     "return 0.5 * x * (1.0 + t);", "return 0.5 * x * (1.0 - t);"),
+     "return x * oracle_sigmoid(2.0 * y);", "return x * oracle_sigmoid(-2.0 * y);"),
+    ("dgelu_complement",
+     "double oms = oracle_sigmoid(-2.0 * y);", "double oms = oracle_sigmoid(2.0 * y);"),
     ("gelu_slope_cubic_term",
      "double dy = ORACLE_GELU_C * (1.0 + 3.0 * ORACLE_GELU_A * x * x);",
      "double dy = ORACLE_GELU_C * (1.0 + ORACLE_GELU_A * x * x);"),
