@@ -101,6 +101,14 @@ class Oracle:
                                                      ctypes.c_int, _D, _P, _P, _P, _P, _P]
         lib.oracle_dswiglu_act_f64.restype = None
         lib.oracle_dswiglu_act_f64.argtypes = [_P, _P, _P, _I64, ctypes.c_int, _D, _P, _P]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_int]
+        lib.oracle_e4m3_encode.restype = ctypes.c_int
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        lib.oracle_ue8m0_exponent.restype = ctypes.c_int
+        lib.oracle_ue8m0_exponent.argtypes = [ctypes.c_double]
+        lib.oracle_quant_e4m3.restype = None
+        lib.oracle_quant_e4m3.argtypes = [_P, _I64, _I64, _P, _P]
         lib.oracle_bwd_dx_f64.restype = None
         lib.oracle_bwd_dx_f64.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _P]
         lib.oracle_bwd_dw_f64.restype = None
@@ -236,6 +244,29 @@ class Oracle:
             raise MemoryError("oracle: row buffer allocation failed")
         return out
 
+    # ---- quantised output ------------------------------------------------------
+    def e4m3_decode(self, code: int) -> float:
+        return self.lib.oracle_e4m3_decode(int(code))
+
+    def e4m3_encode(self, v: float) -> int:
+        return self.lib.oracle_e4m3_encode(float(v))
+
+    def ue8m0_exponent(self, amax: float) -> int:
+        return self.lib.oracle_ue8m0_exponent(float(amax))
+
+    def quant_e4m3(self, H):
+        """(q uint8 [M,N] e4m3 codes, s uint8 [M, ceil(N/32)] UE8M0 codes)
+        of a float64 [M,N] array, per (1,32) block."""
+        H = np.ascontiguousarray(H, dtype=np.float64)
+        if H.ndim == 1:
+            H = H[None, :]
+        M, N = H.shape
+        q = np.empty((M, N), dtype=np.uint8)
+        s = np.empty((M, (N + 31) // 32), dtype=np.uint8)
+        self.lib.oracle_quant_e4m3(_ptr(H), M, N, q.ctypes.data_as(ctypes.c_void_p),
+                                   s.ctypes.data_as(ctypes.c_void_p))
+        return q, s
+
     # ---- backward GEMMs -------------------------------------------------------
     def bwd_dx_f64(self, dG, dU, Wg, Wu):
         """dX [M,K] = dG Wg + dU Wu for dG, dU [M,N] and Wg, Wu [N,K]."""
@@ -306,6 +337,7 @@ def __getattr__(name):
     if name in {"sigmoid", "silu", "dsilu", "gelu_tanh", "dgelu_tanh", "act", "dact",
                 "decode_bf16", "decode",
                 "swiglu_fwd_f64", "swiglu_fwd", "swiglu_fwd_points",
-                "dswiglu_f64", "dswiglu", "bwd_dx_f64", "bwd_dw_f64"}:
+                "dswiglu_f64", "dswiglu", "bwd_dx_f64", "bwd_dw_f64",
+                "e4m3_decode", "e4m3_encode", "ue8m0_exponent", "quant_e4m3"}:
         return getattr(default(), name)
     raise AttributeError(name)

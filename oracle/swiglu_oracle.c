@@ -413,3 +413,103 @@ ORACLE_API void oracle_bwd_dw_f64(const double *dG, const double *dU,
         }
     }
 }
+
+/* ---- quantised output: fp8 e4m3 with UE8M0 block scales ------------------ */
+
+/*
+ * The quantised output of the SwiGLU kernels of TileKernels-PTO PR #20
+ * (implementation notes and validation: fp8 e4m3 output, UE8M0 scale
+ * factors per sf_block = (1, 32), block amax, NaN-preserving casts).  The
+ * page does not write the scale rule out; the reading used here: for each
+ * row and each block of 32 consecutive columns (the last block may be
+ * shorter),
+ *   amax = max |h| over the block,
+ *   e    = the smallest integer with amax <= 448 * 2^e (448 = largest finite
+ *          e4m3), clamped to [-127, 127]; amax = 0 gives e = -127,
+ *   scale code = e + 127 (UE8M0: an 8-bit biased power of two),
+ *   q    = e4m3(h / 2^e), round to nearest, ties to even.
+ * A block holding Inf or NaN gets scale code 0xFF (NaN) and NaN codes.
+ *
+ * e4m3 ("fn": no infinities): sign bit, 4 exponent bits (bias 7), 3
+ * mantissa bits; exponent field 0 holds subnormals m/8 * 2^-6; S.1111.111 is
+ * NaN; the largest finite value is 1.75 * 2^8 = 448.
+ */
+ORACLE_API double oracle_e4m3_decode(int code)
+{
+    int sign = (code >> 7) & 1;
+    int ef = (code >> 3) & 15;
+    int mf = code & 7;
+    double v;
+    if (ef == 15 && mf == 7)
+        return NAN;
+    if (ef == 0)
+        v = ldexp((double)mf / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)mf / 8.0, ef - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 code by exhaustive search over the 127 non-negative finite
+ * codes; an exact tie goes to the even code (mantissa LSB 0).  |v| > 448
+ * has no finite code: NaN (the casts do not saturate). */
+ORACLE_API int oracle_e4m3_encode(double v)
+{
+    if (isnan(v) || fabs(v) > 448.0)
+        return 0x7F;
+    double a = fabs(v);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(oracle_e4m3_decode(c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (v < 0.0 || (v == 0.0 && signbit(v))) ? (best | 0x80) : best;
+}
+
+/* The UE8M0 exponent e of a block with maximum magnitude amax (finite). */
+ORACLE_API int oracle_ue8m0_exponent(double amax)
+{
+    if (amax == 0.0)
+        return -127;
+    int e = -127;
+    while (e < 127 && amax > 448.0 * ldexp(1.0, e))
+        ++e;
+    return e;
+}
+
+/* Quantise one row of n values: q[n] codes, s[ceil(n/32)] scale codes. */
+ORACLE_API void oracle_quant_e4m3_row(const double *h, int64_t n, uint8_t *q, uint8_t *s)
+{
+    for (int64_t b = 0; b * 32 < n; ++b) {
+        int64_t lo = b * 32, hi = lo + 32 < n ? lo + 32 : n;
+        double amax = 0.0;
+        int finite = 1;
+        for (int64_t j = lo; j < hi; ++j) {
+            if (!isfinite(h[j]))
+                finite = 0;
+            else if (fabs(h[j]) > amax)
+                amax = fabs(h[j]);
+        }
+        if (!finite) {
+            s[b] = 0xFF;
+            for (int64_t j = lo; j < hi; ++j)
+                q[j] = 0x7F;
+            continue;
+        }
+        int e = oracle_ue8m0_exponent(amax);
+        s[b] = (uint8_t)(e + 127);
+        for (int64_t j = lo; j < hi; ++j)
+            q[j] = (uint8_t)oracle_e4m3_encode(ldexp(h[j], -e));
+    }
+}
+
+ORACLE_API void oracle_quant_e4m3(const double *H, int64_t M, int64_t N, uint8_t *q, uint8_t *s)
+{
+    int64_t nb = (N + 31) / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        oracle_quant_e4m3_row(H + m * N, N, q + m * N, s + m * nb);
+}

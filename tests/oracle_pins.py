@@ -45,6 +45,14 @@ What pins what:
                         the variant forward, and dU = dh act(alpha g).
   gelu_high_precision   gelu, gelu' against the tanh definition in 120-digit
                         mpmath arithmetic, x in [-12, 8].
+  e4m3_codec            the e4m3 decode of all 256 codes and the round-to-
+                        nearest-even encode of ties, subnormals and random
+                        values against torch's float8_e4m3fn conversion.
+  ue8m0_scale           closed forms of the block exponent (powers of two
+                        times 448, just above them, clamps).
+  quant_blocks          per-(1,32)-block quantisation: dequantised values
+                        within half an e4m3 step, the block maximum lands in
+                        (224, 448], ragged last block, non-finite blocks.
   backward_gemms        dX, dWg, dWu against numpy matmul, and the whole chain
                         (forward, dSwiGLU, backward GEMMs) against central
                         differences of the scalar loss sum(dH * H) in X, Wg, Wu.
@@ -423,8 +431,71 @@ def backward_gemms(o):
             assert abs(fd - grad[idx]) <= 1e-7 * (1 + abs(fd)), (name, idx, fd, grad[idx])
 
 
+def e4m3_codec(o):
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        v = o.e4m3_decode(c)
+        if np.isnan(ref[c]):
+            assert np.isnan(v), c
+        else:
+            assert v == ref[c] and (np.signbit(v) == np.signbit(ref[c])), (c, v, ref[c])
+    finite = np.sort(np.unique(np.abs(ref[np.isfinite(ref)])))
+    mids = (finite[:-1] + finite[1:]) / 2           # exact ties between codes
+    r = _rng(31)
+    vals = np.concatenate([finite, mids, -mids, r.uniform(-448, 448, 3000),
+                           r.uniform(-2 ** -6, 2 ** -6, 500), [0.0, -0.0, 2 ** -10, 2 ** -9 * 0.5]])
+    t = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for v, c in zip(vals, t):
+        assert o.e4m3_encode(float(v)) == int(c), (v, o.e4m3_encode(float(v)), int(c))
+    assert o.e4m3_encode(448.5) == 0x7F and o.e4m3_encode(float("nan")) == 0x7F
+
+
+def ue8m0_scale(o):
+    for k in range(-120, 120, 7):
+        a = 448.0 * 2.0 ** k
+        assert o.ue8m0_exponent(a) == k
+        assert o.ue8m0_exponent(a * (1 + 2 ** -40)) == k + 1
+        assert o.ue8m0_exponent(a * (1 - 2 ** -40)) == k
+    assert o.ue8m0_exponent(1.0) == -8          # 448 / 256 = 1.75 >= 1 > 0.875
+    assert o.ue8m0_exponent(0.0) == -127
+    assert o.ue8m0_exponent(1e-300) == -127     # clamped below
+    assert o.ue8m0_exponent(1e300) == 127       # clamped above
+
+
+def quant_blocks(o):
+    r = _rng(32)
+    H = r.standard_normal((6, 100)) * np.exp(r.uniform(-8, 8, (6, 1)))
+    H[2, 40:50] *= 1e3          # one block with a much larger maximum
+    H[3, 64:96] = 0.0           # an all-zero block
+    q, s = o.quant_e4m3(H)
+    assert q.shape == (6, 100) and s.shape == (6, 4)   # ragged last block of 4
+    dec = np.vectorize(o.e4m3_decode)
+    for m in range(6):
+        for b in range(4):
+            lo, hi = 32 * b, min(32 * b + 32, 100)
+            e = int(s[m, b]) - 127
+            blk = H[m, lo:hi]
+            d = dec(q[m, lo:hi]) * 2.0 ** e
+            if not np.any(blk):
+                assert e == -127 and not np.any(d)
+                continue
+            # the largest element lands in (224, 448] after scaling
+            assert 224.0 < np.max(np.abs(blk)) * 2.0 ** -e <= 448.0
+            # within half a step of the e4m3 grid (relative 2^-4 for normals,
+            # absolute 2^-10 * 2^e in the subnormal range)
+            step = np.maximum(np.abs(blk) * 2.0 ** -3, 2.0 ** (e - 9))
+            assert np.all(np.abs(d - blk) <= 0.5 * step + 1e-300), (m, b)
+    bad = np.zeros((1, 64))
+    bad[0, 3] = np.inf
+    bad[0, 40] = np.nan
+    q, s = o.quant_e4m3(bad)
+    assert list(s[0]) == [0xFF, 0xFF] and np.all(q == 0x7F)
+
+
 ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
             fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
             fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
             dswiglu_special, dswiglu_storage, gelu_closed_forms, variants_fwd,
-            variants_bwd, backward_gemms, gelu_high_precision]
+            variants_bwd, backward_gemms, gelu_high_precision, e4m3_codec, ue8m0_scale,
+            quant_blocks]

@@ -47,6 +47,14 @@ MUTANTS = [
      "acc += dG[m * N + n] * Wu[n * K + k] + dU[m * N + n] * Wg[n * K + k];"),
     ("dw_transposed_index",
      "ag += dG[m * N + n] * X[m * K + k];", "ag += dG[m * N + n] * X[m * K + (K - 1 - k)];"),
+    ("e4m3_ties_to_odd",
+     "(d == best_d && (c & 1) == 0 && (best & 1) == 1)", "(d == best_d && (c & 1) == 1 && (best & 1) == 0)"),
+    ("ue8m0_off_by_one",
+     "while (e < 127 && amax > 448.0 * ldexp(1.0, e))", "while (e < 127 && amax >= 448.0 * ldexp(1.0, e))"),
+    ("quant_block_16",
+     "int64_t lo = b * 32, hi = lo + 32 < n ? lo + 32 : n;", "int64_t lo = b * 32, hi = lo + 16 < n ? lo + 16 : n;"),
+    ("e4m3_exponent_bias",
+     "v = ldexp(1.0 + (double)mf / 8.0, ef - 7);", "v = ldexp(1.0 + (double)mf / 8.0, ef - 8);"),
     ("bf16_decode_shift",
      "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)b) << 15;"),
     ("magnitude_missing_abs",
