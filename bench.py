@@ -451,6 +451,19 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
+    # fp8 output: e4m3 H with UE8M0 scales per (1,32) block
+    Hq = torch.empty((M, N), dtype=torch.uint8, device=dev)
+    Hs = torch.empty((M, N // 32), dtype=torch.uint8, device=dev)
+    ms = time_op(lambda: up.lib().swiglu_fwd_fp8(
+        X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), Hq.data_ptr(), Hs.data_ptr(), M, K, N,
+        None, stream.cuda_stream))
+    tf = fl / (ms * 1e-3) / 1e12
+    add({"workload": "prefill, fp8 e4m3 H + UE8M0 (1,32) scales, LLaMA-3 8B bf16 in",
+         "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+         "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": round(tf / pk["bf16_tflops"], 4)}})
+    del Hq, Hs
     # backward GEMMs at the same size: dX = dG Wg + dU Wu and dWg, dWu
     dGb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)
     dUb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)

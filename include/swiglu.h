@@ -163,6 +163,32 @@ SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu
                                    unsigned int flags, cudaStream_t stream);
 
 /*
+ * swiglu_fwd_fp8 -- the forward with a quantised output: H = act(alpha G) U
+ * as fp8 e4m3 with one UE8M0 scale per (1,32) block of a row (the e4m3
+ * output and sf_block = (1,32) UE8M0 scale factors of TileKernels-PTO
+ * PR #20, implementation notes).  For each row m and block b of columns
+ * [32b, min(32b+32, N)), from the fp32 epilogue values h:
+ *   amax = max |h|,  e = the smallest integer with amax <= 448 * 2^e,
+ *   clamped to [-127, 127] (amax = 0: e = -127),
+ *   Hs[m, b] = e + 127,   Hq[m, n] = e4m3_rne(h / 2^e)  (|h / 2^e| <= 448).
+ * A block holding Inf or NaN: Hs = 0xFF and every code 0x7F (NaN).
+ * Dequantised value: e4m3(Hq) * 2^(Hs - 127).
+ *
+ *  X, Wg, Wu  as swiglu_fwd, bf16 only (dtype argument absent).
+ *  Hq   [M, N] device bytes (e4m3 codes), 16-byte aligned; N a multiple of 16.
+ *  Hs   [M, ceil(N/32)] device bytes (UE8M0 codes), any alignment.
+ *  epi  NULL or activation + gate multiplier; epi->G / epi->U must be NULL
+ *       (SWIGLU_ERR_BAD_EPILOGUE otherwise).
+ *  Every M takes the tcgen05 dual GEMM (route SWIGLU_ROUTE_GEMM_BF16).
+ *  K == 0: Hq and Hs are set to 0.  Outputs must not overlap each other or
+ *  an input.  Allocates no device memory.
+ */
+SWIGLU_API int swiglu_fwd_fp8(const void *X, const void *Wg, const void *Wu,
+                              void *Hq, void *Hs, int64_t M, int64_t K,
+                              int64_t N, const swiglu_epilogue *epi,
+                              cudaStream_t stream);
+
+/*
  * dswiglu_bwd -- elementwise dSwiGLU, bf16.
  *
  *  dH, G, U  [n] device bf16 inputs, 16-byte aligned.

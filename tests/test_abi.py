@@ -170,3 +170,22 @@ def test_bwd_gemm_no_device_is_an_error():
     # empty reduction still needs the device (it writes zeros)
     assert lib.swiglu_bwd_dw(None, None, None, 1 << 20, 1 << 21, 0, 64, 64, 0,
                              None) == _capi.SWIGLU_ERR_NO_DEVICE
+
+
+def test_fwd_fp8_host_validation():
+    import ctypes
+    lib = _capi.lib()
+    ok = (1 << 20, 1 << 21, 1 << 22, 1 << 23, 1 << 24)
+    assert lib.swiglu_fwd_fp8(*ok, 4, 64, 40, None, None) == _capi.SWIGLU_ERR_MISALIGNED_DIM  # N % 16
+    assert lib.swiglu_fwd_fp8(*ok, 4, 60, 64, None, None) == _capi.SWIGLU_ERR_MISALIGNED_DIM  # K % 8
+    assert lib.swiglu_fwd_fp8(1 << 20, 1 << 21, 1 << 22, None, 1 << 24, 4, 64, 64, None,
+                              None) == _capi.SWIGLU_ERR_NULL_POINTER
+    assert lib.swiglu_fwd_fp8(1 << 20, 1 << 21, 1 << 22, (1 << 23) + 8, 1 << 24, 4, 64, 64, None,
+                              None) == _capi.SWIGLU_ERR_MISALIGNED_PTR
+    # scales may sit at any byte; Hq [4,64] bytes overlapping Hs
+    assert lib.swiglu_fwd_fp8(1 << 20, 1 << 21, 1 << 22, 1 << 23, (1 << 23) + 255, 4, 64, 64,
+                              None, None) == _capi.SWIGLU_ERR_OVERLAP
+    with_gu = _capi.Epilogue(0, 1.0, 1 << 25, 1 << 26)
+    assert lib.swiglu_fwd_fp8(*ok, 4, 64, 64, ctypes.byref(with_gu), None) == \
+        _capi.SWIGLU_ERR_BAD_EPILOGUE
+    assert lib.swiglu_fwd_fp8(None, None, None, None, None, 0, 64, 64, None, None) == _capi.SWIGLU_OK

@@ -164,6 +164,12 @@ def test_bwd_python_binding_shapes():
                       "dX via binding")
     with pytest.raises(TypeError):
         _capi.swiglu_bwd_dx(dGd.float(), dUd.float(), Wgd.float(), Wud.float())
+    # N == 0 through the binding: dX = 0 (empty reduction), dW empty
+    e = torch.empty((5, 0), dtype=torch.bfloat16, device=dev())
+    w = torch.empty((0, 64), dtype=torch.bfloat16, device=dev())
+    dX0 = _capi.swiglu_bwd_dx(e, e, w, w)
+    torch.cuda.synchronize()
+    assert dX0.shape == (5, 64) and not bool(dX0.any())
 
 
 def test_training_step_full_size_sampled():

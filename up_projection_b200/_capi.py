@@ -65,6 +65,7 @@ SIGNATURES = {
     "dswiglu_bwd_epilogue": (_I, [_P, _P, _P, _P, _P, _I64, _I, _I, ctypes.c_float, _P]),
     "dswiglu_bwd": (_I, [_P, _P, _P, _P, _P, _I64, _P]),
     "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
+    "swiglu_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.POINTER(Epilogue), _P]),
     "swiglu_bwd_dx": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_bwd_dw": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
@@ -209,6 +210,33 @@ def dswiglu_bwd(dH: torch.Tensor, G: torch.Tensor, U: torch.Tensor,
     return dG, dU
 
 
+def swiglu_fwd_fp8(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor, stream=None,
+                   activation: int = SWIGLU_ACT_SILU, gate_multiplier: float = 1.0):
+    """Quantised forward through the C ABI: returns (Hq, Hs) with Hq the
+    e4m3 codes [..., N] (torch.uint8) and Hs the UE8M0 scale codes
+    [..., ceil(N/32)] (torch.uint8) of H = act(gate_multiplier G) U; the
+    value of element n is e4m3(Hq) * 2^(Hs[n // 32] - 127).  bf16 inputs."""
+    for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
+        _dev(t, n)
+    if not (X.dtype == Wg.dtype == Wu.dtype == torch.bfloat16):
+        raise TypeError("swiglu_fwd_fp8 takes bfloat16 X, Wg, Wu")
+    K = X.shape[-1]
+    N = Wg.shape[0]
+    if Wg.shape != (N, K) or Wu.shape != (N, K):
+        raise ValueError(f"weights must be [N, K] = [{N}, {K}]")
+    lead = X.shape[:-1]
+    M = 1
+    for d in lead:
+        M *= d
+    Hq = torch.empty((*lead, N), dtype=torch.uint8, device=X.device)
+    Hs = torch.empty((*lead, (N + 31) // 32), dtype=torch.uint8, device=X.device)
+    epi = Epilogue(int(activation), float(gate_multiplier), None, None)
+    st = lib().swiglu_fwd_fp8(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), Hq.data_ptr(),
+                              Hs.data_ptr(), M, K, N, ctypes.byref(epi), _stream(stream))
+    _check("swiglu_fwd_fp8", st)
+    return Hq, Hs
+
+
 def _bwd_shapes(dG, dU, name_w, W):
     for t, n in ((dG, "dG"), (dU, "dU"), (W, name_w)):
         _dev(t, n)
@@ -217,7 +245,9 @@ def _bwd_shapes(dG, dU, name_w, W):
     if dG.shape != dU.shape:
         raise ValueError("dG and dU must have the same shape")
     N = dG.shape[-1]
-    M = dG.numel() // N if N else 0
+    M = 1
+    for d in dG.shape[:-1]:
+        M *= d
     return M, N
 
 

@@ -288,6 +288,62 @@ SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu
     return st;
 }
 
+SWIGLU_API int swiglu_fwd_fp8(const void *X, const void *Wg, const void *Wu, void *Hq, void *Hs,
+                              int64_t M, int64_t K, int64_t N, const swiglu_epilogue *epi,
+                              cudaStream_t stream) {
+    int route = SWIGLU_ROUTE_NONE;
+    int st = route_of_shape(M, K, N, SWIGLU_BF16, &route);
+    if (st != SWIGLU_OK) return st;
+    if (N % 16 != 0) return SWIGLU_ERR_MISALIGNED_DIM;
+    if (epi) {
+        if (epi->activation != SWIGLU_ACT_SILU && epi->activation != SWIGLU_ACT_GELU_TANH)
+            return SWIGLU_ERR_BAD_EPILOGUE;
+        if (!isfinite(epi->gate_multiplier)) return SWIGLU_ERR_BAD_EPILOGUE;
+        if (epi->G || epi->U) return SWIGLU_ERR_BAD_EPILOGUE;
+    }
+    if (route == SWIGLU_ROUTE_NONE) {
+        t_last_route = route;
+        return SWIGLU_OK;
+    }
+    if (!Hq || !Hs) return SWIGLU_ERR_NULL_POINTER;
+    if (!aligned16(Hq)) return SWIGLU_ERR_MISALIGNED_PTR;
+    const int64_t qb = M * N, sb = M * ((N + 31) / 32);
+    if (overlaps(Hq, qb, Hs, sb)) return SWIGLU_ERR_OVERLAP;
+    if (route != SWIGLU_ROUTE_ZERO_K) {
+        route = SWIGLU_ROUTE_GEMM_BF16;   // every M: the epilogue quantises
+        if (!X || !Wg || !Wu) return SWIGLU_ERR_NULL_POINTER;
+        if (!aligned16(X) || !aligned16(Wg) || !aligned16(Wu)) return SWIGLU_ERR_MISALIGNED_PTR;
+        const int64_t xb = M * K * 2, wb = N * K * 2;
+        const void *outs[2] = {Hq, Hs};
+        const int64_t ob[2] = {qb, sb};
+        for (int i = 0; i < 2; ++i)
+            if (overlaps(outs[i], ob[i], X, xb) || overlaps(outs[i], ob[i], Wg, wb) ||
+                overlaps(outs[i], ob[i], Wu, wb))
+                return SWIGLU_ERR_OVERLAP;
+    }
+    DeviceInfo dev;
+    st = current_device(dev);
+    if (st != SWIGLU_OK) return st;
+    cudaError_t e;
+    if (route == SWIGLU_ROUTE_ZERO_K) {
+        // h = 0 everywhere: e4m3 code 0 and the scale code of amax = 0 (0).
+        e = cudaMemsetAsync(Hq, 0, static_cast<size_t>(qb), stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(Hs, 0, static_cast<size_t>(sb), stream);
+    } else {
+        Epilogue ep;
+        if (epi) {
+            ep.activation = epi->activation;
+            ep.gate_multiplier = epi->gate_multiplier;
+        }
+        ep.scales = Hs;
+        e = launch_gemm_bf16(X, Wg, Wu, Hq, static_cast<int>(M), static_cast<int>(K),
+                             static_cast<int>(N), ep, dev, stream);
+    }
+    st = from_cuda(e);
+    if (st == SWIGLU_OK) t_last_route = route;
+    return st;
+}
+
 SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U, void *dG,
                                     void *dU, int64_t n, int dtype, int activation,
                                     float gate_multiplier, cudaStream_t stream) {

@@ -80,6 +80,56 @@ __device__ __forceinline__ float gated_fast(int which, float alpha, uint32_t gbi
     return act::gated<false>(which, alpha, __uint_as_float(gbits), __uint_as_float(ubits));
 }
 
+// fp8 output of one (1,32) block held by this lane: h = act(alpha g) u for
+// the 32 accumulator pairs, amax, the UE8M0 exponent e = the smallest
+// integer with amax <= 448 * 2^e (clamped to [-127, 127]), and the e4m3
+// codes of h / 2^e (round to nearest even; |h / 2^e| <= 448, so the
+// saturating conversion never saturates a finite block).  A block holding
+// Inf or NaN gets scale code 0xFF and NaN codes.  Returns the scale code;
+// q receives the 32 codes, 4 per word, column order.
+__device__ __forceinline__ uint32_t quant_block_e4m3(int which, float alpha, const uint32_t (&g)[32],
+                                                    const uint32_t (&u)[32], uint32_t (&q)[8]) {
+    float h[32];
+    float amax = 0.0f;
+    bool finite = true;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        h[i] = gated_fast(which, alpha, g[i], u[i]);
+        finite = finite && ((__float_as_uint(h[i]) & 0x7f800000u) != 0x7f800000u);
+        amax = fmaxf(amax, fabsf(h[i]));
+    }
+    if (!finite) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = 0x7f7f7f7fu;
+        return 0xFFu;
+    }
+    const uint32_t bits = __float_as_uint(amax);
+    const int ef = static_cast<int>(bits >> 23);          // amax >= 0
+    int e = -127;
+    if (ef != 0) {
+        // amax = 1.f * 2^(ef-127) <= 1.75 * 2^(e+8)
+        e = (ef - 127) - 8 + ((bits & 0x7fffffu) > 0x600000u ? 1 : 0);
+        e = max(-127, min(127, e));
+    }
+    // h * 2^-e as two exact power-of-two products (each factor normal)
+    const int n1 = (-e) / 2, n2 = -e - n1;
+    const float s1 = __uint_as_float(static_cast<uint32_t>(127 + n1) << 23);
+    const float s2 = __uint_as_float(static_cast<uint32_t>(127 + n2) << 23);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        // cvt ... d, a, b puts a in the upper byte: column order in memory
+        unsigned short lo, hi;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(lo)
+            : "f"(h[4 * i + 1] * s1 * s2), "f"(h[4 * i] * s1 * s2));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(hi)
+            : "f"(h[4 * i + 3] * s1 * s2), "f"(h[4 * i + 2] * s1 * s2));
+        q[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    return static_cast<uint32_t>(e + 127);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -93,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tm_g,
                             const __grid_constant__ CUtensorMap tm_u, int M, int N, int K,
                             int num_m_tiles, int num_n_tiles, int which_act, float alpha,
-                            int store_gu) {
+                            int store_gu, uint8_t *__restrict__ scales) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -249,11 +299,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kAccCols);
+            if (scales != nullptr) {
+                // fp8 output: the lane's row, one (1,32) block per 32 columns.
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+                const int row = m0 + quad * 32 + lane;
+                const int nblk = (N + 31) / 32;
+#pragma unroll 1
+                for (int b = 0; b < kBN / 32; ++b) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(tacc + 32u * b, g);
+                    tmem_ld_32x32b_x32(tacc + kBN + 32u * b, u);
+                    tmem_ld_wait(g);
+                    tmem_ld_wait(u);
+                    uint32_t q[8];
+                    const uint32_t code = quant_block_e4m3(which_act, alpha, g, u, q);
+                    sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
+                               ((static_cast<uint32_t>(2 * b) ^ swz) << 4),
+                           make_uint4(q[0], q[1], q[2], q[3]));
+                    sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
+                               ((static_cast<uint32_t>(2 * b + 1) ^ swz) << 4),
+                           make_uint4(q[4], q[5], q[6], q[7]));
+                    const int cb = n0 / 32 + b;
+                    if (row < M && cb < nblk)
+                        scales[static_cast<long long>(row) * nblk + cb] = static_cast<uint8_t>(code);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int y = m0 + quad * 32;
+                    if (n0 < N && y < M) {
+                        tma_store_2d(&tm_h, buf, n0, y);
+                        bulk_commit();
+                    }
+                }
+            }
             // Per 64-column chunk: H = act(alpha g) u, then (training
             // forward) G and U themselves, each staged and stored by TMA.
-            const int outputs = store_gu ? 3 : 1;
+            const int outputs = scales != nullptr ? 0 : (store_gu ? 3 : 1);
 #pragma unroll 1
-            for (int c = 0; c < kBN / 64; ++c) {
+            for (int c = 0; c < (outputs ? kBN / 64 : 0); ++c) {
 #pragma unroll 1
                 for (int what = 0; what < outputs; ++what) {
                     // The previous store from this buffer must have read it.
@@ -335,10 +420,15 @@ cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void
     const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     const bool store_gu = epi.G != nullptr;
-    if (!encode_tmap_2d(&tx, X, bf16, K, M, static_cast<uint64_t>(K) * 2, kBK, kBM, sw) ||
+    const bool fp8 = epi.scales != nullptr;
+    // fp8 output: H is [M, N] bytes stored in 128-column boxes.
+    const bool h_ok = fp8 ? encode_tmap_2d(&th, H, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, M,
+                                           static_cast<uint64_t>(N), 128, 32, sw)
+                          : encode_tmap_2d(&th, H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64,
+                                           32, sw);
+    if (!h_ok || !encode_tmap_2d(&tx, X, bf16, K, M, static_cast<uint64_t>(K) * 2, kBK, kBM, sw) ||
         !encode_tmap_2d(&twg, Wg, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
         !encode_tmap_2d(&twu, Wu, bf16, K, N, static_cast<uint64_t>(K) * 2, kBK, kBN, sw) ||
-        !encode_tmap_2d(&th, H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32, sw) ||
         !encode_tmap_2d(&tg, store_gu ? epi.G : H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32,
                         sw) ||
         !encode_tmap_2d(&tu, store_gu ? epi.U : H, bf16, N, M, static_cast<uint64_t>(N) * 2, 64, 32,
@@ -359,7 +449,7 @@ cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
     swiglu_gemm_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
         tx, twg, twu, th, tg, tu, M, N, K, num_m, num_n, epi.activation, epi.gate_multiplier,
-        store_gu ? 1 : 0);
+        store_gu ? 1 : 0, static_cast<uint8_t *>(epi.scales));
     return cudaGetLastError();
 }
 

@@ -17,6 +17,9 @@ struct Epilogue {
     float gate_multiplier = 1.0f;
     void *G = nullptr;
     void *U = nullptr;
+    // fp8 output (bf16 dual GEMM only): H is e4m3 [M, N] and `scales` the
+    // UE8M0 codes [M, ceil(N/32)] of its (1,32) blocks; G/U not stored.
+    void *scales = nullptr;
 };
 
 struct DeviceInfo {
