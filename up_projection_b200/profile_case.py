@@ -5,6 +5,7 @@
     python -m up_projection_b200.profile_case dswiglu --n 117440512 --launches 3
     python -m up_projection_b200.profile_case fp32    --M 2048 --K 5120 --N 13824 --launches 2
     python -m up_projection_b200.profile_case floor   --K 1536 --N 6912 --copies 4 --launches 3
+    python -m up_projection_b200.profile_case fp8     --M 4096 --K 4096 --N 14336 --launches 2
     python -m up_projection_b200.profile_case bwd_dx  --M 4096 --K 4096 --N 14336 --launches 2
     python -m up_projection_b200.profile_case bwd_dw  --M 4096 --K 4096 --N 14336 --launches 2
 
@@ -25,7 +26,7 @@ import torch
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode", "prefill", "dswiglu", "fp32", "floor", "bwd_dx",
-                                       "bwd_dw"])
+                                       "bwd_dw", "fp8"])
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--K", type=int, default=1536)
     ap.add_argument("--N", type=int, default=6912)
@@ -63,6 +64,13 @@ def main(argv=None):
         H = torch.empty((a.M, a.N), dtype=dt, device=dev)
         for _ in range(L):
             up.swiglu_fwd(X, Wg, Wu, H)
+    elif a.case == "fp8":
+        bf = torch.bfloat16
+        X = torch.randn((a.M, a.K), generator=g, device=dev).to(bf)
+        Wg = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+        Wu = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+        for _ in range(L):
+            up.swiglu_fwd_fp8(X, Wg, Wu)
     elif a.case in ("bwd_dx", "bwd_dw"):
         bf = torch.bfloat16
         dG = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
