@@ -348,22 +348,33 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
     out["H"] = {M: Hd[M].cpu() for M in Ms}
 
     if with_e2e:
-        # Through the public API with host buffers: pinned X in, H out, every
-        # call, inside the timed region.
-        Xp = {M: Xs_host[M].pin_memory() for M in Ms}
-        Hp = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
-        h2d = sum(Xp[M].numel() * 2 for M in Ms)
-        d2h = sum(Hp[M].numel() * 2 for M in Ms)
+        # Through the public API with host buffers, every step: one pinned
+        # host->device copy of the step's four X (packed rows), the four
+        # calls on row views of the packed device buffer, one device->host
+        # copy of the four H (packed rows) -- all inside the timed region.
+        rows = sum(Ms)
+        offs, o = {}, 0
+        for M in Ms:
+            offs[M] = o
+            o += M
+        Xpack_h = torch.cat([Xs_host[M] for M in Ms], 0).pin_memory()
+        Hpack_h = torch.empty((rows, N), dtype=torch.bfloat16).pin_memory()
+        Xpack_d = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+        Hpack_d = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+        Xv = {M: Xpack_d[offs[M]:offs[M] + M] for M in Ms}
+        Hv = {M: Hpack_d[offs[M]:offs[M] + M] for M in Ms}
+        h2d = Xpack_h.numel() * 2
+        d2h = Hpack_h.numel() * 2
         cnt = {"c": 0}
 
         def e2e_step():
+            Xpack_d.copy_(Xpack_h, non_blocking=True)
             for M in Ms:
                 c = cnt["c"] % copies
-                Xd[M].copy_(Xp[M], non_blocking=True)
-                up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream,
+                up.swiglu_fwd(Xv[M], Wg_all[c], Wu_all[c], Hv[M], stream=stream,
                               weights_stable=True)
-                Hp[M].copy_(Hd[M], non_blocking=True)
                 cnt["c"] += 1
+            Hpack_h.copy_(Hpack_d, non_blocking=True)
         e_steps = min(args.steps, 2000)
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
@@ -372,6 +383,8 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
             barrier(world)
             e_ms = timed_events(e2e_step, e_steps, stream)
         barrier(world)
+        if not torch.equal(Hpack_h[offs[max(Ms)]:], out["H"][max(Ms)]):
+            raise RuntimeError("e2e: H read back differs from the device-timed run")
         e_ms = max_over_ranks(e_ms, world)
         out["e2e"] = {"ms": e_ms, "steps": e_steps, "h2d": h2d, "d2h": d2h}
     del full, partial

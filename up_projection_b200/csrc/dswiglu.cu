@@ -26,7 +26,7 @@ using namespace dev;
 
 constexpr int kThreads = 256;
 constexpr int kBlocksPerSm = 8;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 4;  // measured at n = 8192 * 14336: 6.15 TB/s vs 5.7 with 2
 
 // dU = dh * act(alpha g),  dG = dh * u * alpha * act'(alpha g).  `which` is
 // a compile-time constant at every call (the kernel is instantiated per
