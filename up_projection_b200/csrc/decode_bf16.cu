@@ -72,7 +72,7 @@ struct Geometry {
     bool ok;
 };
 
-__host__ __device__ inline Geometry geometry(int K, int budget) {
+inline Geometry geometry(int K, int budget) {
     Geometry g{};
     g.inner = 8;
     for (int c = 256; c >= 8; c >>= 1)
@@ -116,7 +116,7 @@ __host__ __device__ inline Geometry geometry(int K, int budget) {
 
 // Shared-memory budget of a launch: the small footprint only when it keeps
 // three or more stages of at least 512 k.
-__host__ __device__ inline int decode_budget(int K, bool weights_stable) {
+inline int decode_budget(int K, bool weights_stable) {
     if (weights_stable) {
         const Geometry g = geometry(K, kPdlSmemBudget);
         if (g.ok && g.stages >= 3 && g.kc >= 512) return kPdlSmemBudget;
@@ -147,11 +147,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                               const __grid_constant__ CUtensorMap tm_wu,
                               const __nv_bfloat16 *__restrict__ X,
                               __nv_bfloat16 *__restrict__ H, int M, int K, int N,
-                              int weights_stable, int budget, int which_act, float alpha,
+                              int weights_stable, int which_act, float alpha,
                               __nv_bfloat16 *__restrict__ Gout,
-                              __nv_bfloat16 *__restrict__ Uout) {
+                              __nv_bfloat16 *__restrict__ Uout, const Geometry geo) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const Geometry geo = geometry(K, budget);
+    // The tensor maps are needed first and their fetch is the longest
+    // dependency of the prologue: start it before anything else.  (The
+    // geometry comes precomputed from the host for the same reason.)
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tm_wg);
+        tma_prefetch_desc(&tm_wu);
+    }
     // Under programmatic dependent launch the next call may be scheduled as
     // soon as every CTA of this one is running: it only prefetches weights
     // until this grid has completed (griddepcontrol.wait below).
@@ -188,8 +194,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(bar_red_empty, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_wg);
-        tma_prefetch_desc(&tm_wu);
     }
     __syncthreads();
 
@@ -413,7 +417,7 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
     __nv_bfloat16 *gp = static_cast<__nv_bfloat16 *>(epi.G);
     __nv_bfloat16 *up = static_cast<__nv_bfloat16 *>(epi.U);
     cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_decode_bf16_kernel, tg, tu, xp, hp, M, K, N,
-                                       ws, budget, which_act, alpha, gp, up);
+                                       ws, which_act, alpha, gp, up, geo);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
