@@ -114,7 +114,8 @@ enum swiglu_route {
     SWIGLU_ROUTE_DECODE_BF16 = 2, /* bf16, M <= 8: weight-streaming kernel  */
     SWIGLU_ROUTE_GEMM_BF16 = 3,   /* bf16, M > 8: tcgen05 dual GEMM         */
     SWIGLU_ROUTE_GEMM_TF32X3 = 4, /* fp32: 3xTF32 tcgen05 dual GEMM         */
-    SWIGLU_ROUTE_BWD_GEMM_BF16 = 5 /* bf16 backward GEMM (swiglu_bwd_dx/_dw) */
+    SWIGLU_ROUTE_BWD_GEMM_BF16 = 5, /* bf16 backward GEMM (swiglu_bwd_dx/_dw) */
+    SWIGLU_ROUTE_BWD_GEMM_TF32X3 = 6 /* fp32 backward GEMM, 3xTF32          */
 };
 
 /*
@@ -223,14 +224,16 @@ SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U
  * fused MLP's forward/backward dataflow, page "[RFC] Testing Methodology for
  * FP32 Convergence Tests on Fused SwiGLU/dSwiGLU Kernels", Background).
  *
- *  dG, dU  [M, N] device bf16 (the outputs of dswiglu_bwd), 16-byte aligned.
- *  Wg, Wu  [N, K] device bf16, the forward's weights, 16-byte aligned.
- *  dX      [M, K] device bf16 output, 16-byte aligned; written, never read.
- *  M, K, N >= 0; K and N multiples of 8.  dtype must be SWIGLU_BF16 (any
- *  other value: SWIGLU_ERR_BAD_DTYPE).
+ *  dG, dU  [M, N] device, dtype elements (the outputs of dswiglu_bwd),
+ *          16-byte aligned.
+ *  Wg, Wu  [N, K] device, dtype elements, the forward's weights, aligned.
+ *  dX      [M, K] device, dtype elements, 16-byte aligned; written only.
+ *  M, K, N >= 0; K and N multiples of 8 (bf16) / 4 (fp32).
+ *  dtype   SWIGLU_BF16 or SWIGLU_FP32 (else SWIGLU_ERR_BAD_DTYPE).
  *
- *  Both products accumulate in ONE fp32 accumulator (tcgen05, TMEM); dX is
- *  rounded once to bf16 (RNE).  M == 0 or K == 0: nothing enqueued.  N == 0:
+ *  Both products accumulate in ONE fp32 accumulator (tcgen05, TMEM); bf16:
+ *  dX is rounded once to bf16 (RNE); fp32: 3xTF32 products accumulated in
+ *  256-deep chunks folded with round-to-nearest adds, as swiglu_fwd's fp32.  M == 0 or K == 0: nothing enqueued.  N == 0:
  *  dX is set to +0.  dX must not overlap an input (SWIGLU_ERR_OVERLAP).
  *  Allocates no device memory.
  */
@@ -243,13 +246,15 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
  *   dWg = dG^T X,  dWu = dU^T X,  dWg[n,k] = sum_m dG[m,n] X[m,k]
  * (same passage as swiglu_bwd_dx).
  *
- *  dG, dU    [M, N] device bf16, 16-byte aligned.
- *  X         [M, K] device bf16, the forward's input, 16-byte aligned.
- *  dWg, dWu  [N, K] device bf16 outputs, 16-byte aligned; written, never
+ *  dG, dU    [M, N] device, dtype elements, 16-byte aligned.
+ *  X         [M, K] device, dtype elements, the forward's input, aligned.
+ *  dWg, dWu  [N, K] device, dtype elements, 16-byte aligned; written, never
  *            read (not accumulated into).
- *  M, K, N >= 0; K and N multiples of 8.  dtype must be SWIGLU_BF16.
+ *  M, K, N >= 0; K and N multiples of 8 (bf16) / 4 (fp32).  dtype
+ *  SWIGLU_BF16 or SWIGLU_FP32.
  *
- *  fp32 accumulation over all M rows in TMEM, one RNE rounding per output.
+ *  fp32 accumulation over all M rows in TMEM (fp32: 3xTF32, chunked as in
+ *  swiglu_bwd_dx), one rounding per output.
  *  N == 0 or K == 0: nothing enqueued.  M == 0: dWg and dWu are set to +0.
  *  Outputs must not overlap each other or an input (SWIGLU_ERR_OVERLAP).
  *  Allocates no device memory.

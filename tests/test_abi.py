@@ -126,8 +126,9 @@ def test_status_strings():
     ((16, 32, 48, 64, None, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
     ((None, 32, 48, 64, 80, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
     ((16, 32, 48, 64, 88, 4, 64, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_PTR),
-    ((16, 32, 48, 64, 80, 4, 64, 64, 1), _capi.SWIGLU_ERR_BAD_DTYPE),   # bf16 only
+    ((16, 32, 48, 64, 80, 4, 64, 64, 2), _capi.SWIGLU_ERR_BAD_DTYPE),
     ((16, 32, 48, 64, 80, 4, 60, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, 80, 4, 66, 64, 1), _capi.SWIGLU_ERR_MISALIGNED_DIM),   # fp32: K % 4
     ((16, 32, 48, 64, 80, 4, 64, 68, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
     ((16, 32, 48, 64, 80, -1, 64, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
     ((16, 32, 48, 64, 80, 1 << 31, 64, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
@@ -146,8 +147,9 @@ def test_bwd_dx_host_validation(args, code):
     ((16, 32, 48, None, 80, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
     ((16, None, 48, 1 << 20, 1 << 21, 4, 64, 64, 0), _capi.SWIGLU_ERR_NULL_POINTER),
     ((16, 32, 48, 1 << 20, (1 << 21) + 4, 4, 64, 64, 0), _capi.SWIGLU_ERR_MISALIGNED_PTR),
-    ((16, 32, 48, 64, 80, 4, 64, 64, 1), _capi.SWIGLU_ERR_BAD_DTYPE),
+    ((16, 32, 48, 64, 80, 4, 64, 64, 2), _capi.SWIGLU_ERR_BAD_DTYPE),
     ((16, 32, 48, 64, 80, 4, 64, 12, 0), _capi.SWIGLU_ERR_MISALIGNED_DIM),
+    ((16, 32, 48, 64, 80, 4, 64, 10, 1), _capi.SWIGLU_ERR_MISALIGNED_DIM),   # fp32: N % 4
     ((16, 32, 48, 64, 80, 4, -8, 64, 0), _capi.SWIGLU_ERR_BAD_DIM),
     # dWu [64,64] bf16 = 8 KiB starts inside dWg
     ((1 << 22, 1 << 23, 1 << 24, 1 << 20, (1 << 20) + 4096, 4, 64, 64, 0), _capi.SWIGLU_ERR_OVERLAP),

@@ -162,8 +162,8 @@ def test_bwd_python_binding_shapes():
     assert dWg.shape == (N, K) and dWu.shape == (N, K)
     assert_bf16_close(f64(dX).reshape(M, K), oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu)),
                       "dX via binding")
-    with pytest.raises(TypeError):
-        _capi.swiglu_bwd_dx(dGd.float(), dUd.float(), Wgd.float(), Wud.float())
+    with pytest.raises(TypeError):   # mixed dtypes
+        _capi.swiglu_bwd_dx(dGd, dUd, Wgd.float(), Wud.float())
     # N == 0 through the binding: dX = 0 (empty reduction), dW empty
     e = torch.empty((5, 0), dtype=torch.bfloat16, device=dev())
     w = torch.empty((0, 64), dtype=torch.bfloat16, device=dev())
@@ -198,3 +198,74 @@ def test_training_step_full_size_sampled():
     rdg, rdu = oracle.dswiglu_f64(f64(dH[rows]), f64(G.cpu()[rows]), f64(U.cpu()[rows]))
     assert_bf16_close(f64(dGc[rows]), rdg, "dG rows")
     assert_bf16_close(f64(dUc[rows]), rdu, "dU rows")
+
+
+# ---- fp32 (3xTF32) -----------------------------------------------------------
+
+def _run_f32(fn, *args):
+    out = fn(*(a.to(dev()) for a in args))
+    assert _capi.swiglu_sync_status() == 0
+    assert _capi.swiglu_last_route() == _capi.ROUTE_BWD_GEMM_TF32X3
+    return out
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 4, 4), (130, 260, 196), (300, 516, 136), (257, 1028, 68),
+                                   (200, 2048, 1032)])
+def test_bwd_fp32_within_mixed_bound(M, K, N):
+    """fp32 backward GEMMs within 1e-5 of the size of the terms summed
+    (sum |dG||Wg| + |dU||Wu|, resp. sum |dG||X|): the fp32 forward's bound,
+    read the same way for the backward."""
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=M + 1)
+    dG = synth.normal((M, N), N + 20, 1.0, "f32")
+    dU = synth.normal((M, N), N + 21, 1.0, "f32")
+    g, u, x, wg, wu = (f64(t) for t in (dG, dU, X, Wg, Wu))
+    dX = _run_f32(_capi.swiglu_bwd_dx, dG, dU, Wg, Wu)
+    ref = oracle.bwd_dx_f64(g, u, wg, wu)
+    mag = np.abs(g) @ np.abs(wg) + np.abs(u) @ np.abs(wu)
+    err = np.abs(f64(dX) - ref)
+    assert np.all(err <= 1e-5 * (mag + np.abs(ref)) + 1e-30), float((err / (mag + 1e-30)).max())
+    dWg, dWu = _run_f32(_capi.swiglu_bwd_dw, dG, dU, X)
+    rg, ru = oracle.bwd_dw_f64(g, u, x)
+    for got, r, mg in ((dWg, rg, np.abs(g).T @ np.abs(x)), (dWu, ru, np.abs(u).T @ np.abs(x))):
+        e = np.abs(f64(got) - r)
+        assert np.all(e <= 1e-5 * (mg + np.abs(r)) + 1e-30), float((e / (mg + 1e-30)).max())
+    # near-IEEE: norm-wise error well below plain TF32's (~1e-4 at these sizes)
+    assert np.linalg.norm(f64(dX) - ref) <= 1e-5 * np.linalg.norm(ref)
+
+
+def test_bwd_fp32_integer_exact():
+    """Small integers are exact in TF32's hi part (lo = 0) and every sum is
+    exact in fp32: bit-exact against the oracle."""
+    M, K, N = 300, 264, 200
+    X = synth.ternary((M, K), 1, 0.5, "f32")
+    Wg = synth.ternary((N, K), 2, 0.05, "f32")
+    Wu = synth.ternary((N, K), 3, 0.05, "f32")
+    dG = synth.ternary((M, N), 4, 0.05, "f32")
+    dU = synth.ternary((M, N), 5, 0.05, "f32")
+    np.testing.assert_array_equal(f64(_run_f32(_capi.swiglu_bwd_dx, dG, dU, Wg, Wu)),
+                                  oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu)))
+    dWg, dWu = _run_f32(_capi.swiglu_bwd_dw, dG, dU, X)
+    rg, ru = oracle.bwd_dw_f64(f64(dG), f64(dU), f64(X))
+    np.testing.assert_array_equal(f64(dWg), rg)
+    np.testing.assert_array_equal(f64(dWu), ru)
+
+
+def test_bwd_fp32_full_size_sampled():
+    """LLaMA-2 13B fp32 shape at M = 2048 (the fp32 forward's workload):
+    sampled rows of dX and of dWg, dWu against the oracle, mixed bound."""
+    M, K, N = 2048, 5120, 13824
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=77)
+    dG = synth.normal((M, N), 78, 1.0, "f32")
+    dU = synth.normal((M, N), 79, 1.0, "f32")
+    dX = _run_f32(_capi.swiglu_bwd_dx, dG, dU, Wg, Wu).cpu()
+    dWg, dWu = _run_f32(_capi.swiglu_bwd_dw, dG, dU, X)
+    dWg, dWu = dWg.cpu(), dWu.cpu()
+    rows = np.array([0, 1, 1000, 2047])
+    cols = np.array([0, 5000, 13823])
+    g, u, wg, wu, x = f64(dG), f64(dU), f64(Wg), f64(Wu), f64(X)
+    ref = oracle.bwd_dx_f64(g[rows], u[rows], wg, wu)
+    mag = np.abs(g[rows]) @ np.abs(wg) + np.abs(u[rows]) @ np.abs(wu)
+    assert np.all(np.abs(f64(dX)[rows] - ref) <= 1e-5 * mag + 1e-30)
+    rg, ru = oracle.bwd_dw_f64(g[:, cols], u[:, cols], x)
+    assert np.all(np.abs(f64(dWg)[cols] - rg) <= 1e-5 * (np.abs(g[:, cols]).T @ np.abs(x)) + 1e-30)
+    assert np.all(np.abs(f64(dWu)[cols] - ru) <= 1e-5 * (np.abs(u[:, cols]).T @ np.abs(x)) + 1e-30)

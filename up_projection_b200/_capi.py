@@ -44,6 +44,7 @@ ROUTE_DECODE_BF16 = 2
 ROUTE_GEMM_BF16 = 3
 ROUTE_GEMM_TF32X3 = 4
 ROUTE_BWD_GEMM_BF16 = 5
+ROUTE_BWD_GEMM_TF32X3 = 6
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -240,8 +241,8 @@ def swiglu_fwd_fp8(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor, stream=N
 def _bwd_shapes(dG, dU, name_w, W):
     for t, n in ((dG, "dG"), (dU, "dU"), (W, name_w)):
         _dev(t, n)
-    if not (dG.dtype == dU.dtype == W.dtype == torch.bfloat16):
-        raise TypeError("the backward GEMMs take bfloat16 tensors")
+    if not (dG.dtype == dU.dtype == W.dtype) or dG.dtype not in _DT:
+        raise TypeError("the backward GEMMs take bfloat16 or float32 tensors of one dtype")
     if dG.shape != dU.shape:
         raise ValueError("dG and dU must have the same shape")
     N = dG.shape[-1]
@@ -253,13 +254,13 @@ def _bwd_shapes(dG, dU, name_w, W):
 
 def swiglu_bwd_dx(dG: torch.Tensor, dU: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
                   dX: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """dX = dG Wg + dU Wu through the C ABI (bf16).  dG, dU [..., N] (leading
+    """dX = dG Wg + dU Wu through the C ABI (bf16, or fp32 by 3xTF32).  dG, dU [..., N] (leading
     dims flattened to M rows), Wg, Wu [N, K]; dX has dG's leading dims."""
     M, N = _bwd_shapes(dG, dU, "Wg", Wg)
     _dev(Wu, "Wu")
     K = Wg.shape[-1]
     if Wg.shape != (N, K) or Wu.shape != (N, K) or Wu.dtype != Wg.dtype:
-        raise ValueError(f"weights must be bf16 [N, K] = [{N}, {K}]")
+        raise ValueError(f"weights must be [N, K] = [{N}, {K}] of dG's dtype")
     if dX is None:
         dX = torch.empty((*dG.shape[:-1], K), dtype=dG.dtype, device=dG.device)
     else:
@@ -267,7 +268,7 @@ def swiglu_bwd_dx(dG: torch.Tensor, dU: torch.Tensor, Wg: torch.Tensor, Wu: torc
         if dX.dtype != dG.dtype or dX.numel() != M * K:
             raise ValueError("dX has the wrong dtype or size")
     st = lib().swiglu_bwd_dx(dG.data_ptr(), dU.data_ptr(), Wg.data_ptr(), Wu.data_ptr(),
-                             dX.data_ptr(), M, K, N, SWIGLU_BF16, _stream(stream))
+                             dX.data_ptr(), M, K, N, _dtype_code(dG), _stream(stream))
     _check("swiglu_bwd_dx", st)
     return dX
 
@@ -275,7 +276,7 @@ def swiglu_bwd_dx(dG: torch.Tensor, dU: torch.Tensor, Wg: torch.Tensor, Wu: torc
 def swiglu_bwd_dw(dG: torch.Tensor, dU: torch.Tensor, X: torch.Tensor,
                   dWg: torch.Tensor | None = None, dWu: torch.Tensor | None = None,
                   stream=None):
-    """(dWg, dWu) = (dG^T X, dU^T X) through the C ABI (bf16).  dG, dU
+    """(dWg, dWu) = (dG^T X, dU^T X) through the C ABI (bf16, or fp32 by 3xTF32).  dG, dU
     [..., N] and X [..., K] with the same leading dims (M rows)."""
     M, N = _bwd_shapes(dG, dU, "X", X)
     K = X.shape[-1]
@@ -288,7 +289,7 @@ def swiglu_bwd_dw(dG: torch.Tensor, dU: torch.Tensor, X: torch.Tensor,
         if t.dtype != X.dtype or t.numel() != N * K:
             raise ValueError(f"{n} has the wrong dtype or size")
     st = lib().swiglu_bwd_dw(dG.data_ptr(), dU.data_ptr(), X.data_ptr(), dWg.data_ptr(),
-                             dWu.data_ptr(), M, K, N, SWIGLU_BF16, _stream(stream))
+                             dWu.data_ptr(), M, K, N, _dtype_code(dG), _stream(stream))
     _check("swiglu_bwd_dw", st)
     return dWg, dWu
 

@@ -150,12 +150,13 @@ int check_bwd(const void *dH, const void *G, const void *U, const void *dG, cons
     return SWIGLU_OK;
 }
 
-// Shape rules shared by the backward GEMMs (bf16 only).
+// Shape rules shared by the backward GEMMs.
 int check_bwd_shape(int64_t M, int64_t K, int64_t N, int dtype) {
-    if (dtype != SWIGLU_BF16) return SWIGLU_ERR_BAD_DTYPE;
+    if (dtype != SWIGLU_BF16 && dtype != SWIGLU_FP32) return SWIGLU_ERR_BAD_DTYPE;
     if (M < 0 || K < 0 || N < 0) return SWIGLU_ERR_BAD_DIM;
     if (M > kMaxDim || K > kMaxDim || N > kMaxDim) return SWIGLU_ERR_BAD_DIM;
-    if (K % 8 != 0 || N % 8 != 0) return SWIGLU_ERR_MISALIGNED_DIM;
+    const int align = dtype == SWIGLU_BF16 ? 8 : 4;  // elements per 16 bytes
+    if (K % align != 0 || N % align != 0) return SWIGLU_ERR_MISALIGNED_DIM;
     return SWIGLU_OK;
 }
 
@@ -170,11 +171,12 @@ int check_bwd_dx(const void *dG, const void *dU, const void *Wg, const void *Wu,
     if (!aligned16(dX)) return SWIGLU_ERR_MISALIGNED_PTR;
     *route = SWIGLU_ROUTE_ZERO_K;
     if (N == 0) return SWIGLU_OK;
-    *route = SWIGLU_ROUTE_BWD_GEMM_BF16;
+    *route = dtype == SWIGLU_BF16 ? SWIGLU_ROUTE_BWD_GEMM_BF16 : SWIGLU_ROUTE_BWD_GEMM_TF32X3;
     if (!dG || !dU || !Wg || !Wu) return SWIGLU_ERR_NULL_POINTER;
     if (!aligned16(dG) || !aligned16(dU) || !aligned16(Wg) || !aligned16(Wu))
         return SWIGLU_ERR_MISALIGNED_PTR;
-    const int64_t xb = M * K * 2, gb = M * N * 2, wb = N * K * 2;
+    const int es = elem_size(dtype);
+    const int64_t xb = M * K * es, gb = M * N * es, wb = N * K * es;
     if (overlaps(dX, xb, dG, gb) || overlaps(dX, xb, dU, gb) || overlaps(dX, xb, Wg, wb) ||
         overlaps(dX, xb, Wu, wb))
         return SWIGLU_ERR_OVERLAP;
@@ -190,14 +192,15 @@ int check_bwd_dw(const void *dG, const void *dU, const void *X, const void *dWg,
     if (N == 0 || K == 0) return SWIGLU_OK;
     if (!dWg || !dWu) return SWIGLU_ERR_NULL_POINTER;
     if (!aligned16(dWg) || !aligned16(dWu)) return SWIGLU_ERR_MISALIGNED_PTR;
-    const int64_t wb = N * K * 2;
+    const int es = elem_size(dtype);
+    const int64_t wb = N * K * es;
     if (overlaps(dWg, wb, dWu, wb)) return SWIGLU_ERR_OVERLAP;
     *route = SWIGLU_ROUTE_ZERO_K;
     if (M == 0) return SWIGLU_OK;
-    *route = SWIGLU_ROUTE_BWD_GEMM_BF16;
+    *route = dtype == SWIGLU_BF16 ? SWIGLU_ROUTE_BWD_GEMM_BF16 : SWIGLU_ROUTE_BWD_GEMM_TF32X3;
     if (!dG || !dU || !X) return SWIGLU_ERR_NULL_POINTER;
     if (!aligned16(dG) || !aligned16(dU) || !aligned16(X)) return SWIGLU_ERR_MISALIGNED_PTR;
-    const int64_t gb = M * N * 2, xb = M * K * 2;
+    const int64_t gb = M * N * es, xb = M * K * es;
     const void *outs[2] = {dWg, dWu};
     for (const void *o : outs) {
         if (overlaps(o, wb, dG, gb) || overlaps(o, wb, dU, gb) || overlaps(o, wb, X, xb))
@@ -384,10 +387,13 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg, con
     if (st != SWIGLU_OK) return st;
     cudaError_t e;
     if (route == SWIGLU_ROUTE_ZERO_K)
-        e = cudaMemsetAsync(dX, 0, static_cast<size_t>(M) * K * 2, stream);
-    else
+        e = cudaMemsetAsync(dX, 0, static_cast<size_t>(M) * K * elem_size(dtype), stream);
+    else if (route == SWIGLU_ROUTE_BWD_GEMM_BF16)
         e = launch_bwd_dx_bf16(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
                                static_cast<int>(N), dev, stream);
+    else
+        e = launch_bwd_dx_tf32x3(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
+                                 static_cast<int>(N), dev, stream);
     st = from_cuda(e);
     if (st == SWIGLU_OK) t_last_route = route;
     return st;
@@ -408,12 +414,15 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X, void
     if (st != SWIGLU_OK) return st;
     cudaError_t e;
     if (route == SWIGLU_ROUTE_ZERO_K) {
-        const size_t bytes = static_cast<size_t>(N) * K * 2;
+        const size_t bytes = static_cast<size_t>(N) * K * elem_size(dtype);
         e = cudaMemsetAsync(dWg, 0, bytes, stream);
         if (e == cudaSuccess) e = cudaMemsetAsync(dWu, 0, bytes, stream);
-    } else {
+    } else if (route == SWIGLU_ROUTE_BWD_GEMM_BF16) {
         e = launch_bwd_dw_bf16(dG, dU, X, dWg, dWu, static_cast<int>(M), static_cast<int>(K),
                                static_cast<int>(N), dev, stream);
+    } else {
+        e = launch_bwd_dw_tf32x3(dG, dU, X, dWg, dWu, static_cast<int>(M), static_cast<int>(K),
+                                 static_cast<int>(N), dev, stream);
     }
     st = from_cuda(e);
     if (st == SWIGLU_OK) t_last_route = route;
@@ -447,7 +456,7 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
@@ -456,7 +465,9 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_bwd_status_fetch_and_clear(&w4, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2 | w3 | w4) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = gemm_bwd_tf32x3_status_fetch_and_clear(&w5, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3 | w4 | w5) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
 }
 
 SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes, void *sink,

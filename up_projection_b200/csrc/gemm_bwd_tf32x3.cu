@@ -1,0 +1,434 @@
+// gemm_bwd_tf32x3.cu -- the backward GEMMs of the projection for fp32
+// tensors, near-IEEE on the tensor cores by 3xTF32 splitting, sm_100a:
+//
+//   dX  [M,K] = dG Wg + dU Wu                  (reduction over N)
+//   dWg [N,K] = dG^T X,   dWu [N,K] = dU^T X    (reduction over M)
+//
+// An fp32 training step needs these at fp32 accuracy as much as the forward
+// (Liger-Kernel issue #1383, "[RFC] Testing Methodology for FP32 Convergence
+// Tests on Fused SwiGLU/dSwiGLU Kernels": the fused MLP's forward and
+// backward are checked together against fp32; plain TF32 fails).
+//
+// The operand layouts and the tile raster are those of the bf16 backward
+// kernel (gemm_bwd_bf16.cu): dX accumulates both products in one accumulator
+// over the 2N-long reduction [dG | dU] x [Wg ; Wu]; dW treats [dWg ; dWu] as
+// one [2N x K] output.  The 3xTF32 machinery is that of the fp32 forward
+// (tf32x3.cuh): the split warps rewrite each raw stage as hi in place and
+// write lo beside it; per 8-deep step three kind::tf32 MMAs (lo*hi, hi*lo,
+// hi*hi) accumulate into a chunk accumulator; the epilogue warps fold every
+// 256-deep chunk into a running sum with round-to-nearest fp32 adds, then
+// store the fp32 tile by TMA.
+//
+// fp32 operands: K-major tiles are 16 fp32 (64 bytes) per row in the 64-byte
+// swizzle; MN-major tiles are atoms of 32 fp32 (128 bytes) by 16 reduction
+// rows in the 128-byte swizzle with 32-byte atoms (the layout tf32 MN-major
+// operands take), one TMA box {32, 16} per atom.  Output tile
+// 128 x 256, MMA M=128 N=256 K=8.  Every wait is bounded.
+#include <atomic>
+
+#include "gemm_common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tf32x3.cuh"
+#include "tmap.cuh"
+
+namespace swiglu {
+
+// Bit 0: a bounded wait gave up.  Read by gemm_bwd_tf32x3_status_fetch_and_clear().
+__device__ unsigned int g_gemm_bwd_tf32x3_status;
+
+namespace {
+
+using namespace dev;
+using gemm::mbar_wait_drain;
+using gemm::tile_coords;
+
+enum : int { kModeDx = 0, kModeDw = 1 };
+
+constexpr int kBM = 128;                 // output rows per tile (= MMA M)
+constexpr int kBN = 256;                 // output columns per tile (= MMA N)
+constexpr int kBR = 16;                  // reduction depth per stage
+constexpr int kStages = 4;
+constexpr int kUmmaK = 8;                // k per tcgen05.mma, kind::tf32
+constexpr int kAccCols = kBN;
+constexpr int kTmemCols = 2 * kAccCols;  // chunk accumulator + running sum
+constexpr int kChunkKB = 16;             // stages per accumulation chunk (256 deep)
+constexpr int kSplitWarps = 4;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * (kSplitWarps + kEpiWarps);  // 320
+constexpr int kFirstSplitWarp = 2;
+constexpr int kFirstEpiWarp = kFirstSplitWarp + kSplitWarps;    // 6
+
+constexpr uint32_t kAtomBytes = 32 * kBR * 4;          // MN-major atom: 32 x 16 fp32 = 2 KB
+constexpr uint32_t kABytes = kBM * kBR * 4;            // 8 KB
+constexpr uint32_t kBBytes = kBN * kBR * 4;            // 16 KB
+constexpr uint32_t kRawBytes = kABytes + kBBytes;      // 24 KB loaded per stage
+constexpr uint32_t kStageBytes = 2 * kRawBytes;        // + lo copies
+constexpr uint32_t kEpiBufBytes = 32 * 128;            // 32 rows x 32 fp32
+
+constexpr uint32_t kOffStages = 0;
+constexpr uint32_t kOffEpi = kOffStages + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
+constexpr uint32_t kNumBars = 3 * kStages + 3;  // full, ready, empty, chunk full/empty, drain
+constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
+constexpr uint32_t kSmemBytes = kOffAbort + 8 + 1024;
+
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
+
+// Problem geometry (as in the bf16 backward kernel).
+struct Geo {
+    int rows;        // output rows of one output matrix
+    int cols;        // output columns (K)
+    int row_tiles;   // row tiles of one output matrix
+    int num_m;       // row tiles in the raster
+    int num_n;       // column tiles
+    int kb_pair;     // 16-deep reduction blocks of one pair
+};
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    swiglu_gemm_bwd_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                                  const __grid_constant__ CUtensorMap tm_a1,
+                                  const __grid_constant__ CUtensorMap tm_b0,
+                                  const __grid_constant__ CUtensorMap tm_b1,
+                                  const __grid_constant__ CUtensorMap tm_o0,
+                                  const __grid_constant__ CUtensorMap tm_o1, Geo geo) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+
+    const uint32_t sst = base + kOffStages;
+    const uint32_t se = base + kOffEpi;
+    const uint32_t bar_full = base + kOffBar;
+    const uint32_t bar_ready = bar_full + 8 * kStages;
+    const uint32_t bar_empty = bar_ready + 8 * kStages;
+    const uint32_t bar_cfull = bar_empty + 8 * kStages;
+    const uint32_t bar_cempty = bar_cfull + 8;
+    const uint32_t bar_drain = bar_cempty + 8;
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + kOffTmemPtr);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int num_tiles = geo.num_m * geo.num_n;
+    const int num_kb = kMode == kModeDx ? 2 * geo.kb_pair : geo.kb_pair;
+    const int num_chunks = (num_kb + kChunkKB - 1) / kChunkKB;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_ready + 8 * s, kSplitWarps);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_cfull, 1);
+        mbar_init(bar_cempty, kEpiWarps);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_a0);
+        tma_prefetch_desc(&tm_a1);
+        tma_prefetch_desc(&tm_b0);
+        tma_prefetch_desc(&tm_b1);
+        tma_prefetch_desc(&tm_o0);
+        tma_prefetch_desc(&tm_o1);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
+
+    bool failed = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, geo.num_m, geo.num_n, mt, nt);
+                const int c0 = nt * kBN;
+                const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
+                const int r0 = (mt - second * geo.row_tiles) * kBM;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t st = sst + stage * kStageBytes;
+                    mbar_arrive_expect_tx(fb, kRawBytes);
+                    if (kMode == kModeDx) {
+                        const int pair = kb >= geo.kb_pair ? 1 : 0;
+                        const int red0 = (kb - pair * geo.kb_pair) * kBR;
+                        // A: [128 rows of dG or dU] x [16 of N], K-major.
+                        tma_load_2d(pair ? &tm_a1 : &tm_a0, fb, st, red0, r0);
+                        // B: [16 rows of Wg or Wu] x [256 of K], MN-major atoms.
+#pragma unroll
+                        for (int j = 0; j < kBN / 32; ++j)
+                            tma_load_2d(pair ? &tm_b1 : &tm_b0, fb, st + kABytes + j * kAtomBytes,
+                                        c0 + 32 * j, red0);
+                    } else {
+                        const int red0 = kb * kBR;
+                        // A: [16 rows of M] x [128 of N] of dG or dU, MN-major.
+#pragma unroll
+                        for (int j = 0; j < kBM / 32; ++j)
+                            tma_load_2d(second ? &tm_a1 : &tm_a0, fb, st + j * kAtomBytes,
+                                        r0 + 32 * j, red0);
+                        // B: [16 rows of M] x [256 of K] of X, MN-major.
+#pragma unroll
+                        for (int j = 0; j < kBN / 32; ++j)
+                            tma_load_2d(&tm_b0, fb, st + kABytes + j * kAtomBytes, c0 + 32 * j,
+                                        red0);
+                    }
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < kStages; ++s) {
+                if (issued > s) {
+                    const long long uses = (issued - 1 - s) / kStages + 1;
+                    mbar_wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------- MMA issuer
+            constexpr uint32_t idesc = make_idesc(2u, kBM, kBN) | kIdescBMnMajor |
+                                       (kMode == kModeDw ? kIdescAMnMajor : 0u);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t chunk_phase = 0;
+            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+                for (int q = 0; q < num_chunks && !failed; ++q) {
+                    if (!mbar_wait(bar_cempty, chunk_phase ^ 1u, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kb_end = min(num_kb, (q + 1) * kChunkKB);
+                    for (int kb = q * kChunkKB; kb < kb_end; ++kb) {
+                        if (!mbar_wait(bar_ready + 8 * stage, phase, abort_flag)) {
+                            failed = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t st = sst + stage * kStageBytes;
+                        const uint64_t a_hi = kMode == kModeDx ? sw64_kmajor_desc(st)
+                                                               : sw128b32_mnmajor_desc(st, kAtomBytes);
+                        const uint64_t a_lo = kMode == kModeDx
+                                                  ? sw64_kmajor_desc(st + kRawBytes)
+                                                  : sw128b32_mnmajor_desc(st + kRawBytes, kAtomBytes);
+                        const uint64_t b_hi = sw128b32_mnmajor_desc(st + kABytes, kAtomBytes);
+                        const uint64_t b_lo = sw128b32_mnmajor_desc(st + kRawBytes + kABytes, kAtomBytes);
+#pragma unroll
+                        for (int kk = 0; kk < kBR / kUmmaK; ++kk) {
+                            // K-major: +32 B along the 64-byte swizzled row (+2);
+                            // MN-major: +8 rows of 128 B (+64).
+                            const uint32_t oa = kMode == kModeDx ? 2u * kk : 64u * kk;
+                            const uint32_t ob = 64u * kk;
+                            const uint32_t acc = (kb == q * kChunkKB && kk == 0) ? 0u : 1u;
+                            mma_tf32(tmem_base, a_lo + oa, b_hi + ob, idesc, acc);
+                            mma_tf32(tmem_base, a_hi + oa, b_lo + ob, idesc, 1u);
+                            mma_tf32(tmem_base, a_hi + oa, b_hi + ob, idesc, 1u);
+                        }
+                        mma_commit(bar_empty + 8 * stage);
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (failed) break;
+                    mma_commit(bar_cfull);
+                    chunk_phase ^= 1u;
+                }
+            }
+            mma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0);
+        }
+    } else if (warp < kFirstEpiWarp) {
+        // ---------------------------------------------------- hi/lo split
+        const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                tf32x3::split_stage<kRawBytes, 32 * kSplitWarps>(sst + stage * kStageBytes, sidx);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_ready + 8 * stage);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------ accumulation + epilogue
+        const int quad = warp & 3;
+        const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t chunk_acc = tmem_base + row_off;
+        const uint32_t run_acc = tmem_base + row_off + kAccCols;
+        const uint32_t buf = se + static_cast<uint32_t>(warp - kFirstEpiWarp) * kEpiBufBytes;
+        const uint32_t swz = static_cast<uint32_t>(lane & 7);
+        uint32_t chunk_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            int mt, nt;
+            tile_coords(t, geo.num_m, geo.num_n, mt, nt);
+            const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
+            const int r0 = (mt - second * geo.row_tiles) * kBM;
+            const int c0 = nt * kBN;
+            for (int q = 0; q < num_chunks; ++q) {
+                if (!mbar_wait(bar_cfull, chunk_phase, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                chunk_phase ^= 1u;
+                tc_fence_after();
+                tf32x3::fold_chunk<kAccCols>(chunk_acc, run_acc, q);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_cempty);
+            }
+            if (failed) break;
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(run_acc + 32u * c, v);
+                tmem_ld_wait(v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    sts_v4(buf + static_cast<uint32_t>(lane) * 128u +
+                               ((static_cast<uint32_t>(j) ^ swz) << 4),
+                           make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = c0 + c * 32;
+                    const int y = r0 + quad * 32;
+                    if (x < geo.cols && y < geo.rows) {
+                        tma_store_2d(second ? &tm_o1 : &tm_o0, buf, x, y);
+                        bulk_commit();
+                    }
+                }
+            }
+        }
+        if (lane == 0) bulk_wait<0>();
+    }
+
+    if (failed) atomicOr(&g_gemm_bwd_tf32x3_status, 1u);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        __syncwarp();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+std::atomic<unsigned> g_attr_set_mask[2];
+
+template <int kMode>
+cudaError_t launch_tiles(const CUtensorMap (&tm)[6], const Geo &geo, const DeviceInfo &dev,
+                         cudaStream_t stream) {
+    auto kernel = swiglu_gemm_bwd_tf32x3_kernel<kMode>;
+    const unsigned bit = 1u << (dev.device & 31);
+    if (!(g_attr_set_mask[kMode].load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        g_attr_set_mask[kMode].fetch_or(bit);
+    }
+    const long long tiles = static_cast<long long>(geo.num_m) * geo.num_n;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], geo);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                 void *dX, int M, int K, int N, const DeviceInfo &dev,
+                                 cudaStream_t stream) {
+    Geo geo{};
+    geo.rows = M;
+    geo.cols = K;
+    geo.row_tiles = (M + kBM - 1) / kBM;
+    geo.num_m = geo.row_tiles;
+    geo.num_n = (K + kBN - 1) / kBN;
+    geo.kb_pair = (N + kBR - 1) / kBR;
+    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle mn = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+    const uint64_t n_bytes = static_cast<uint64_t>(N) * 4, k_bytes = static_cast<uint64_t>(K) * 4;
+    CUtensorMap tm[6];
+    if (!encode_tmap_2d(&tm[0], dG, f32, N, M, n_bytes, kBR, kBM, sw64) ||
+        !encode_tmap_2d(&tm[1], dU, f32, N, M, n_bytes, kBR, kBM, sw64) ||
+        !encode_tmap_2d(&tm[2], Wg, f32, K, N, k_bytes, 32, kBR, mn) ||
+        !encode_tmap_2d(&tm[3], Wu, f32, K, N, k_bytes, 32, kBR, mn) ||
+        !encode_tmap_2d(&tm[4], dX, f32, K, M, k_bytes, 32, 32, sw128)) {
+        return cudaErrorInvalidValue;
+    }
+    tm[5] = tm[4];
+    return launch_tiles<kModeDx>(tm, geo, dev, stream);
+}
+
+cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
+                                 void *dWu, int M, int K, int N, const DeviceInfo &dev,
+                                 cudaStream_t stream) {
+    Geo geo{};
+    geo.rows = N;
+    geo.cols = K;
+    geo.row_tiles = (N + kBM - 1) / kBM;
+    geo.num_m = 2 * geo.row_tiles;
+    geo.num_n = (K + kBN - 1) / kBN;
+    geo.kb_pair = (M + kBR - 1) / kBR;
+    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle mn = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+    const uint64_t n_bytes = static_cast<uint64_t>(N) * 4, k_bytes = static_cast<uint64_t>(K) * 4;
+    CUtensorMap tm[6];
+    if (!encode_tmap_2d(&tm[0], dG, f32, N, M, n_bytes, 32, kBR, mn) ||
+        !encode_tmap_2d(&tm[1], dU, f32, N, M, n_bytes, 32, kBR, mn) ||
+        !encode_tmap_2d(&tm[2], X, f32, K, M, k_bytes, 32, kBR, mn) ||
+        !encode_tmap_2d(&tm[4], dWg, f32, K, N, k_bytes, 32, 32, sw128) ||
+        !encode_tmap_2d(&tm[5], dWu, f32, K, N, k_bytes, 32, 32, sw128)) {
+        return cudaErrorInvalidValue;
+    }
+    tm[3] = tm[2];
+    return launch_tiles<kModeDw>(tm, geo, dev, stream);
+}
+
+cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host_out, g_gemm_bwd_tf32x3_status,
+                                              sizeof(unsigned int), 0, cudaMemcpyDeviceToHost,
+                                              stream);
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_gemm_bwd_tf32x3_status, &zero, sizeof(unsigned int), 0,
+                                cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
+}
+
+}  // namespace swiglu

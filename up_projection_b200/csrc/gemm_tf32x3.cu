@@ -41,6 +41,7 @@
 #include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "tf32x3.cuh"
 #include "tmap.cuh"
 
 namespace swiglu {
@@ -85,24 +86,6 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
 
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
 static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
-
-__device__ __forceinline__ uint32_t tf32_rna(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-// Split 4 fp32 values in place: returns hi in `v`, lo in `lo`.
-__device__ __forceinline__ void split4(uint4 &v, uint4 &lo) {
-    uint32_t *pv = &v.x, *pl = &lo.x;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float a = __uint_as_float(pv[i]);
-        const uint32_t hi = tf32_rna(a);
-        pl[i] = tf32_rna(a - __uint_as_float(hi));
-        pv[i] = hi;
-    }
-}
 
 // h = act(alpha g) * u in fp32 with expf / tanhf and IEEE division (a few
 // ulp in total).
@@ -261,10 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kFirstEpiWarp) {
         // ---------------------------------------------------- hi/lo split
         const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
-        constexpr int kThreadsSplit = 32 * kSplitWarps;
-        constexpr int kVecs = kRawBytes / 16;                  // 1536 per stage
-        constexpr int kPerThread = kVecs / kThreadsSplit;      // 12
-        static_assert(kVecs % kThreadsSplit == 0, "split work must divide evenly");
         int stage = 0;
         uint32_t phase = 0;
         for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
@@ -273,21 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     failed = true;
                     break;
                 }
-                const uint32_t st = sst + stage * kStageBytes;
-                // all loads first, then the splits and stores, so the shared-
-                // memory latency is paid once per stage
-                uint4 x[kPerThread];
-#pragma unroll
-                for (int i = 0; i < kPerThread; ++i)
-                    x[i] = lds_v4(st + 16u * (sidx + i * kThreadsSplit));
-#pragma unroll
-                for (int i = 0; i < kPerThread; ++i) {
-                    uint4 lo;
-                    split4(x[i], lo);
-                    const uint32_t off = 16u * (sidx + i * kThreadsSplit);
-                    sts_v4(st + off, x[i]);
-                    sts_v4(st + kRawBytes + off, lo);
-                }
+                tf32x3::split_stage<kRawBytes, 32 * kSplitWarps>(sst + stage * kStageBytes, sidx);
                 // make the generic-proxy writes visible to the tensor cores
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -321,22 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 chunk_phase ^= 1u;
                 tc_fence_after();
-#pragma unroll 1
-                for (int col = 0; col < kAccCols; col += 32) {
-                    uint32_t c[32], r[32];
-                    tmem_ld_32x32b_x32(chunk_acc + col, c);
-                    if (q > 0) tmem_ld_32x32b_x32(run_acc + col, r);
-                    tmem_ld_wait(c);
-                    if (q > 0) {
-                        tmem_ld_wait(r);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            c[i] = __float_as_uint(__fadd_rn(__uint_as_float(r[i]),
-                                                             __uint_as_float(c[i])));
-                    }
-                    tmem_st_32x32b_x32(run_acc + col, c);
-                }
-                tmem_st_wait();
+                tf32x3::fold_chunk<kAccCols>(chunk_acc, run_acc, q);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_cempty);

@@ -64,6 +64,13 @@ cudaError_t launch_bwd_dx_bf16(const void *dG, const void *dU, const void *Wg, c
 cudaError_t launch_bwd_dw_bf16(const void *dG, const void *dU, const void *X, void *dWg,
                                void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                cudaStream_t stream);
+// fp32 backward GEMMs (3xTF32), same operations, K and N multiples of 4.
+cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                 void *dX, int M, int K, int N, const DeviceInfo &dev,
+                                 cudaStream_t stream);
+cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
+                                 void *dWu, int M, int K, int N, const DeviceInfo &dev,
+                                 cudaStream_t stream);
 // Output tile width (128, 192 or 256 columns) the backward GEMMs use for a raster
 // of `row_tiles_total` 128-row tiles by `cols` columns.
 int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
@@ -79,6 +86,7 @@ cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_
 cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool tensor_maps_available();

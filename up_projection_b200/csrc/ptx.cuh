@@ -233,6 +233,21 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint3
     return d;
 }
 
+// MN-major 32-bit (tf32) operands take the 128-byte swizzle with 32-byte
+// atoms instead (layout type 1; TMA CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B):
+// 128-byte rows of 32 elements, 32-byte chunks permuted over groups of 4
+// rows, so the stride byte offset is 4 rows = 512 B; consecutive 32-wide MN
+// atoms `atom_bytes` apart.  8 reduction rows further on = +1024 B = +64.
+__device__ __forceinline__ uint64_t sw128b32_mnmajor_desc(uint32_t smem_addr, uint32_t atom_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((atom_bytes >> 4) & 0x3FFFu) << 16;  // LBO: next MN atom
+    d |= static_cast<uint64_t>(512u >> 4) << 32;                    // SBO: next 4 rows
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(1u) << 61;                           // 128B, 32-byte atoms
+    return d;
+}
+
 // Instruction-descriptor bits that mark A (bit 15) or B (bit 16) as MN-major.
 constexpr uint32_t kIdescAMnMajor = 1u << 15;
 constexpr uint32_t kIdescBMnMajor = 1u << 16;
