@@ -534,6 +534,26 @@ def run_extras(stream, pk):
                                  "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32 MMA)",
                                  "frac": round(3 * tf / tf32_peak, 4),
                                  "frac_vs_bf16_peak_literal": round(tf / pk["bf16_tflops"], 4)}})
+        if K == 5120:
+            # the fp32 backward GEMMs at the same shape (3xTF32)
+            dGf = torch.randn((M, N), generator=gen, device=dev)
+            dUf = torch.randn((M, N), generator=gen, device=dev)
+            dXf = torch.empty((M, K), device=dev)
+            dWgf = torch.empty((N, K), device=dev)
+            dWuf = torch.empty((N, K), device=dev)
+            for what, fn in (("dX = dG Wg + dU Wu",
+                              lambda: up.swiglu_bwd_dx(dGf, dUf, Wg, Wu, dXf, stream=stream)),
+                             ("dWg = dG^T X, dWu = dU^T X",
+                              lambda: up.swiglu_bwd_dw(dGf, dUf, X, dWgf, dWuf, stream=stream))):
+                ms = time_op(fn, iters=5)
+                tf = fl / (ms * 1e-3) / 1e12
+                add({"workload": f"fp32 3xTF32 backward {what}, {name} M=2048",
+                     "metric": "TFLOP/s (fp32-equivalent)", "value": round(tf, 1),
+                     "ms": round(ms, 4),
+                     "roofline": {"bound": "tensor", "achieved": round(3 * tf, 1),
+                                  "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32 MMA)",
+                                  "frac": round(3 * tf / tf32_peak, 4)}})
+            del dGf, dUf, dXf, dWgf, dWuf
         del X, Wg, Wu, H
     torch.cuda.empty_cache()
     return res
