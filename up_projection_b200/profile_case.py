@@ -33,6 +33,7 @@ def main(argv=None):
     ap.add_argument("--n", type=int, default=8192 * 14336)
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--fp32", action="store_true", help="bwd_dx / bwd_dw: fp32 (3xTF32) operands")
     ap.add_argument("--weights-stable", action="store_true",
                     help="decode: SWIGLU_FLAG_WEIGHTS_STABLE (programmatic dependent launch)")
     a = ap.parse_args(argv)
@@ -72,7 +73,7 @@ def main(argv=None):
         for _ in range(L):
             up.swiglu_fwd_fp8(X, Wg, Wu)
     elif a.case in ("bwd_dx", "bwd_dw"):
-        bf = torch.bfloat16
+        bf = torch.float32 if a.fp32 else torch.bfloat16
         dG = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
         dU = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
         if a.case == "bwd_dx":
