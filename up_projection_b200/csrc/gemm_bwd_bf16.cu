@@ -93,7 +93,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
 struct Geo {
     int rows;        // output rows of one output matrix
     int cols;        // output columns (K)
-    int red;         // reduction length of one pair
     int row_tiles;   // row tiles of one output matrix
     int num_m;       // row tiles in the raster
     int num_n;       // column tiles
@@ -397,7 +396,6 @@ cudaError_t launch_bwd_dx_bf16(const void *dG, const void *dU, const void *Wg, c
     Geo geo{};
     geo.rows = M;
     geo.cols = K;
-    geo.red = N;
     geo.row_tiles = (M + kBM - 1) / kBM;
     geo.num_m = geo.row_tiles;
     geo.kb_pair = (N + kBR - 1) / kBR;
@@ -428,7 +426,6 @@ cudaError_t launch_bwd_dw_bf16(const void *dG, const void *dU, const void *X, vo
     Geo geo{};
     geo.rows = N;
     geo.cols = K;
-    geo.red = M;
     geo.row_tiles = (N + kBM - 1) / kBM;
     geo.num_m = 2 * geo.row_tiles;
     geo.kb_pair = (M + kBR - 1) / kBR;
