@@ -323,27 +323,45 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
                       "p99_us": round(float(q[2]), 2)}
     out["latency"] = lat
 
-    # Unfused comparator for context: torch F.linear twice + silu * mul
-    # (library GEMMs, G and U through HBM), same rotated copies, one graph.
+    # Comparators for context at the largest M, timed A-B-C-C-B-A, each a
+    # graph of one rotation of the copies: A = this library's fused call,
+    # B = torch F.linear twice + silu * mul (library GEMMs, G and U through
+    # HBM), C = torch F.linear on the stacked [2N, K] weights + silu * mul of
+    # the two halves.
     M = max(Ms)
     F = torch.nn.functional
+    Wcat_all = torch.cat([Wg_all, Wu_all], dim=1)   # [copies, 2N, K]
 
-    def unfused(c):
+    def arm_a(c):
+        up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream, weights_stable=True)
+
+    def arm_b(c):
         return F.silu(F.linear(Xd[M], Wg_all[c])) * F.linear(Xd[M], Wu_all[c])
+
+    def arm_c(c):
+        gu = F.linear(Xd[M], Wcat_all[c])
+        return F.silu(gu[:, :N]) * gu[:, N:]
+    graphs = {}
     with torch.cuda.stream(stream):
-        for c in range(copies):
-            unfused(c)
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
+        for name, fn in (("A", arm_a), ("B", arm_b), ("C", arm_c)):
             for c in range(copies):
-                unfused(c)
+                fn(c)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for c in range(copies):
+                    fn(c)
+            graphs[name] = gr
         reps = min(200, max(1, 2 * args.steps // copies))
-        for _ in range(2):
-            gr.replay()
-        t = timed_events(gr.replay, reps, stream) / (reps * copies)
-        del gr
-    out["torch_unfused"] = {"M": M, "us": t * 1e3,
-                            "GB/s": decode_bytes(M, K, N) / (t * 1e-3) / 1e9}
+        samples = {"A": [], "B": [], "C": []}
+        for name in "ABCCBA":
+            for _ in range(2):
+                graphs[name].replay()
+            samples[name].append(timed_events(graphs[name].replay, reps, stream) / (reps * copies))
+    del graphs, Wcat_all
+    cmp_us = {k: 1e3 * sum(v) / len(v) for k, v in samples.items()}
+    out["comparators"] = {"M": M, "order": "A-B-C-C-B-A", "us": cmp_us,
+                          "GB/s": {k: decode_bytes(M, K, N) / (v * 1e-6) / 1e9
+                                   for k, v in cmp_us.items()}}
 
     out["H"] = {M: Hd[M].cpu() for M in Ms}
 
@@ -583,6 +601,17 @@ def cpu_baseline_decode(K, N, Ms, budget_s=12.0, gpu_H=None):
     dt = time.perf_counter() - t0
     step_bytes = sum(decode_bytes(M, K, N) for M in Ms)
     threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    # the same oracle on one thread, on a smaller bounded sample (M = 8 only)
+    o.set_num_threads(1)
+    t1 = time.perf_counter()
+    n1 = 0
+    while time.perf_counter() - t1 < budget_s / 3:
+        o.swiglu_fwd_f64(Xd[:max(Ms)], Wgd, Wud)
+        n1 += 1
+    dt1 = time.perf_counter() - t1
+    o.set_num_threads(0)
+    single = {"value": round(decode_bytes(max(Ms), K, N) * n1 / dt1 / 1e9, 4), "unit": "GB/s",
+              "cores": 1, "sample": f"{n1} decode calls at M={max(Ms)}, {dt1:.1f} s"}
     parity = None
     if gpu_H is not None:
         g = np.concatenate([gpu_H[M].to(torch.float64).numpy().ravel() for M in Ms])
@@ -594,6 +623,7 @@ def cpu_baseline_decode(K, N, Ms, budget_s=12.0, gpu_H=None):
                   "within_bf16_tol": float(np.mean(err <= 1e-2 * np.abs(r) + 1e-3))}
     return {"value": round(step_bytes * steps / dt / 1e9, 4), "unit": "GB/s",
             "cores": min(threads, max(Ms)), "kind": "oracle", "parity_vs_gpu": parity,
+            "single_thread": single,
             "sample": f"{steps} full decode steps (M=1,2,4,8 at K={K}, N={N}), fp64 C loops, "
                       f"OpenMP over output rows ({threads} threads available), {dt:.1f} s"}
 
@@ -710,10 +740,13 @@ def main(argv=None):
                        "what": "pure streaming read of the same Wg+Wu copies (swiglu_read_floor)",
                        "decode_frac_of_floor": round(achieved / dec["floor"]["GB/s"], 4)},
         "latency_single_call": {str(M): v for M, v in dec["latency"].items()},
-        "torch_unfused": {"what": "F.silu(F.linear(X, Wg)) * F.linear(X, Wu), same rotated copies",
-                          "M": dec["torch_unfused"]["M"],
-                          "us": round(dec["torch_unfused"]["us"], 2),
-                          "GB/s": round(dec["torch_unfused"]["GB/s"], 1)},
+        "comparators": {
+            "what": {"A": "this library (fused decode call)",
+                     "B": "torch F.silu(F.linear(X, Wg)) * F.linear(X, Wu)",
+                     "C": "torch F.linear(X, [Wg; Wu]) then silu(g) * u"},
+            "M": dec["comparators"]["M"], "order": dec["comparators"]["order"],
+            "us": {k: round(v, 2) for k, v in dec["comparators"]["us"].items()},
+            "GB/s": {k: round(v, 1) for k, v in dec["comparators"]["GB/s"].items()}},
     }
     if rank == 0 and not args.no_extra:
         line["also"] = run_extras(stream, pk)
@@ -733,7 +766,8 @@ def main(argv=None):
                              "read_floor_GB/s": round(d7["floor"]["GB/s"], 1),
                              "frac_of_floor": round(v7 / d7["floor"]["GB/s"], 4),
                              "latency_single_call": {str(M): v for M, v in d7["latency"].items()},
-                             "torch_unfused_us": round(d7["torch_unfused"]["us"], 2)})
+                             "comparators_us": {k: round(v, 2) for k, v in
+                                                d7["comparators"]["us"].items()}})
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline_decode(K, N, DECODE_MS, gpu_H=dec["H"])
     if rank == 0:

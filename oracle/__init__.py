@@ -101,6 +101,8 @@ class Oracle:
                                                      ctypes.c_int, _D, _P, _P, _P, _P, _P]
         lib.oracle_dswiglu_act_f64.restype = None
         lib.oracle_dswiglu_act_f64.argtypes = [_P, _P, _P, _I64, ctypes.c_int, _D, _P, _P]
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_e4m3_decode.restype = ctypes.c_double
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_int]
         lib.oracle_e4m3_encode.restype = ctypes.c_int
@@ -244,6 +246,10 @@ class Oracle:
             raise MemoryError("oracle: row buffer allocation failed")
         return out
 
+    def set_num_threads(self, n: int) -> None:
+        """OpenMP threads of the row loops (timing only; results unchanged)."""
+        self.lib.oracle_set_num_threads(int(n))
+
     # ---- quantised output ------------------------------------------------------
     def e4m3_decode(self, code: int) -> float:
         return self.lib.oracle_e4m3_decode(int(code))
@@ -338,6 +344,7 @@ def __getattr__(name):
                 "decode_bf16", "decode",
                 "swiglu_fwd_f64", "swiglu_fwd", "swiglu_fwd_points",
                 "dswiglu_f64", "dswiglu", "bwd_dx_f64", "bwd_dw_f64",
-                "e4m3_decode", "e4m3_encode", "ue8m0_exponent", "quant_e4m3"}:
+                "e4m3_decode", "e4m3_encode", "ue8m0_exponent", "quant_e4m3",
+                "set_num_threads"}:
         return getattr(default(), name)
     raise AttributeError(name)

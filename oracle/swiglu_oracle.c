@@ -513,3 +513,14 @@ ORACLE_API void oracle_quant_e4m3(const double *H, int64_t M, int64_t N, uint8_t
     for (int64_t m = 0; m < M; ++m)
         oracle_quant_e4m3_row(H + m * N, N, q + m * N, s + m * nb);
 }
+
+/* ---- timing support ------------------------------------------------------ */
+
+/* Number of OpenMP threads the oracle's row loops use (n <= 0: the
+ * runtime default).  The results do not depend on it: every output is
+ * summed by one thread in ascending index order. */
+#include <omp.h>
+ORACLE_API void oracle_set_num_threads(int n)
+{
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+}
