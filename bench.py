@@ -460,6 +460,13 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
+    # context: the unfused library chain (two cuBLAS GEMMs, G and U through
+    # HBM, then silu * mul)
+    F = torch.nn.functional
+    with torch.no_grad():
+        ms_t = time_op(lambda: F.silu(F.linear(X, Wg)) * F.linear(X, Wu), iters=5)
+    res[-1]["torch_unfused_ms"] = round(ms_t, 4)
+    res[-1]["speedup_vs_torch_unfused"] = round(ms_t / ms, 3)
     # training forward: the same call also storing G and U for the backward
     Gs = torch.empty_like(H)
     Us = torch.empty_like(H)
@@ -515,7 +522,26 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
-    del X, Wg, Wu, H, Gs, Us, dGb, dUb, dX, dWg, dWu
+    # one whole training step of the projection: forward storing G and U,
+    # dSwiGLU, dX, dWg/dWu (dH stands in for the gradient from above)
+    dHb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)
+    epi_gu = up_capi.Epilogue(0, 1.0, Gs.data_ptr(), Us.data_ptr())
+
+    def train_step():
+        up.lib().swiglu_fwd_epilogue(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
+                                     M, K, N, 0, ctypes.byref(epi_gu), 0, stream.cuda_stream)
+        up.dswiglu_bwd(dHb, Gs, Us, dGb, dUb, stream=stream)
+        up.swiglu_bwd_dx(dGb, dUb, Wg, Wu, dX, stream=stream)
+        up.swiglu_bwd_dw(dGb, dUb, X, dWg, dWu, stream=stream)
+    ms = time_op(train_step, iters=5)
+    tf = 3 * fl / (ms * 1e-3) / 1e12
+    add({"workload": "training step (forward storing G, U; dSwiGLU; dX; dWg, dWu), "
+                     "LLaMA-3 8B M=8192 bf16",
+         "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+         "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4),
+                      "note": "3 x 4MNK GEMM FLOPs; the dSwiGLU pass (1.17 GB) is counted as time only"}})
+    del X, Wg, Wu, H, Gs, Us, dGb, dUb, dX, dWg, dWu, dHb
     # dSwiGLU on [8192, 14336] bf16
     n = 8192 * 14336
     dH = torch.randn(n, generator=gen, device=dev).to(torch.bfloat16)
