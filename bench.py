@@ -638,6 +638,16 @@ def cpu_baseline_decode(K, N, Ms, budget_s=12.0, gpu_H=None):
     o.set_num_threads(0)
     single = {"value": round(decode_bytes(max(Ms), K, N) * n1 / dt1 / 1e9, 4), "unit": "GB/s",
               "cores": 1, "sample": f"{n1} decode calls at M={max(Ms)}, {dt1:.1f} s"}
+    # informative, not a gate: the shift of the "eager" trajectory that rounds
+    # G and U to bf16 before silu * mul, against the fused reference (which
+    # keeps them unrounded), on the M = 8 call
+    r8 = o.swiglu_fwd_f64(Xd[:max(Ms)], Wgd, Wud)
+    g8 = torch.from_numpy(r8["G"]).to(torch.bfloat16).to(torch.float64).numpy()
+    u8 = torch.from_numpy(r8["U"]).to(torch.bfloat16).to(torch.float64).numpy()
+    eager = g8 / (1.0 + np.exp(-g8)) * u8
+    shift = np.abs(eager - r8["H"])
+    eager_shift = {"max_abs": float(shift.max()),
+                   "rel_norm": float(np.linalg.norm(shift) / np.linalg.norm(r8["H"]))}
     parity = None
     if gpu_H is not None:
         g = np.concatenate([gpu_H[M].to(torch.float64).numpy().ravel() for M in Ms])
@@ -649,7 +659,7 @@ def cpu_baseline_decode(K, N, Ms, budget_s=12.0, gpu_H=None):
                   "within_bf16_tol": float(np.mean(err <= 1e-2 * np.abs(r) + 1e-3))}
     return {"value": round(step_bytes * steps / dt / 1e9, 4), "unit": "GB/s",
             "cores": min(threads, max(Ms)), "kind": "oracle", "parity_vs_gpu": parity,
-            "single_thread": single,
+            "single_thread": single, "eager_trajectory_shift": eager_shift,
             "sample": f"{steps} full decode steps (M=1,2,4,8 at K={K}, N={N}), fp64 C loops, "
                       f"OpenMP over output rows ({threads} threads available), {dt:.1f} s"}
 
