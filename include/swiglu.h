@@ -285,6 +285,17 @@ SWIGLU_API const char *swiglu_status_string(int status);
 SWIGLU_API int swiglu_sync_status(cudaStream_t stream);
 
 /*
+ * Failure-path self-test (the pages have no counterpart; it exercises this
+ * library's own failure detection).  Enqueues a one-CTA kernel whose bounded
+ * mbarrier wait nothing ever completes: after about a millisecond the wait
+ * gives up, the kernel records it in its device status word and returns
+ * normally (no trap, no fault, no hang).  The next swiglu_sync_status on the
+ * stream then returns SWIGLU_ERR_TIMEOUT (and clears the word); the context
+ * stays usable.  Returns SWIGLU_OK once enqueued.
+ */
+SWIGLU_API int swiglu_selftest_wait_timeout(cudaStream_t stream);
+
+/*
  * Bench-only probe: stream-read `bytes` bytes from each of A and B (device,
  * 16-byte aligned, bytes a multiple of 16) with the same 128-bit loads the
  * decode kernel uses, and write one 32-bit word per CTA to `sink`

@@ -60,3 +60,20 @@ def test_rank3_input_is_flattened():
     H3 = _capi.swiglu_fwd(Xd.view(2, 3, 64), Wgd, Wud)
     assert H3.shape == (2, 3, 32)
     assert torch.equal(H3.reshape(6, 32), flat)
+
+
+def test_bounded_wait_timeout_is_reported_and_recoverable():
+    """The failure path without a fault: a wait that nothing completes gives
+    up after ~1 ms, the host reads SWIGLU_ERR_TIMEOUT once, and the context
+    keeps working."""
+    import torch
+    from up_projection_b200 import _capi
+    s = torch.cuda.current_stream().cuda_stream
+    assert _capi.swiglu_sync_status() == 0
+    assert _capi.lib().swiglu_selftest_wait_timeout(s) == 0
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_ERR_TIMEOUT
+    assert _capi.swiglu_sync_status() == 0          # the word was cleared
+    X = torch.randn(130, 64, device="cuda").to(torch.bfloat16)
+    W = (torch.randn(64, 64, device="cuda") / 8).to(torch.bfloat16)
+    H = _capi.swiglu_fwd(X, W, W)
+    assert _capi.swiglu_sync_status() == 0 and bool(torch.isfinite(H.float()).all())

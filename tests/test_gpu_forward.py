@@ -190,3 +190,28 @@ def test_decode_weights_stable_chain_reads_x_after_producer():
         got = outs[i].cpu()
         assert_bf16_close(f64(got), ref, f"chain step {i}")
         prev = got
+
+
+def _random_shapes(seed, count, ms):
+    r = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for i in range(count):
+        M = int(ms[i % len(ms)])
+        K = int(r.integers(1, 80)) * 8
+        N = int(r.integers(1, 80)) * 8
+        out.append((M, K, N))
+    return out
+
+
+@pytest.mark.parametrize("M,K,N", _random_shapes(2024, 16, [9, 10, 12, 63, 127, 129, 255, 257]))
+def test_gemm_random_odd_shapes(M, K, N):
+    """Seeded random shapes around tile boundaries: ragged M (127, 129, 257...),
+    K and N any multiple of 8 up to 632, every output against the oracle."""
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 7 + K * 3 + N)
+    check_full(X, Wg, Wu, _capi.ROUTE_GEMM_BF16, f"gemm M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M,K,N", _random_shapes(2025, 10, [1, 2, 3, 5, 7, 8]))
+def test_decode_random_odd_shapes(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 11 + K * 5 + N)
+    check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"decode M={M} K={K} N={N}")

@@ -74,6 +74,7 @@ SIGNATURES = {
     "swiglu_status_string": (ctypes.c_char_p, [_I]),
     "swiglu_sync_status": (_I, [_P]),
     "swiglu_read_floor": (_I, [_P, _P, _I64, _P, _P]),
+    "swiglu_selftest_wait_timeout": (_I, [_P]),
     "swiglu_read_floor_sink_words": (_I64, []),
 }
 

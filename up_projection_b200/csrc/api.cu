@@ -456,7 +456,7 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0, w6 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
@@ -467,7 +467,17 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_bwd_tf32x3_status_fetch_and_clear(&w5, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2 | w3 | w4 | w5) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = selftest_status_fetch_and_clear(&w6, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3 | w4 | w5 | w6) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+}
+
+SWIGLU_API int swiglu_selftest_wait_timeout(cudaStream_t stream) {
+    DeviceInfo dev;
+    int st = current_device(dev);
+    if (st != SWIGLU_OK) return st;
+    // about one millisecond at the B200 boost clock
+    return from_cuda(launch_selftest_wait(2000000LL, stream));
 }
 
 SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes, void *sink,

@@ -87,6 +87,11 @@ cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStrea
 cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t selftest_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+
+// Failure-path self-test: one CTA whose bounded mbarrier wait (limit in SM
+// clock cycles) never completes and gives up.
+cudaError_t launch_selftest_wait(long long limit_cycles, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool tensor_maps_available();
