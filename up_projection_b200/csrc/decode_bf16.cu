@@ -72,7 +72,10 @@ struct Geometry {
     bool ok;
 };
 
-inline Geometry geometry(int K, int budget) {
+// `xrows` rows of X are staged: 8 (rows >= M zero-filled in shared memory),
+// or M in the compact layout (rows M..7 of the MMA's B operand are zeros in
+// registers), which leaves more shared memory for weight stages.
+inline Geometry geometry(int K, int budget, int xrows) {
     Geometry g{};
     g.inner = 8;
     for (int c = 256; c >= 8; c >>= 1)
@@ -92,7 +95,7 @@ inline Geometry geometry(int K, int budget) {
             const int kc = (per + g.inner - 1) / g.inner * g.inner;
             if (kc / g.inner > 256) continue;
             const int stage = 32 * kc;  // 16 rows x kc bf16
-            const int xbytes = 16 * s * kc;
+            const int xbytes = 2 * xrows * s * kc;
             int st = (budget - xbytes) / stage;
             if (st > kMaxStages) st = kMaxStages;
             if (xbytes < budget && st >= min_stages) {
@@ -107,7 +110,7 @@ inline Geometry geometry(int K, int budget) {
     if (!g.ok) return g;
     g.kx = g.slices * g.kc;
     g.off_x = g.stages * 32 * g.kc;
-    g.off_red = g.off_x + 16 * g.kx;
+    g.off_red = g.off_x + 2 * xrows * g.kx;
     g.off_bar = g.off_red + kRedBytes;
     g.smem = g.off_bar + 8 * kNumBars + 16 + 1024;  // + alignment slack
     if (g.smem > kMaxSmem) g.ok = false;
@@ -116,9 +119,9 @@ inline Geometry geometry(int K, int budget) {
 
 // Shared-memory budget of a launch: the small footprint only when it keeps
 // three or more stages of at least 512 k.
-inline int decode_budget(int K, bool weights_stable) {
+inline int decode_budget(int K, bool weights_stable, int xrows) {
     if (weights_stable) {
-        const Geometry g = geometry(K, kPdlSmemBudget);
+        const Geometry g = geometry(K, kPdlSmemBudget, xrows);
         if (g.ok && g.stages >= 3 && g.kc >= 512) return kPdlSmemBudget;
     }
     return kSmemBudget;
@@ -142,6 +145,7 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], uint32_t a0, ui
 }
 
 
+template <bool kCompactX>
 __global__ void __launch_bounds__(kThreads, 2)
     swiglu_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_wg,
                               const __grid_constant__ CUtensorMap tm_wu,
@@ -223,7 +227,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             long long issued = 0;
             for (int u = u_begin; u < u_end && !failed; ++u) {
                 for (int j = 0; j < geo.slices; ++j) {
-                    if (!x_issued && issued >= geo.stages) issue_x();
+                    // compact layout (deeper ring): X right after the first
+                    // three stages, the rest of the ring fills behind it
+                    const int x_after = (kCompactX && geo.stages > 3) ? 3 : geo.stages;
+                    if (!x_issued && issued >= x_after) issue_x();
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
@@ -257,11 +264,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int ct = threadIdx.x - 32;  // 0..127
         const int grp = lane >> 2;
         const int tig = lane & 3;
-        // Zero the X stage where the copies do not write: rows >= M, and the
-        // columns [K, kx) of rows < M (disjoint from the copies' bytes).
+        // Zero the X stage where the copies do not write: the columns
+        // [K, kx) of rows < M and (8-row layout) the rows >= M.
         {
             const int vec_per_row = static_cast<int>(x_pitch / 16);
-            for (int i = ct; i < 8 * vec_per_row; i += 32 * kConsumerWarps) {
+            const int rows = kCompactX ? M : 8;
+            for (int i = ct; i < rows * vec_per_row; i += 32 * kConsumerWarps) {
                 const int r = i / vec_per_row;
                 const int byte = (i - r * vec_per_row) * 16;
                 if (r >= M || byte >= K * 2) sts_v4(xs + r * x_pitch + byte, make_uint4(0, 0, 0, 0));
@@ -273,7 +281,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         const uint32_t w_pitch = 2u * geo.kc;
         const int chunks = (geo.kc + 31) / 32;
-        const uint32_t x_lane = xs + grp * x_pitch + tig * 16;
+        // compact layout: lanes of X rows >= M (grp >= M) read row 0 and
+        // feed zeros (the load stays unconditional, a select discards it)
+        const bool x_row_live = !kCompactX || grp < M;
+        const uint32_t x_lane = xs + (x_row_live ? grp : 0) * x_pitch + tig * 16;
         int stage = 0;
         uint32_t phase = 0;
         for (int u = u_begin; u < u_end && !failed; ++u) {
@@ -293,7 +304,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     if (c * 32 + tig * 8 < geo.kc) {  // only a kc not divisible by 32 fails
                         wg = lds_v4(g_row + c * 64);
                         wu = lds_v4(u_row + c * 64);
-                        x = lds_v4(x_row + c * 64);
+                        if constexpr (kCompactX) {
+                            const uint4 xv = lds_v4(x_row + c * 64);
+                            x = x_row_live ? xv : x;
+                        } else {
+                            x = lds_v4(x_row + c * 64);
+                        }
                     }
                     // lane (grp, tig) holds physical k 8*tig + {0..3} of the
                     // chunk for the first MMA and 8*tig + {4..7} for the
@@ -359,20 +375,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (failed) atomicOr(&g_decode_status, 1u);
 }
 
-std::atomic<unsigned> g_attr_set_mask{0};
+std::atomic<unsigned> g_attr_set_mask[2];
 
 }  // namespace
 
 bool decode_bf16_supported(int K) {
     if (K < 8 || K % 8 != 0 || K > (1 << 16)) return false;
-    return geometry(K, kSmemBudget).ok;
+    return geometry(K, kSmemBudget, 8).ok;
 }
 
 cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, void *H, int M,
                                int K, int N, const Epilogue &epi, bool weights_stable,
                                const DeviceInfo &dev, cudaStream_t stream) {
-    const int budget = decode_budget(K, weights_stable);
-    const Geometry geo = geometry(K, budget);
+    int budget = decode_budget(K, weights_stable, 8);
+    Geometry geo = geometry(K, budget, 8);
+    // When the 8-row X stage rules out the overlapped two-CTAs-per-SM launch
+    // (large K), staging only the M rows of X may fit it.
+    bool compact = false;
+    if (weights_stable && M < 8 && budget != kPdlSmemBudget &&
+        decode_budget(K, true, M) == kPdlSmemBudget) {
+        compact = true;
+        budget = kPdlSmemBudget;
+        geo = geometry(K, budget, M);
+    }
     if (!geo.ok) return cudaErrorInvalidValue;
     // 3-D view of each weight matrix: [N rows][K / inner blocks][inner]; a box
     // is inner x (kc / inner) x 8 rows.
@@ -385,12 +410,14 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
                         2ull * geo.inner, 2ull * K, geo.inner, kb, 8)) {
         return cudaErrorInvalidValue;
     }
+    auto kernel = compact ? swiglu_decode_bf16_kernel<true> : swiglu_decode_bf16_kernel<false>;
     const unsigned bit = 1u << (dev.device & 31);
-    if (!(g_attr_set_mask.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(swiglu_decode_bf16_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    std::atomic<unsigned> &mask = g_attr_set_mask[compact ? 1 : 0];
+    if (!(mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kMaxSmem);
         if (e != cudaSuccess) return e;
-        g_attr_set_mask.fetch_or(bit);
+        mask.fetch_or(bit);
     }
     // The small footprint fits two CTAs per SM: launch two per SM so each SM
     // keeps twice the bytes in flight (and the next call's CTAs take over SMs
@@ -416,8 +443,8 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
     const float alpha = epi.gate_multiplier;
     __nv_bfloat16 *gp = static_cast<__nv_bfloat16 *>(epi.G);
     __nv_bfloat16 *up = static_cast<__nv_bfloat16 *>(epi.U);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_decode_bf16_kernel, tg, tu, xp, hp, M, K, N,
-                                       ws, which_act, alpha, gp, up, geo);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tg, tu, xp, hp, M, K, N, ws, which_act, alpha,
+                                       gp, up, geo);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
