@@ -263,6 +263,20 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X,
                              void *dWg, void *dWu, int64_t M, int64_t K,
                              int64_t N, int dtype, cudaStream_t stream);
 
+/*
+ * swiglu_bwd_gemms -- swiglu_bwd_dx and swiglu_bwd_dw in one call:
+ * dX = dG Wg + dU Wu, dWg = dG^T X, dWu = dU^T X, with the argument rules of
+ * both (and dX must not overlap dWg or dWu).  For fp32 the three GEMMs run
+ * as ONE persistent launch whose static schedule gives every CTA its share
+ * of the long dX tiles and fills with the short dW tiles, so the launch ends
+ * in one balanced tail (dX alone has few tiles at small M).  Same results as
+ * the two calls, bit for bit (same per-tile arithmetic).
+ */
+SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg,
+                                const void *Wu, const void *X, void *dX,
+                                void *dWg, void *dWu, int64_t M, int64_t K,
+                                int64_t N, int dtype, cudaStream_t stream);
+
 /* Route swiglu_fwd takes for these arguments (pure host function; returns a
  * swiglu_route, or -1 for arguments swiglu_fwd would reject). */
 SWIGLU_API int swiglu_route_for(int64_t M, int64_t K, int64_t N, int dtype);

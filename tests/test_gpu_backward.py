@@ -269,3 +269,58 @@ def test_bwd_fp32_full_size_sampled():
     rg, ru = oracle.bwd_dw_f64(g[:, cols], u[:, cols], x)
     assert np.all(np.abs(f64(dWg)[cols] - rg) <= 1e-5 * (np.abs(g[:, cols]).T @ np.abs(x)) + 1e-30)
     assert np.all(np.abs(f64(dWu)[cols] - ru) <= 1e-5 * (np.abs(u[:, cols]).T @ np.abs(x)) + 1e-30)
+
+
+# ---- all three GEMMs in one call -------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("M,K,N", [(130, 264, 200), (257, 1032, 72), (2048, 520, 264),
+                                   (1, 8, 8)])
+def test_bwd_gemms_equals_separate_calls(dtype, M, K, N):
+    """swiglu_bwd_gemms gives exactly the separate calls' results (for fp32 it
+    is one scheduled launch; every tile's arithmetic is the same) and matches
+    the oracle."""
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, dtype, seed=M + 3)
+    dG = synth.normal((M, N), N + 30, 1.0, dtype)
+    dU = synth.normal((M, N), N + 31, 1.0, dtype)
+    d = to_dev(dG, dU, Wg, Wu, X)
+    dX, dWg, dWu = _capi.swiglu_bwd_gemms(*d)
+    assert _capi.swiglu_sync_status() == 0
+    sx = _capi.swiglu_bwd_dx(d[0], d[1], d[2], d[3])
+    sg, su = _capi.swiglu_bwd_dw(d[0], d[1], d[4])
+    assert _capi.swiglu_sync_status() == 0
+    assert torch.equal(dX, sx) and torch.equal(dWg, sg) and torch.equal(dWu, su)
+    if dtype == "f32":
+        g, u = f64(dG), f64(dU)
+        ref = oracle.bwd_dx_f64(g, u, f64(Wg), f64(Wu))
+        mag = np.abs(g) @ np.abs(f64(Wg)) + np.abs(u) @ np.abs(f64(Wu))
+        assert np.all(np.abs(f64(dX) - ref) <= 1e-5 * (mag + np.abs(ref)) + 1e-30)
+    else:
+        assert_bf16_close(f64(dX), oracle.bwd_dx_f64(f64(dG), f64(dU), f64(Wg), f64(Wu)), "dX")
+        rg, ru = oracle.bwd_dw_f64(f64(dG), f64(dU), f64(X))
+        assert_bf16_close(f64(dWg), rg, "dWg")
+        assert_bf16_close(f64(dWu), ru, "dWu")
+
+
+def test_bwd_gemms_fp32_integer_exact_13b_schedule():
+    """The schedule of the 13B shape at M = 2048 (320 dX tiles, 2.2 waves, and
+    4320 dW tiles) on integer operands: bit-exact against the oracle on
+    sampled rows -- every tile is computed once and stored where it belongs."""
+    M, K, N = 2048, 5120, 13824
+    X = synth.ternary((M, K), 1, 0.5, "f32")
+    Wg = synth.ternary((N, K), 2, 0.02, "f32")
+    Wu = synth.ternary((N, K), 3, 0.02, "f32")
+    dG = synth.ternary((M, N), 4, 0.02, "f32")
+    dU = synth.ternary((M, N), 5, 0.02, "f32")
+    dX, dWg, dWu = _capi.swiglu_bwd_gemms(*to_dev(dG, dU, Wg, Wu, X))
+    assert _capi.swiglu_sync_status() == 0
+    assert _capi.swiglu_last_route() == _capi.ROUTE_BWD_GEMM_TF32X3
+    r = np.random.Generator(np.random.PCG64(8))
+    rows = np.concatenate([r.integers(0, M, 5), [0, 127, 128, M - 1]])
+    cols = np.concatenate([r.integers(0, N, 5), [0, 127, 128, N - 1]])
+    g, u = f64(dG), f64(dU)
+    np.testing.assert_array_equal(f64(dX.cpu())[rows],
+                                  oracle.bwd_dx_f64(g[rows], u[rows], f64(Wg), f64(Wu)))
+    rg, ru = oracle.bwd_dw_f64(g[:, cols], u[:, cols], f64(X))
+    np.testing.assert_array_equal(f64(dWg.cpu())[cols], rg)
+    np.testing.assert_array_equal(f64(dWu.cpu())[cols], ru)

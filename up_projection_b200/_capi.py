@@ -69,6 +69,7 @@ SIGNATURES = {
     "swiglu_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.POINTER(Epilogue), _P]),
     "swiglu_bwd_dx": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_bwd_dw": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
+    "swiglu_bwd_gemms": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),
     "swiglu_last_route": (_I, []),
     "swiglu_status_string": (ctypes.c_char_p, [_I]),
@@ -293,6 +294,28 @@ def swiglu_bwd_dw(dG: torch.Tensor, dU: torch.Tensor, X: torch.Tensor,
                              dWu.data_ptr(), M, K, N, _dtype_code(dG), _stream(stream))
     _check("swiglu_bwd_dw", st)
     return dWg, dWu
+
+
+def swiglu_bwd_gemms(dG: torch.Tensor, dU: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
+                     X: torch.Tensor, stream=None):
+    """(dX, dWg, dWu) of the projection in one call (bf16 or fp32; for fp32
+    one balanced launch runs all three GEMMs)."""
+    M, N = _bwd_shapes(dG, dU, "Wg", Wg)
+    for t, n in ((Wu, "Wu"), (X, "X")):
+        _dev(t, n)
+    K = Wg.shape[-1]
+    if Wg.shape != (N, K) or Wu.shape != (N, K) or X.shape[-1] != K or X.numel() != M * K:
+        raise ValueError("shapes: dG, dU [.., N], Wg, Wu [N, K], X [.., K] with dG's leading dims")
+    if not (Wu.dtype == X.dtype == dG.dtype):
+        raise TypeError("all tensors must share one dtype")
+    dX = torch.empty((*dG.shape[:-1], K), dtype=dG.dtype, device=dG.device)
+    dWg = torch.empty((N, K), dtype=dG.dtype, device=dG.device)
+    dWu = torch.empty((N, K), dtype=dG.dtype, device=dG.device)
+    st = lib().swiglu_bwd_gemms(dG.data_ptr(), dU.data_ptr(), Wg.data_ptr(), Wu.data_ptr(),
+                                X.data_ptr(), dX.data_ptr(), dWg.data_ptr(), dWu.data_ptr(),
+                                M, K, N, _dtype_code(dG), _stream(stream))
+    _check("swiglu_bwd_gemms", st)
+    return dX, dWg, dWu
 
 
 def swiglu_route_for(M: int, K: int, N: int, dtype: int) -> int:

@@ -429,6 +429,36 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X, void
     return st;
 }
 
+SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                const void *X, void *dX, void *dWg, void *dWu, int64_t M, int64_t K,
+                                int64_t N, int dtype, cudaStream_t stream) {
+    int rx = SWIGLU_ROUTE_NONE, rw = SWIGLU_ROUTE_NONE;
+    int st = check_bwd_dx(dG, dU, Wg, Wu, dX, M, K, N, dtype, &rx);
+    if (st != SWIGLU_OK) return st;
+    st = check_bwd_dw(dG, dU, X, dWg, dWu, M, K, N, dtype, &rw);
+    if (st != SWIGLU_OK) return st;
+    if (rx != SWIGLU_ROUTE_NONE && rw != SWIGLU_ROUTE_NONE) {
+        const int es = elem_size(dtype);
+        const int64_t xb = M * K * es, wb = N * K * es;
+        if (overlaps(dX, xb, dWg, wb) || overlaps(dX, xb, dWu, wb)) return SWIGLU_ERR_OVERLAP;
+    }
+    const bool gemm_x = rx == SWIGLU_ROUTE_BWD_GEMM_BF16 || rx == SWIGLU_ROUTE_BWD_GEMM_TF32X3;
+    const bool gemm_w = rw == SWIGLU_ROUTE_BWD_GEMM_BF16 || rw == SWIGLU_ROUTE_BWD_GEMM_TF32X3;
+    if (gemm_x && gemm_w && dtype == SWIGLU_FP32) {
+        DeviceInfo dev;
+        st = current_device(dev);
+        if (st != SWIGLU_OK) return st;
+        st = from_cuda(launch_bwd_all_tf32x3(dG, dU, Wg, Wu, X, dX, dWg, dWu, static_cast<int>(M),
+                                             static_cast<int>(K), static_cast<int>(N), dev, stream));
+        if (st == SWIGLU_OK) t_last_route = SWIGLU_ROUTE_BWD_GEMM_TF32X3;
+        return st;
+    }
+    // otherwise one call each (zero fills of empty reductions included)
+    st = swiglu_bwd_dx(dG, dU, Wg, Wu, dX, M, K, N, dtype, stream);
+    if (st != SWIGLU_OK) return st;
+    return swiglu_bwd_dw(dG, dU, X, dWg, dWu, M, K, N, dtype, stream);
+}
+
 SWIGLU_API int swiglu_last_route(void) { return t_last_route; }
 
 SWIGLU_API const char *swiglu_status_string(int status) {

@@ -19,11 +19,19 @@
 // 256-deep chunk into a running sum with round-to-nearest fp32 adds, then
 // store the fp32 tile by TMA.
 //
+// One launch can run dX, dW or both: a persistent grid walks a static
+// schedule (gemm_common.cuh) that gives each CTA its round-robin share of the
+// long dX tiles first and then fills with the short dW tiles in the order in
+// which CTAs free up, so the whole backward ends in one balanced wave tail
+// instead of dX's alone (at M = 2048 its 320 tiles are 2.2 waves).
+//
 // fp32 operands: K-major tiles are 16 fp32 (64 bytes) per row in the 64-byte
 // swizzle; MN-major tiles are atoms of 32 fp32 (128 bytes) by 16 reduction
 // rows in the 128-byte swizzle with 32-byte atoms (the layout tf32 MN-major
 // operands take), one TMA box {32, 16} per atom.  Output tile
 // 128 x 256, MMA M=128 N=256 K=8.  Every wait is bounded.
+#include <string.h>
+
 #include <atomic>
 
 #include "gemm_common.cuh"
@@ -42,8 +50,6 @@ namespace {
 using namespace dev;
 using gemm::mbar_wait_drain;
 using gemm::tile_coords;
-
-enum : int { kModeDx = 0, kModeDw = 1 };
 
 constexpr int kBM = 128;                 // output rows per tile (= MMA M)
 constexpr int kBN = 256;                 // output columns per tile (= MMA N)
@@ -77,24 +83,51 @@ constexpr uint32_t kSmemBytes = kOffAbort + 8 + 1024;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
 static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
 
-// Problem geometry (as in the bf16 backward kernel).
-struct Geo {
-    int rows;        // output rows of one output matrix
-    int cols;        // output columns (K)
-    int row_tiles;   // row tiles of one output matrix
-    int num_m;       // row tiles in the raster
-    int num_n;       // column tiles
-    int kb_pair;     // 16-deep reduction blocks of one pair
+// Geometry of the two tile kinds and the schedule of one launch.
+struct Plan {
+    int M, N, K;
+    int dx_num_m, dw_row_tiles, dw_num_m, num_n;   // tiles: dx_num_m x num_n, dw_num_m x num_n
+    int dx_kb, dw_kb;                              // 16-deep reduction blocks per tile
+    int kb_pair;                                   // dX: blocks of one pair (dG Wg, dU Wu)
+    gemm::BwdSched sched;
 };
 
-template <int kMode>
+// Tensor maps of both kinds (only those of the kinds a launch runs are used).
+struct Maps {
+    CUtensorMap dx_a[2];   // dG, dU: K-major {16, 128}
+    CUtensorMap dx_b[2];   // Wg, Wu: MN-major atoms {32, 16}
+    CUtensorMap dx_o;      // dX
+    CUtensorMap dw_a[2];   // dG, dU: MN-major atoms {32, 16}
+    CUtensorMap dw_b;      // X: MN-major atoms {32, 16}
+    CUtensorMap dw_o[2];   // dWg, dWu
+};
+
+struct TileInfo {
+    int kind, r0, c0, num_kb, second;
+};
+
+__device__ __forceinline__ bool next_tile(const Plan &p, int seq, TileInfo &ti) {
+    int kind, t;
+    if (!gemm::bwd_tile_of(p.sched, blockIdx.x, gridDim.x, seq, kind, t)) return false;
+    int mt, nt;
+    ti.kind = kind;
+    if (kind == gemm::kTileDx) {
+        tile_coords(t, p.dx_num_m, p.num_n, mt, nt);
+        ti.second = 0;
+        ti.r0 = mt * kBM;
+        ti.num_kb = p.dx_kb;
+    } else {
+        tile_coords(t, p.dw_num_m, p.num_n, mt, nt);
+        ti.second = mt >= p.dw_row_tiles ? 1 : 0;
+        ti.r0 = (mt - ti.second * p.dw_row_tiles) * kBM;
+        ti.num_kb = p.dw_kb;
+    }
+    ti.c0 = nt * kBN;
+    return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    swiglu_gemm_bwd_tf32x3_kernel(const __grid_constant__ CUtensorMap tm_a0,
-                                  const __grid_constant__ CUtensorMap tm_a1,
-                                  const __grid_constant__ CUtensorMap tm_b0,
-                                  const __grid_constant__ CUtensorMap tm_b1,
-                                  const __grid_constant__ CUtensorMap tm_o0,
-                                  const __grid_constant__ CUtensorMap tm_o1, Geo geo) {
+    swiglu_gemm_bwd_tf32x3_kernel(const __grid_constant__ Maps maps, const Plan plan) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -113,9 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int num_tiles = geo.num_m * geo.num_n;
-    const int num_kb = kMode == kModeDx ? 2 * geo.kb_pair : geo.kb_pair;
-    const int num_chunks = (num_kb + kChunkKB - 1) / kChunkKB;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -128,12 +158,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_a0);
-        tma_prefetch_desc(&tm_a1);
-        tma_prefetch_desc(&tm_b0);
-        tma_prefetch_desc(&tm_b1);
-        tma_prefetch_desc(&tm_o0);
-        tma_prefetch_desc(&tm_o1);
+        if (plan.sched.T_dx > 0) {
+            tma_prefetch_desc(&maps.dx_a[0]);
+            tma_prefetch_desc(&maps.dx_a[1]);
+            tma_prefetch_desc(&maps.dx_b[0]);
+            tma_prefetch_desc(&maps.dx_b[1]);
+            tma_prefetch_desc(&maps.dx_o);
+        }
+        if (plan.sched.T_dw > 0) {
+            tma_prefetch_desc(&maps.dw_a[0]);
+            tma_prefetch_desc(&maps.dw_a[1]);
+            tma_prefetch_desc(&maps.dw_b);
+            tma_prefetch_desc(&maps.dw_o[0]);
+            tma_prefetch_desc(&maps.dw_o[1]);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
@@ -145,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
 
     bool failed = false;
+    TileInfo ti;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -152,13 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
-                int mt, nt;
-                tile_coords(t, geo.num_m, geo.num_n, mt, nt);
-                const int c0 = nt * kBN;
-                const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
-                const int r0 = (mt - second * geo.row_tiles) * kBM;
-                for (int kb = 0; kb < num_kb; ++kb) {
+            for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+                for (int kb = 0; kb < ti.num_kb; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
@@ -166,28 +200,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t st = sst + stage * kStageBytes;
                     mbar_arrive_expect_tx(fb, kRawBytes);
-                    if (kMode == kModeDx) {
-                        const int pair = kb >= geo.kb_pair ? 1 : 0;
-                        const int red0 = (kb - pair * geo.kb_pair) * kBR;
+                    if (ti.kind == gemm::kTileDx) {
+                        const int pair = kb >= plan.kb_pair ? 1 : 0;
+                        const int red0 = (kb - pair * plan.kb_pair) * kBR;
                         // A: [128 rows of dG or dU] x [16 of N], K-major.
-                        tma_load_2d(pair ? &tm_a1 : &tm_a0, fb, st, red0, r0);
+                        tma_load_2d(&maps.dx_a[pair], fb, st, red0, ti.r0);
                         // B: [16 rows of Wg or Wu] x [256 of K], MN-major atoms.
 #pragma unroll
                         for (int j = 0; j < kBN / 32; ++j)
-                            tma_load_2d(pair ? &tm_b1 : &tm_b0, fb, st + kABytes + j * kAtomBytes,
-                                        c0 + 32 * j, red0);
+                            tma_load_2d(&maps.dx_b[pair], fb, st + kABytes + j * kAtomBytes,
+                                        ti.c0 + 32 * j, red0);
                     } else {
                         const int red0 = kb * kBR;
                         // A: [16 rows of M] x [128 of N] of dG or dU, MN-major.
 #pragma unroll
                         for (int j = 0; j < kBM / 32; ++j)
-                            tma_load_2d(second ? &tm_a1 : &tm_a0, fb, st + j * kAtomBytes,
-                                        r0 + 32 * j, red0);
+                            tma_load_2d(&maps.dw_a[ti.second], fb, st + j * kAtomBytes,
+                                        ti.r0 + 32 * j, red0);
                         // B: [16 rows of M] x [256 of K] of X, MN-major.
 #pragma unroll
                         for (int j = 0; j < kBN / 32; ++j)
-                            tma_load_2d(&tm_b0, fb, st + kABytes + j * kAtomBytes, c0 + 32 * j,
-                                        red0);
+                            tma_load_2d(&maps.dw_b, fb, st + kABytes + j * kAtomBytes,
+                                        ti.c0 + 32 * j, red0);
                     }
                     ++issued;
                     if (++stage == kStages) {
@@ -206,19 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = make_idesc(2u, kBM, kBN) | kIdescBMnMajor |
-                                       (kMode == kModeDw ? kIdescAMnMajor : 0u);
+            constexpr uint32_t idesc_dx = make_idesc(2u, kBM, kBN) | kIdescBMnMajor;
+            constexpr uint32_t idesc_dw = idesc_dx | kIdescAMnMajor;
             int stage = 0;
             uint32_t phase = 0;
             uint32_t chunk_phase = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+                const bool dx = ti.kind == gemm::kTileDx;
+                const uint32_t idesc = dx ? idesc_dx : idesc_dw;
+                const int num_chunks = (ti.num_kb + kChunkKB - 1) / kChunkKB;
                 for (int q = 0; q < num_chunks && !failed; ++q) {
                     if (!mbar_wait(bar_cempty, chunk_phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
                     }
                     tc_fence_after();
-                    const int kb_end = min(num_kb, (q + 1) * kChunkKB);
+                    const int kb_end = min(ti.num_kb, (q + 1) * kChunkKB);
                     for (int kb = q * kChunkKB; kb < kb_end; ++kb) {
                         if (!mbar_wait(bar_ready + 8 * stage, phase, abort_flag)) {
                             failed = true;
@@ -226,18 +263,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tc_fence_after();
                         const uint32_t st = sst + stage * kStageBytes;
-                        const uint64_t a_hi = kMode == kModeDx ? sw64_kmajor_desc(st)
-                                                               : sw128b32_mnmajor_desc(st, kAtomBytes);
-                        const uint64_t a_lo = kMode == kModeDx
-                                                  ? sw64_kmajor_desc(st + kRawBytes)
-                                                  : sw128b32_mnmajor_desc(st + kRawBytes, kAtomBytes);
+                        const uint64_t a_hi = dx ? sw64_kmajor_desc(st)
+                                                 : sw128b32_mnmajor_desc(st, kAtomBytes);
+                        const uint64_t a_lo = dx ? sw64_kmajor_desc(st + kRawBytes)
+                                                 : sw128b32_mnmajor_desc(st + kRawBytes, kAtomBytes);
                         const uint64_t b_hi = sw128b32_mnmajor_desc(st + kABytes, kAtomBytes);
                         const uint64_t b_lo = sw128b32_mnmajor_desc(st + kRawBytes + kABytes, kAtomBytes);
 #pragma unroll
                         for (int kk = 0; kk < kBR / kUmmaK; ++kk) {
                             // K-major: +32 B along the 64-byte swizzled row (+2);
                             // MN-major: +8 rows of 128 B (+64).
-                            const uint32_t oa = kMode == kModeDx ? 2u * kk : 64u * kk;
+                            const uint32_t oa = dx ? 2u * kk : 64u * kk;
                             const uint32_t ob = 64u * kk;
                             const uint32_t acc = (kb == q * kChunkKB && kk == 0) ? 0u : 1u;
                             mma_tf32(tmem_base, a_lo + oa, b_hi + ob, idesc, acc);
@@ -263,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
-        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
-            for (int kb = 0; kb < num_kb; ++kb) {
+        for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+            for (int kb = 0; kb < ti.num_kb; ++kb) {
                 if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
                     failed = true;
                     break;
@@ -288,12 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t buf = se + static_cast<uint32_t>(warp - kFirstEpiWarp) * kEpiBufBytes;
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
         uint32_t chunk_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
-            int mt, nt;
-            tile_coords(t, geo.num_m, geo.num_n, mt, nt);
-            const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
-            const int r0 = (mt - second * geo.row_tiles) * kBM;
-            const int c0 = nt * kBN;
+        for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+            const int num_chunks = (ti.num_kb + kChunkKB - 1) / kChunkKB;
             for (int q = 0; q < num_chunks; ++q) {
                 if (!mbar_wait(bar_cfull, chunk_phase, abort_flag)) {
                     failed = true;
@@ -307,6 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(bar_cempty);
             }
             if (failed) break;
+            const bool dx = ti.kind == gemm::kTileDx;
+            const CUtensorMap *out = dx ? &maps.dx_o : &maps.dw_o[ti.second];
+            const int rows = dx ? plan.M : plan.N;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 if (lane == 0) bulk_wait_read<0>();
@@ -322,10 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int x = c0 + c * 32;
-                    const int y = r0 + quad * 32;
-                    if (x < geo.cols && y < geo.rows) {
-                        tma_store_2d(second ? &tm_o1 : &tm_o0, buf, x, y);
+                    const int x = ti.c0 + c * 32;
+                    const int y = ti.r0 + quad * 32;
+                    if (x < plan.K && y < rows) {
+                        tma_store_2d(out, buf, x, y);
                         bulk_commit();
                     }
                 }
@@ -345,22 +380,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-std::atomic<unsigned> g_attr_set_mask[2];
+std::atomic<unsigned> g_attr_set_mask{0};
 
-template <int kMode>
-cudaError_t launch_tiles(const CUtensorMap (&tm)[6], const Geo &geo, const DeviceInfo &dev,
-                         cudaStream_t stream) {
-    auto kernel = swiglu_gemm_bwd_tf32x3_kernel<kMode>;
+// Encodes the maps of the kinds requested (null pointers: kind not run) and
+// launches one persistent grid over all their tiles.
+cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                        const void *X, void *dX, void *dWg, void *dWu, int M, int K, int N,
+                        bool do_dx, bool do_dw, const DeviceInfo &dev, cudaStream_t stream) {
+    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle mn = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+    const uint64_t n_bytes = static_cast<uint64_t>(N) * 4, k_bytes = static_cast<uint64_t>(K) * 4;
+    Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (do_dx &&
+        (!encode_tmap_2d(&maps.dx_a[0], dG, f32, N, M, n_bytes, kBR, kBM, sw64) ||
+         !encode_tmap_2d(&maps.dx_a[1], dU, f32, N, M, n_bytes, kBR, kBM, sw64) ||
+         !encode_tmap_2d(&maps.dx_b[0], Wg, f32, K, N, k_bytes, 32, kBR, mn) ||
+         !encode_tmap_2d(&maps.dx_b[1], Wu, f32, K, N, k_bytes, 32, kBR, mn) ||
+         !encode_tmap_2d(&maps.dx_o, dX, f32, K, M, k_bytes, 32, 32, sw128)))
+        return cudaErrorInvalidValue;
+    if (do_dw &&
+        (!encode_tmap_2d(&maps.dw_a[0], dG, f32, N, M, n_bytes, 32, kBR, mn) ||
+         !encode_tmap_2d(&maps.dw_a[1], dU, f32, N, M, n_bytes, 32, kBR, mn) ||
+         !encode_tmap_2d(&maps.dw_b, X, f32, K, M, k_bytes, 32, kBR, mn) ||
+         !encode_tmap_2d(&maps.dw_o[0], dWg, f32, K, N, k_bytes, 32, 32, sw128) ||
+         !encode_tmap_2d(&maps.dw_o[1], dWu, f32, K, N, k_bytes, 32, 32, sw128)))
+        return cudaErrorInvalidValue;
+    Plan plan{};
+    plan.M = M;
+    plan.N = N;
+    plan.K = K;
+    plan.num_n = (K + kBN - 1) / kBN;
+    plan.dx_num_m = (M + kBM - 1) / kBM;
+    plan.dw_row_tiles = (N + kBM - 1) / kBM;
+    plan.dw_num_m = 2 * plan.dw_row_tiles;
+    plan.kb_pair = (N + kBR - 1) / kBR;
+    plan.dx_kb = 2 * plan.kb_pair;
+    plan.dw_kb = (M + kBR - 1) / kBR;
+    const long long t_dx = do_dx ? static_cast<long long>(plan.dx_num_m) * plan.num_n : 0;
+    const long long t_dw = do_dw ? static_cast<long long>(plan.dw_num_m) * plan.num_n : 0;
+    const long long tiles = t_dx + t_dw;
+    if (tiles == 0) return cudaSuccess;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    plan.sched = gemm::make_bwd_sched(static_cast<int>(t_dx), static_cast<int>(t_dw), grid,
+                                      plan.dx_kb, plan.dw_kb);
     const unsigned bit = 1u << (dev.device & 31);
-    if (!(g_attr_set_mask[kMode].load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!(g_attr_set_mask.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bwd_tf32x3_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemBytes));
         if (e != cudaSuccess) return e;
-        g_attr_set_mask[kMode].fetch_or(bit);
+        g_attr_set_mask.fetch_or(bit);
     }
-    const long long tiles = static_cast<long long>(geo.num_m) * geo.num_n;
-    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm[0], tm[1], tm[2], tm[3], tm[4], tm[5], geo);
+    swiglu_gemm_bwd_tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, plan);
     return cudaGetLastError();
 }
 
@@ -369,54 +443,21 @@ cudaError_t launch_tiles(const CUtensorMap (&tm)[6], const Geo &geo, const Devic
 cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                  void *dX, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
-    Geo geo{};
-    geo.rows = M;
-    geo.cols = K;
-    geo.row_tiles = (M + kBM - 1) / kBM;
-    geo.num_m = geo.row_tiles;
-    geo.num_n = (K + kBN - 1) / kBN;
-    geo.kb_pair = (N + kBR - 1) / kBR;
-    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
-    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
-    const CUtensorMapSwizzle mn = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
-    const uint64_t n_bytes = static_cast<uint64_t>(N) * 4, k_bytes = static_cast<uint64_t>(K) * 4;
-    CUtensorMap tm[6];
-    if (!encode_tmap_2d(&tm[0], dG, f32, N, M, n_bytes, kBR, kBM, sw64) ||
-        !encode_tmap_2d(&tm[1], dU, f32, N, M, n_bytes, kBR, kBM, sw64) ||
-        !encode_tmap_2d(&tm[2], Wg, f32, K, N, k_bytes, 32, kBR, mn) ||
-        !encode_tmap_2d(&tm[3], Wu, f32, K, N, k_bytes, 32, kBR, mn) ||
-        !encode_tmap_2d(&tm[4], dX, f32, K, M, k_bytes, 32, 32, sw128)) {
-        return cudaErrorInvalidValue;
-    }
-    tm[5] = tm[4];
-    return launch_tiles<kModeDx>(tm, geo, dev, stream);
+    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, dev,
+                       stream);
 }
 
 cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
                                  void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
-    Geo geo{};
-    geo.rows = N;
-    geo.cols = K;
-    geo.row_tiles = (N + kBM - 1) / kBM;
-    geo.num_m = 2 * geo.row_tiles;
-    geo.num_n = (K + kBN - 1) / kBN;
-    geo.kb_pair = (M + kBR - 1) / kBR;
-    const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
-    const CUtensorMapSwizzle mn = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
-    const uint64_t n_bytes = static_cast<uint64_t>(N) * 4, k_bytes = static_cast<uint64_t>(K) * 4;
-    CUtensorMap tm[6];
-    if (!encode_tmap_2d(&tm[0], dG, f32, N, M, n_bytes, 32, kBR, mn) ||
-        !encode_tmap_2d(&tm[1], dU, f32, N, M, n_bytes, 32, kBR, mn) ||
-        !encode_tmap_2d(&tm[2], X, f32, K, M, k_bytes, 32, kBR, mn) ||
-        !encode_tmap_2d(&tm[4], dWg, f32, K, N, k_bytes, 32, 32, sw128) ||
-        !encode_tmap_2d(&tm[5], dWu, f32, K, N, k_bytes, 32, 32, sw128)) {
-        return cudaErrorInvalidValue;
-    }
-    tm[3] = tm[2];
-    return launch_tiles<kModeDw>(tm, geo, dev, stream);
+    return launch_plan(dG, dU, nullptr, nullptr, X, nullptr, dWg, dWu, M, K, N, false, true, dev,
+                       stream);
+}
+
+cudaError_t launch_bwd_all_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                  const void *X, void *dX, void *dWg, void *dWu, int M, int K,
+                                  int N, const DeviceInfo &dev, cudaStream_t stream) {
+    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, dev, stream);
 }
 
 cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {

@@ -29,5 +29,65 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
     (void)dev::mbar_wait(bar, parity, reinterpret_cast<volatile int *>(&never));
 }
 
+// ---------------------------------------------------------------------------
+// Static schedule of the backward GEMMs' tiles over the persistent CTAs, for
+// one launch computing dX and/or dWg, dWu.  dX tiles are long (a 2N-deep
+// reduction), dW tiles short (M-deep), so a CTA first takes its round-robin
+// share of the dX tiles (T_dx = q G + r: CTAs below r take q + 1) and then
+// fills with dW tiles in the order in which the CTAs become free:
+//   phase 1: the CTAs with q dX tiles (nB = G - r of them) start dW one dX
+//            tile's time earlier and take R1 = c_dx / c_dw rounds of dW tiles
+//            alone: tile j * nB + b for round j, b their rank among them;
+//   phase 2: from P1 = R1 * nB on, every CTA takes tile P1 + round * G + cta.
+// It is an exact partition of the T_dw tiles (phase 1 covers [0, P1), phase 2
+// the rest, each index once), fixed per launch (deterministic), and the dW
+// tiles in flight at any time are neighbours in the raster (they share the
+// operand blocks in L2).  With T_dw = 0 it is plain round-robin over dX, with
+// T_dx = 0 over dW.
+struct BwdSched {
+    int T_dx, T_dw;   // tiles of each kind
+    int q, r;         // T_dx = q * G + r
+    int R1, nB, P1;   // phase 1: R1 rounds over nB CTAs, P1 = R1 * nB tiles
+};
+
+inline BwdSched make_bwd_sched(int T_dx, int T_dw, int G, long long c_dx, long long c_dw) {
+    BwdSched s{};
+    s.T_dx = T_dx;
+    s.T_dw = T_dw;
+    s.q = T_dx / G;
+    s.r = T_dx % G;
+    s.nB = G - s.r;
+    s.R1 = (s.r > 0 && c_dw > 0) ? static_cast<int>(c_dx / c_dw) : 0;
+    const long long p1 = static_cast<long long>(s.R1) * s.nB;
+    s.P1 = static_cast<int>(p1 < T_dw ? p1 : T_dw);
+    if (s.P1 < p1) s.R1 = (s.P1 + s.nB - 1) / s.nB;  // phase 1 cut short by T_dw
+    return s;
+}
+
+enum : int { kTileDx = 0, kTileDw = 1 };
+
+// The seq-th tile of CTA `cta` of G: returns false once the CTA is done.
+__device__ __forceinline__ bool bwd_tile_of(const BwdSched &s, int cta, int G, int seq,
+                                            int &kind, int &t) {
+    const int ndx = s.q + (cta < s.r ? 1 : 0);
+    if (seq < ndx) {
+        kind = kTileDx;
+        t = cta + seq * G;
+        return true;
+    }
+    const int j = seq - ndx;
+    long long idx;
+    if (cta >= s.r && j < s.R1)
+        idx = static_cast<long long>(j) * s.nB + (cta - s.r);
+    else
+        idx = static_cast<long long>(s.P1) +
+              static_cast<long long>(cta < s.r ? j : j - s.R1) * G + cta;
+    if (cta >= s.r && j < s.R1 && idx >= s.P1) return false;
+    if (idx >= s.T_dw) return false;
+    kind = kTileDw;
+    t = static_cast<int>(idx);
+    return true;
+}
+
 }  // namespace gemm
 }  // namespace swiglu

@@ -71,6 +71,10 @@ cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg,
 cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
                                  void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream);
+// All three fp32 backward GEMMs in one persistent launch (balanced schedule).
+cudaError_t launch_bwd_all_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                  const void *X, void *dX, void *dWg, void *dWu, int M, int K,
+                                  int N, const DeviceInfo &dev, cudaStream_t stream);
 // Output tile width (128, 192 or 256 columns) the backward GEMMs use for a raster
 // of `row_tiles_total` 128-row tiles by `cols` columns.
 int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
