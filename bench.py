@@ -586,6 +586,15 @@ def run_extras(stream, pk):
                 "roofline": {"bound": "tensor", "achieved": round(tf, 1),
                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": round(tf / pk["bf16_tflops"], 4)}})
+    # all three backward GEMMs in one scheduled launch
+    ms = time_op(lambda: up.lib().swiglu_bwd_gemms(
+        dGb.data_ptr(), dUb.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), X.data_ptr(), dX.data_ptr(),
+        dWg.data_ptr(), dWu.data_ptr(), M, K, N, 0, stream.cuda_stream))
+    tf = 2 * fl / (ms * 1e-3) / 1e12
+    add({"workload": "backward dX, dWg, dWu in one launch (swiglu_bwd_gemms), LLaMA-3 8B M=8192 bf16",
+         "metric": "TFLOP/s", "value": round(tf, 1), "ms": round(ms, 4),
+         "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4)}})
     # one whole training step of the projection: forward storing G and U,
     # dSwiGLU, dX, dWg/dWu (dH stands in for the gradient from above)
     dHb = torch.randn((M, N), generator=gen, device=dev).to(torch.bfloat16)
@@ -595,8 +604,9 @@ def run_extras(stream, pk):
         up.lib().swiglu_fwd_epilogue(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
                                      M, K, N, 0, ctypes.byref(epi_gu), 0, stream.cuda_stream)
         up.dswiglu_bwd(dHb, Gs, Us, dGb, dUb, stream=stream)
-        up.swiglu_bwd_dx(dGb, dUb, Wg, Wu, dX, stream=stream)
-        up.swiglu_bwd_dw(dGb, dUb, X, dWg, dWu, stream=stream)
+        up.lib().swiglu_bwd_gemms(dGb.data_ptr(), dUb.data_ptr(), Wg.data_ptr(), Wu.data_ptr(),
+                                  X.data_ptr(), dX.data_ptr(), dWg.data_ptr(), dWu.data_ptr(),
+                                  M, K, N, 0, stream.cuda_stream)
     ms = time_op(train_step, iters=5)
     tf = 3 * fl / (ms * 1e-3) / 1e12
     add({"workload": "training step (forward storing G, U; dSwiGLU; dX; dWg, dWu), "
@@ -661,6 +671,16 @@ def run_extras(stream, pk):
                      "roofline": {"bound": "tensor", "achieved": round(3 * tf, 1),
                                   "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32 MMA)",
                                   "frac": round(3 * tf / tf32_peak, 4)}})
+            ms = time_op(lambda: up.lib().swiglu_bwd_gemms(
+                dGf.data_ptr(), dUf.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), X.data_ptr(),
+                dXf.data_ptr(), dWgf.data_ptr(), dWuf.data_ptr(), M, K, N, 1, stream.cuda_stream),
+                iters=5)
+            tf = 2 * fl / (ms * 1e-3) / 1e12
+            add({"workload": f"fp32 3xTF32 backward dX, dWg, dWu in one launch, {name} M=2048",
+                 "metric": "TFLOP/s (fp32-equivalent)", "value": round(tf, 1), "ms": round(ms, 4),
+                 "roofline": {"bound": "tensor", "achieved": round(3 * tf, 1),
+                              "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32 MMA)",
+                              "frac": round(3 * tf / tf32_peak, 4)}})
             del dGf, dUf, dXf, dWgf, dWuf
         del X, Wg, Wu, H
     torch.cuda.empty_cache()

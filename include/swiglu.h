@@ -266,11 +266,12 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X,
 /*
  * swiglu_bwd_gemms -- swiglu_bwd_dx and swiglu_bwd_dw in one call:
  * dX = dG Wg + dU Wu, dWg = dG^T X, dWu = dU^T X, with the argument rules of
- * both (and dX must not overlap dWg or dWu).  For fp32 the three GEMMs run
- * as ONE persistent launch whose static schedule gives every CTA its share
- * of the long dX tiles and fills with the short dW tiles, so the launch ends
- * in one balanced tail (dX alone has few tiles at small M).  Same results as
- * the two calls, bit for bit (same per-tile arithmetic).
+ * both (and dX must not overlap dWg or dWu).  The three GEMMs run as ONE
+ * persistent launch whose static schedule gives every CTA its share of the
+ * long dX tiles and fills with the short dW tiles, so the launch ends in one
+ * balanced tail (dX alone has few tiles at small M).  fp32: the same results
+ * as the two calls, bit for bit; bf16: the same per element as the two calls
+ * whenever those pick 256-wide tiles (the combined launch always does).
  */
 SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg,
                                 const void *Wu, const void *X, void *dX,

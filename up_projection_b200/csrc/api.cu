@@ -444,13 +444,15 @@ SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg, 
     }
     const bool gemm_x = rx == SWIGLU_ROUTE_BWD_GEMM_BF16 || rx == SWIGLU_ROUTE_BWD_GEMM_TF32X3;
     const bool gemm_w = rw == SWIGLU_ROUTE_BWD_GEMM_BF16 || rw == SWIGLU_ROUTE_BWD_GEMM_TF32X3;
-    if (gemm_x && gemm_w && dtype == SWIGLU_FP32) {
+    if (gemm_x && gemm_w) {
         DeviceInfo dev;
         st = current_device(dev);
         if (st != SWIGLU_OK) return st;
-        st = from_cuda(launch_bwd_all_tf32x3(dG, dU, Wg, Wu, X, dX, dWg, dWu, static_cast<int>(M),
-                                             static_cast<int>(K), static_cast<int>(N), dev, stream));
-        if (st == SWIGLU_OK) t_last_route = SWIGLU_ROUTE_BWD_GEMM_TF32X3;
+        const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+        st = from_cuda(dtype == SWIGLU_FP32
+                           ? launch_bwd_all_tf32x3(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream)
+                           : launch_bwd_all_bf16(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream));
+        if (st == SWIGLU_OK) t_last_route = rx;
         return st;
     }
     // otherwise one call each (zero fills of empty reductions included)

@@ -24,6 +24,10 @@
 //    (they are rastered together); one MMA of N = BN per 16-deep step keeps
 //    the shared-memory operand traffic at the forward's 12 KB per MFLOP.
 //
+// One launch can run dX, dW or both, on the static schedule of
+// gemm_common.cuh (each CTA: its dX tiles first, then dW tiles in the order
+// the CTAs free up), so the combined call ends in one balanced tail.
+//
 // MN-major tiles are TMA boxes {64, 64} in the 128-byte swizzle, one per
 // 64-wide MN atom; the UMMA descriptor walks atoms with its leading byte
 // offset (ptx.cuh).  Out-of-range rows/columns/reduction steps are
@@ -32,6 +36,8 @@
 // bounded: a stuck pipeline sets the status word and the kernel returns
 // after releasing what it holds.
 #include <cuda_bf16.h>
+
+#include <string.h>
 
 #include <atomic>
 
@@ -50,8 +56,6 @@ namespace {
 using namespace dev;
 using gemm::mbar_wait_drain;
 using gemm::tile_coords;
-
-enum : int { kModeDx = 0, kModeDw = 1 };
 
 constexpr int kBM = 128;             // output rows per tile (= MMA M)
 constexpr int kBR = 64;              // reduction depth per stage (128-byte rows)
@@ -87,26 +91,53 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Problem geometry shared by the three roles.
-//   dX: rows = M, red = N per pair (two pairs), row tiles ceil(M/128)
-//   dW: rows = N per matrix (two matrices), red = M, row tiles 2 ceil(N/128)
-struct Geo {
-    int rows;        // output rows of one output matrix
-    int cols;        // output columns (K)
-    int row_tiles;   // row tiles of one output matrix
-    int num_m;       // row tiles in the raster
-    int num_n;       // column tiles
-    int kb_pair;     // 64-deep reduction blocks of one pair
+// Geometry of the two tile kinds and the schedule of one launch.
+struct Plan {
+    int M, N, K;
+    int dx_num_m, dw_row_tiles, dw_num_m, num_n;   // tiles: dx_num_m x num_n, dw_num_m x num_n
+    int dx_kb, dw_kb;                              // 64-deep reduction blocks per tile
+    int kb_pair;                                   // dX: blocks of one pair (dG Wg, dU Wu)
+    gemm::BwdSched sched;
 };
 
-template <int kMode, int kBN>
+// Tensor maps of both kinds (only those of the kinds a launch runs are used).
+struct Maps {
+    CUtensorMap dx_a[2];   // dG, dU: K-major {64, 128}
+    CUtensorMap dx_b[2];   // Wg, Wu: MN-major atoms {64, 64}
+    CUtensorMap dx_o;      // dX
+    CUtensorMap dw_a[2];   // dG, dU: MN-major atoms {64, 64}
+    CUtensorMap dw_b;      // X: MN-major atoms {64, 64}
+    CUtensorMap dw_o[2];   // dWg, dWu
+};
+
+struct TileInfo {
+    int kind, r0, c0, num_kb, second;
+};
+
+template <int kBN>
+__device__ __forceinline__ bool next_tile(const Plan &p, int seq, TileInfo &ti) {
+    int kind, t;
+    if (!gemm::bwd_tile_of(p.sched, blockIdx.x, gridDim.x, seq, kind, t)) return false;
+    int mt, nt;
+    ti.kind = kind;
+    if (kind == gemm::kTileDx) {
+        tile_coords(t, p.dx_num_m, p.num_n, mt, nt);
+        ti.second = 0;
+        ti.r0 = mt * kBM;
+        ti.num_kb = p.dx_kb;
+    } else {
+        tile_coords(t, p.dw_num_m, p.num_n, mt, nt);
+        ti.second = mt >= p.dw_row_tiles ? 1 : 0;
+        ti.r0 = (mt - ti.second * p.dw_row_tiles) * kBM;
+        ti.num_kb = p.dw_kb;
+    }
+    ti.c0 = nt * kBN;
+    return true;
+}
+
+template <int kBN>
 __global__ void __launch_bounds__(kThreads, 1)
-    swiglu_gemm_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_a0,
-                                const __grid_constant__ CUtensorMap tm_a1,
-                                const __grid_constant__ CUtensorMap tm_b0,
-                                const __grid_constant__ CUtensorMap tm_b1,
-                                const __grid_constant__ CUtensorMap tm_o0,
-                                const __grid_constant__ CUtensorMap tm_o1, Geo geo) {
+    swiglu_gemm_bwd_bf16_kernel(const __grid_constant__ Maps maps, const Plan plan) {
     using C = Cfg<kBN>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -126,8 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int num_tiles = geo.num_m * geo.num_n;
-    const int num_kb = kMode == kModeDx ? 2 * geo.kb_pair : geo.kb_pair;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -141,12 +170,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_a0);
-        tma_prefetch_desc(&tm_a1);
-        tma_prefetch_desc(&tm_b0);
-        tma_prefetch_desc(&tm_b1);
-        tma_prefetch_desc(&tm_o0);
-        tma_prefetch_desc(&tm_o1);
+        if (plan.sched.T_dx > 0) {
+            tma_prefetch_desc(&maps.dx_a[0]);
+            tma_prefetch_desc(&maps.dx_a[1]);
+            tma_prefetch_desc(&maps.dx_b[0]);
+            tma_prefetch_desc(&maps.dx_b[1]);
+            tma_prefetch_desc(&maps.dx_o);
+        }
+        if (plan.sched.T_dw > 0) {
+            tma_prefetch_desc(&maps.dw_a[0]);
+            tma_prefetch_desc(&maps.dw_a[1]);
+            tma_prefetch_desc(&maps.dw_b);
+            tma_prefetch_desc(&maps.dw_o[0]);
+            tma_prefetch_desc(&maps.dw_o[1]);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_ptr), C::kTmemCols);
@@ -158,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
 
     bool failed = false;
+    TileInfo ti;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -165,14 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
-                int mt, nt;
-                tile_coords(t, geo.num_m, geo.num_n, mt, nt);
-                const int c0 = nt * kBN;
-                // dW: which matrix this row tile belongs to, and its first row.
-                const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
-                const int r0 = (mt - second * geo.row_tiles) * kBM;
-                for (int kb = 0; kb < num_kb; ++kb) {
+            for (int seq = 0; !failed && next_tile<kBN>(plan, seq, ti); ++seq) {
+                for (int kb = 0; kb < ti.num_kb; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
                         break;
@@ -181,27 +213,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a_dst = sa + stage * kABytes;
                     const uint32_t b_dst = sb + stage * C::kBBytes;
                     mbar_arrive_expect_tx(fb, C::kStageBytes);
-                    if (kMode == kModeDx) {
-                        const int pair = kb >= geo.kb_pair ? 1 : 0;
-                        const int red0 = (kb - pair * geo.kb_pair) * kBR;
+                    if (ti.kind == gemm::kTileDx) {
+                        const int pair = kb >= plan.kb_pair ? 1 : 0;
+                        const int red0 = (kb - pair * plan.kb_pair) * kBR;
                         // A: [128 rows of dG or dU] x [64 of N], K-major.
-                        tma_load_2d(pair ? &tm_a1 : &tm_a0, fb, a_dst, red0, r0);
+                        tma_load_2d(&maps.dx_a[pair], fb, a_dst, red0, ti.r0);
                         // B: [64 rows of Wg or Wu] x [BN of K], MN-major atoms.
 #pragma unroll
                         for (int j = 0; j < kBN / 64; ++j)
-                            tma_load_2d(pair ? &tm_b1 : &tm_b0, fb, b_dst + j * kAtomBytes,
-                                        c0 + 64 * j, red0);
+                            tma_load_2d(&maps.dx_b[pair], fb, b_dst + j * kAtomBytes,
+                                        ti.c0 + 64 * j, red0);
                     } else {
                         const int red0 = kb * kBR;
                         // A: [64 rows of M] x [128 of N] of dG or dU, MN-major.
 #pragma unroll
                         for (int j = 0; j < kBM / 64; ++j)
-                            tma_load_2d(second ? &tm_a1 : &tm_a0, fb, a_dst + j * kAtomBytes,
-                                        r0 + 64 * j, red0);
+                            tma_load_2d(&maps.dw_a[ti.second], fb, a_dst + j * kAtomBytes,
+                                        ti.r0 + 64 * j, red0);
                         // B: [64 rows of M] x [BN of K] of X, MN-major.
 #pragma unroll
                         for (int j = 0; j < kBN / 64; ++j)
-                            tma_load_2d(&tm_b0, fb, b_dst + j * kAtomBytes, c0 + 64 * j, red0);
+                            tma_load_2d(&maps.dw_b, fb, b_dst + j * kAtomBytes, ti.c0 + 64 * j,
+                                        red0);
                     }
                     ++issued;
                     if (++stage == C::kStages) {
@@ -220,35 +253,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = make_idesc(1u, kBM, kBN) | kIdescBMnMajor |
-                                       (kMode == kModeDw ? kIdescAMnMajor : 0u);
+            constexpr uint32_t idesc_dx = make_idesc(1u, kBM, kBN) | kIdescBMnMajor;
+            constexpr uint32_t idesc_dw = idesc_dx | kIdescAMnMajor;
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            for (int seq = 0; !failed && next_tile<kBN>(plan, seq, ti); ++seq) {
+                const bool dx = ti.kind == gemm::kTileDx;
+                const uint32_t idesc = dx ? idesc_dx : idesc_dw;
                 if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag)) {
                     failed = true;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = 0; kb < ti.num_kb; ++kb) {
                     if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
                         failed = true;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_addr = sa + stage * kABytes;
-                    const uint64_t adesc = kMode == kModeDx
-                                               ? sw128_kmajor_desc(a_addr)
-                                               : sw128_mnmajor_desc(a_addr, kAtomBytes);
+                    const uint64_t adesc = dx ? sw128_kmajor_desc(a_addr)
+                                              : sw128_mnmajor_desc(a_addr, kAtomBytes);
                     const uint64_t bdesc = sw128_mnmajor_desc(sb + stage * C::kBBytes, kAtomBytes);
 #pragma unroll
                     for (int kk = 0; kk < kBR / kUmmaK; ++kk) {
                         // K-major: +32 B along the swizzled row (+2); MN-major:
                         // +16 rows of 128 B (+128).
-                        const uint64_t a_step = kMode == kModeDx ? 2u * kk : 128u * kk;
+                        const uint64_t a_step = dx ? 2u * kk : 128u * kk;
                         mma_f16(d_tmem, adesc + a_step, bdesc + 128u * kk, idesc,
                                 (kb > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -276,17 +310,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            int mt, nt;
-            tile_coords(t, geo.num_m, geo.num_n, mt, nt);
-            const int second = (kMode == kModeDw && mt >= geo.row_tiles) ? 1 : 0;
-            const int r0 = (mt - second * geo.row_tiles) * kBM;
-            const int c0 = nt * kBN;
+        for (int seq = 0; next_tile<kBN>(plan, seq, ti); ++seq) {
             if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
                 failed = true;
                 break;
             }
             tc_fence_after();
+            const bool dx = ti.kind == gemm::kTileDx;
+            const CUtensorMap *out = dx ? &maps.dx_o : &maps.dw_o[ti.second];
+            const int rows = dx ? plan.M : plan.N;
             const uint32_t tacc = tmem_base + row_off + static_cast<uint32_t>(acc * kBN);
 #pragma unroll 1
             for (int c = 0; c < kBN / 64; ++c) {
@@ -313,10 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int x = c0 + c * 64;
-                    const int y = r0 + quad * 32;
-                    if (x < geo.cols && y < geo.rows) {
-                        tma_store_2d(second ? &tm_o1 : &tm_o0, buf, x, y);
+                    const int x = ti.c0 + c * 64;
+                    const int y = ti.r0 + quad * 32;
+                    if (x < plan.K && y < rows) {
+                        tma_store_2d(out, buf, x, y);
                         bulk_commit();
                     }
                 }
@@ -343,13 +375,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-std::atomic<unsigned> g_attr_set_mask[6];
+std::atomic<unsigned> g_attr_set_mask[3];
 
-template <int kMode, int kBN>
-cudaError_t launch_tiles(const CUtensorMap (&tm)[6], const Geo &geo, const DeviceInfo &dev,
+template <int kBN>
+cudaError_t launch_width(const Maps &maps, const Plan &plan, int grid, const DeviceInfo &dev,
                          cudaStream_t stream) {
-    auto kernel = swiglu_gemm_bwd_bf16_kernel<kMode, kBN>;
-    constexpr int slot = kMode * 3 + kBN / 64 - 2;
+    auto kernel = swiglu_gemm_bwd_bf16_kernel<kBN>;
+    constexpr int slot = kBN / 64 - 2;
     const unsigned bit = 1u << (dev.device & 31);
     if (!(g_attr_set_mask[slot].load() & bit)) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -357,11 +389,58 @@ cudaError_t launch_tiles(const CUtensorMap (&tm)[6], const Geo &geo, const Devic
         if (e != cudaSuccess) return e;
         g_attr_set_mask[slot].fetch_or(bit);
     }
-    const long long tiles = static_cast<long long>(geo.num_m) * geo.num_n;
-    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    kernel<<<grid, kThreads, Cfg<kBN>::kSmemBytes, stream>>>(tm[0], tm[1], tm[2], tm[3], tm[4],
-                                                             tm[5], geo);
+    kernel<<<grid, kThreads, Cfg<kBN>::kSmemBytes, stream>>>(maps, plan);
     return cudaGetLastError();
+}
+
+// Encodes the maps of the kinds requested and launches one persistent grid
+// over all their tiles, `bn` columns wide.
+cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                        const void *X, void *dX, void *dWg, void *dWu, int M, int K, int N,
+                        bool do_dx, bool do_dw, int bn, const DeviceInfo &dev,
+                        cudaStream_t stream) {
+    const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint64_t n_bytes = static_cast<uint64_t>(N) * 2, k_bytes = static_cast<uint64_t>(K) * 2;
+    Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (do_dx &&
+        (!encode_tmap_2d(&maps.dx_a[0], dG, bf16, N, M, n_bytes, kBR, kBM, sw) ||
+         !encode_tmap_2d(&maps.dx_a[1], dU, bf16, N, M, n_bytes, kBR, kBM, sw) ||
+         !encode_tmap_2d(&maps.dx_b[0], Wg, bf16, K, N, k_bytes, 64, kBR, sw) ||
+         !encode_tmap_2d(&maps.dx_b[1], Wu, bf16, K, N, k_bytes, 64, kBR, sw) ||
+         !encode_tmap_2d(&maps.dx_o, dX, bf16, K, M, k_bytes, 64, 32, sw)))
+        return cudaErrorInvalidValue;
+    if (do_dw &&
+        (!encode_tmap_2d(&maps.dw_a[0], dG, bf16, N, M, n_bytes, 64, kBR, sw) ||
+         !encode_tmap_2d(&maps.dw_a[1], dU, bf16, N, M, n_bytes, 64, kBR, sw) ||
+         !encode_tmap_2d(&maps.dw_b, X, bf16, K, M, k_bytes, 64, kBR, sw) ||
+         !encode_tmap_2d(&maps.dw_o[0], dWg, bf16, K, N, k_bytes, 64, 32, sw) ||
+         !encode_tmap_2d(&maps.dw_o[1], dWu, bf16, K, N, k_bytes, 64, 32, sw)))
+        return cudaErrorInvalidValue;
+    Plan plan{};
+    plan.M = M;
+    plan.N = N;
+    plan.K = K;
+    plan.num_n = (K + bn - 1) / bn;
+    plan.dx_num_m = (M + kBM - 1) / kBM;
+    plan.dw_row_tiles = (N + kBM - 1) / kBM;
+    plan.dw_num_m = 2 * plan.dw_row_tiles;
+    plan.kb_pair = (N + kBR - 1) / kBR;
+    plan.dx_kb = 2 * plan.kb_pair;
+    plan.dw_kb = (M + kBR - 1) / kBR;
+    const long long t_dx = do_dx ? static_cast<long long>(plan.dx_num_m) * plan.num_n : 0;
+    const long long t_dw = do_dw ? static_cast<long long>(plan.dw_num_m) * plan.num_n : 0;
+    const long long tiles = t_dx + t_dw;
+    if (tiles == 0) return cudaSuccess;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    plan.sched = gemm::make_bwd_sched(static_cast<int>(t_dx), static_cast<int>(t_dw), grid,
+                                      plan.dx_kb, plan.dw_kb);
+    switch (bn) {
+        case 128: return launch_width<128>(maps, plan, grid, dev, stream);
+        case 192: return launch_width<192>(maps, plan, grid, dev, stream);
+        default: return launch_width<256>(maps, plan, grid, dev, stream);
+    }
 }
 
 }  // namespace
@@ -393,61 +472,24 @@ int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count) {
 cudaError_t launch_bwd_dx_bf16(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                void *dX, int M, int K, int N, const DeviceInfo &dev,
                                cudaStream_t stream) {
-    Geo geo{};
-    geo.rows = M;
-    geo.cols = K;
-    geo.row_tiles = (M + kBM - 1) / kBM;
-    geo.num_m = geo.row_tiles;
-    geo.kb_pair = (N + kBR - 1) / kBR;
-    const int bn = bwd_gemm_tile_n(geo.num_m, K, dev.sm_count);
-    geo.num_n = (K + bn - 1) / bn;
-    const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    const uint64_t n_bytes = static_cast<uint64_t>(N) * 2, k_bytes = static_cast<uint64_t>(K) * 2;
-    CUtensorMap tm[6];
-    if (!encode_tmap_2d(&tm[0], dG, bf16, N, M, n_bytes, kBR, kBM, sw) ||
-        !encode_tmap_2d(&tm[1], dU, bf16, N, M, n_bytes, kBR, kBM, sw) ||
-        !encode_tmap_2d(&tm[2], Wg, bf16, K, N, k_bytes, 64, kBR, sw) ||
-        !encode_tmap_2d(&tm[3], Wu, bf16, K, N, k_bytes, 64, kBR, sw) ||
-        !encode_tmap_2d(&tm[4], dX, bf16, K, M, k_bytes, 64, 32, sw)) {
-        return cudaErrorInvalidValue;
-    }
-    tm[5] = tm[4];
-    switch (bn) {
-        case 128: return launch_tiles<kModeDx, 128>(tm, geo, dev, stream);
-        case 192: return launch_tiles<kModeDx, 192>(tm, geo, dev, stream);
-        default: return launch_tiles<kModeDx, 256>(tm, geo, dev, stream);
-    }
+    const int bn = bwd_gemm_tile_n((M + kBM - 1) / kBM, K, dev.sm_count);
+    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, bn,
+                       dev, stream);
 }
 
 cudaError_t launch_bwd_dw_bf16(const void *dG, const void *dU, const void *X, void *dWg,
                                void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                cudaStream_t stream) {
-    Geo geo{};
-    geo.rows = N;
-    geo.cols = K;
-    geo.row_tiles = (N + kBM - 1) / kBM;
-    geo.num_m = 2 * geo.row_tiles;
-    geo.kb_pair = (M + kBR - 1) / kBR;
-    const int bn = bwd_gemm_tile_n(geo.num_m, K, dev.sm_count);
-    geo.num_n = (K + bn - 1) / bn;
-    const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    const uint64_t n_bytes = static_cast<uint64_t>(N) * 2, k_bytes = static_cast<uint64_t>(K) * 2;
-    CUtensorMap tm[6];
-    if (!encode_tmap_2d(&tm[0], dG, bf16, N, M, n_bytes, 64, kBR, sw) ||
-        !encode_tmap_2d(&tm[1], dU, bf16, N, M, n_bytes, 64, kBR, sw) ||
-        !encode_tmap_2d(&tm[2], X, bf16, K, M, k_bytes, 64, kBR, sw) ||
-        !encode_tmap_2d(&tm[4], dWg, bf16, K, N, k_bytes, 64, 32, sw) ||
-        !encode_tmap_2d(&tm[5], dWu, bf16, K, N, k_bytes, 64, 32, sw)) {
-        return cudaErrorInvalidValue;
-    }
-    tm[3] = tm[2];
-    switch (bn) {
-        case 128: return launch_tiles<kModeDw, 128>(tm, geo, dev, stream);
-        case 192: return launch_tiles<kModeDw, 192>(tm, geo, dev, stream);
-        default: return launch_tiles<kModeDw, 256>(tm, geo, dev, stream);
-    }
+    const int bn = bwd_gemm_tile_n(2 * ((N + kBM - 1) / kBM), K, dev.sm_count);
+    return launch_plan(dG, dU, nullptr, nullptr, X, nullptr, dWg, dWu, M, K, N, false, true, bn,
+                       dev, stream);
+}
+
+// All three in one launch: the dW tiles fill dX's tail, so the full width.
+cudaError_t launch_bwd_all_bf16(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                const void *X, void *dX, void *dWg, void *dWu, int M, int K,
+                                int N, const DeviceInfo &dev, cudaStream_t stream) {
+    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, 256, dev, stream);
 }
 
 cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {

@@ -64,6 +64,10 @@ cudaError_t launch_bwd_dx_bf16(const void *dG, const void *dU, const void *Wg, c
 cudaError_t launch_bwd_dw_bf16(const void *dG, const void *dU, const void *X, void *dWg,
                                void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                cudaStream_t stream);
+// All three bf16 backward GEMMs in one persistent launch (balanced schedule).
+cudaError_t launch_bwd_all_bf16(const void *dG, const void *dU, const void *Wg, const void *Wu,
+                                const void *X, void *dX, void *dWg, void *dWu, int M, int K,
+                                int N, const DeviceInfo &dev, cudaStream_t stream);
 // fp32 backward GEMMs (3xTF32), same operations, K and N multiples of 4.
 cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                  void *dX, int M, int K, int N, const DeviceInfo &dev,
