@@ -10,10 +10,13 @@ call streams its weights cold from HBM -- the cold-weight protocol of
 AstrAI swiglu_benchmark.md ("HBM re-measurement and kernel simplification").
 Metric: algorithmic bytes (Wg + Wu + X + H) / device time, GB/s.
 
-Also measured (key "also", not part of the step): prefill at the LLaMA-3 8B
-shape (TFLOP/s), dSwiGLU on [8192, 14336] bf16 (GB/s), the fp32 3xTF32 mode
-at the LLaMA-2 13B and GPT-NeoX 20B shapes (TFLOP/s), and the LLaMA-2 7B
-decode shape (GB/s), each with its roofline fraction.
+Also measured on single-GPU runs (key "also", not part of the step): the
+prefill at the LLaMA-3 8B shape and its variants (training forward storing
+G and U, GEGLU with a gate multiplier, fp8 output), the backward GEMMs (dX,
+dW, all three in one launch) and a whole training step of the projection
+(TFLOP/s), dSwiGLU on [8192, 14336] bf16 (GB/s), the fp32 3xTF32 forward and
+backward at the LLaMA-2 13B and GPT-NeoX 20B shapes, and the LLaMA-2 7B
+decode shape (GB/s), each with its roofline fraction and the SM clock seen.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and cuda synchronize, CUDA events on the launching stream, max over ranks.
@@ -873,7 +876,10 @@ def main(argv=None):
             "us": {k: round(v, 2) for k, v in dec["comparators"]["us"].items()},
             "GB/s": {k: round(v, 1) for k, v in dec["comparators"]["GB/s"].items()}},
     }
-    if rank == 0 and not args.no_extra:
+    # The extra single-GPU measurements take about a minute; under torchrun
+    # the other ranks would idle in the closing barrier meanwhile, so they
+    # run in single-GPU runs only.
+    if rank == 0 and world == 1 and not args.no_extra:
         line["also"] = run_extras(stream, pk)
         # LLaMA-2 7B decode shape as a second cold-weight line
         s7 = max(40, min(2000, args.steps // 4))
