@@ -103,7 +103,8 @@ enum swiglu_flags {
      * the decode kernel may start streaming them before that work has
      * finished (programmatic dependent launch).  X is still read, and H
      * written, only after all earlier work on the stream has completed.
-     * Ignored by routes other than SWIGLU_ROUTE_DECODE_BF16. */
+     * Used by SWIGLU_ROUTE_DECODE_BF16 and SWIGLU_ROUTE_STREAM_TC_BF16,
+     * ignored by the other routes. */
     SWIGLU_FLAG_WEIGHTS_STABLE = 1
 };
 
@@ -111,11 +112,16 @@ enum swiglu_flags {
 enum swiglu_route {
     SWIGLU_ROUTE_NONE = 0,        /* empty problem: nothing enqueued        */
     SWIGLU_ROUTE_ZERO_K = 1,      /* K == 0: H is filled with zeros         */
-    SWIGLU_ROUTE_DECODE_BF16 = 2, /* bf16, M <= 8: weight-streaming kernel  */
-    SWIGLU_ROUTE_GEMM_BF16 = 3,   /* bf16, M > 8: tcgen05 dual GEMM         */
+    SWIGLU_ROUTE_DECODE_BF16 = 2, /* bf16, M <= 8: weight streaming with
+                                     warp-level tensor-core MMA             */
+    SWIGLU_ROUTE_GEMM_BF16 = 3,   /* bf16, larger M: tcgen05 dual GEMM      */
     SWIGLU_ROUTE_GEMM_TF32X3 = 4, /* fp32: 3xTF32 tcgen05 dual GEMM         */
     SWIGLU_ROUTE_BWD_GEMM_BF16 = 5, /* bf16 backward GEMM (swiglu_bwd_dx/_dw) */
-    SWIGLU_ROUTE_BWD_GEMM_TF32X3 = 6 /* fp32 backward GEMM, 3xTF32          */
+    SWIGLU_ROUTE_BWD_GEMM_TF32X3 = 6, /* fp32 backward GEMM, 3xTF32         */
+    SWIGLU_ROUTE_STREAM_TC_BF16 = 7 /* bf16, 9 <= M <= 128, K a multiple of
+                                     64: weight streaming on tcgen05 (X the
+                                     128-row operand, 8 gate + 8 up weight
+                                     rows the 16-row one)                   */
 };
 
 /*
@@ -135,6 +141,7 @@ enum swiglu_route {
  *  one round-to-nearest-even to bf16; NaN/Inf propagate (no saturation).
  *  fp32: each operand is split a = hi + lo (hi, lo TF32), and the three
  *  products hi*hi + hi*lo + lo*hi are accumulated in fp32 on tensor cores.
+ *  The route (swiglu_route_for) is a pure function of M, K, N and dtype.
  *  No call allocates device memory.
  */
 SWIGLU_API int swiglu_fwd(const void *X, const void *Wg, const void *Wu,

@@ -32,7 +32,16 @@ def test_routes_are_a_pure_function_of_shape():
     r = _capi.swiglu_route_for
     assert r(8, 1536, 6912, 0) == _capi.ROUTE_DECODE_BF16
     assert r(1, 4096, 11008, 0) == _capi.ROUTE_DECODE_BF16
-    assert r(9, 4096, 11008, 0) == _capi.ROUTE_GEMM_BF16
+    for M in (9, 24, 64, 128):
+        assert r(M, 4096, 11008, 0) == _capi.ROUTE_STREAM_TC_BF16
+        assert r(M, 1536, 6912, 0) == _capi.ROUTE_STREAM_TC_BF16
+    assert r(129, 4096, 11008, 0) == _capi.ROUTE_GEMM_BF16
+    for M in (9, 12, 16, 17, 24, 25, 31, 32, 100, 128):
+        for K, N in ((264, 72), (8, 8), (40, 1032), (2000, 264), (520, 6912)):
+            # K not a multiple of 64
+            assert r(M, K, N, 0) == _capi.ROUTE_GEMM_BF16, (M, K, N)
+        for K, N in ((64, 8), (256, 512), (1536, 6912), (832, 1032), (4096, 264)):
+            assert r(M, K, N, 0) == _capi.ROUTE_STREAM_TC_BF16, (M, K, N)
     assert r(8192, 4096, 14336, 0) == _capi.ROUTE_GEMM_BF16
     assert r(2048, 5120, 13824, 1) == _capi.ROUTE_GEMM_TF32X3
     assert r(8, 64, 64, 1) == _capi.ROUTE_GEMM_TF32X3

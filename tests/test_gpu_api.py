@@ -46,7 +46,8 @@ def test_error_codes_with_device_pointers():
 
 def test_routes_engage_their_kernels():
     for M, route in ((1, _capi.ROUTE_DECODE_BF16), (8, _capi.ROUTE_DECODE_BF16),
-                     (9, _capi.ROUTE_GEMM_BF16), (64, _capi.ROUTE_GEMM_BF16)):
+                     (9, _capi.ROUTE_STREAM_TC_BF16), (128, _capi.ROUTE_STREAM_TC_BF16),
+                     (129, _capi.ROUTE_GEMM_BF16), (200, _capi.ROUTE_GEMM_BF16)):
         X, Wg, Wu = (t.to(dev()) for t in synth.swiglu_inputs(M, 128, 64, "bf16"))
         _capi.swiglu_fwd(X, Wg, Wu)
         assert _capi.swiglu_last_route() == route, M

@@ -58,18 +58,74 @@ def test_decode_llama7b_full(M):
     check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"llama7b M={M}")
 
 
-def test_decode_integer_exact():
+@pytest.mark.parametrize("M", [9, 16, 17, 31, 64, 128])
+@pytest.mark.parametrize("K,N", [(264, 72), (8, 8), (40, 1032), (2000, 264), (520, 6912)])
+def test_small_m_gemm_shapes(M, K, N):
+    """9 <= M <= 128 with K not a multiple of 64 takes the dual GEMM (one
+    ragged M tile); every output against the oracle."""
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 1000 + K + 1)
+    check_full(X, Wg, Wu, _capi.ROUTE_GEMM_BF16, f"gemm M={M} K={K} N={N}")
+
+
+# ------------------------------------------------- tcgen05 weight stream
+
+@pytest.mark.parametrize("M", [9, 15, 16, 17, 24, 32, 33, 47, 64, 65, 100, 127, 128])
+@pytest.mark.parametrize("K,N", [(64, 8), (128, 520), (256, 512), (1536, 6912), (832, 1032),
+                                 (4096, 264)])
+def test_stream_tc_shapes(M, K, N):
+    """9 <= M <= 128, K a multiple of 64: one k-block (K = 64), a partial last
+    slice (K = 832), several slices, ragged M against the 8-row X boxes;
+    every output against the oracle."""
+    assert _capi.swiglu_route_for(M, K, N, 0) == _capi.ROUTE_STREAM_TC_BF16
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 977 + K + N)
+    check_full(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16, f"stream M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M", [16, 32, 64])
+def test_stream_tc_llama7b_full(M):
+    """LLaMA-2 7B up/gate shape at batched-decode M (all outputs checked)."""
+    X, Wg, Wu = synth.swiglu_inputs(M, 4096, 11008, "bf16", seed=70 + M)
+    check_full(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16, f"llama7b M={M}")
+
+
+def test_stream_tc_many_units_per_cta():
+    """N = 8 * 148 * 32 + 8: more units than TMEM holds for one CTA per SM,
+    so the grid grows past the SM count; sampled outputs incl. the last."""
+    M, K, N = 24, 128, 8 * 148 * 32 + 8
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=5)
+    H = run_fwd(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16)
+    im, inn = sample_indices(M, N, 6000)
+    im = np.concatenate([im, np.arange(M)])
+    inn = np.concatenate([inn, np.full(M, N - 1)])
+    ref = oracle.swiglu_fwd_points(X, Wg, Wu, im, inn, "bf16")["H"]
+    assert_bf16_close(f64(H[im, inn]), ref, "stream many units")
+
+
+def test_stream_tc_deterministic():
+    X, Wg, Wu = synth.swiglu_inputs(32, 1536, 6912, "bf16", seed=4)
+    a = run_fwd(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16)
+    b = run_fwd(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_small_m_integer_exact():
     """Integer operands with every gate pre-activation >= 17: sigmoid rounds
     to 1 in fp32, so H = bf16_rne(fp32(G * U)) exactly, for every tile and
-    lane position -- any indexing or layout slip changes bits."""
-    for M, K, N in [(8, 256, 512), (3, 136, 1024), (1, 64, 8)]:
+    lane position -- any indexing or layout slip changes bits.  Covers the
+    decode kernel, the tcgen05 weight stream and the dual GEMM at small M."""
+    routes = set()
+    for M, K, N in [(8, 256, 512), (3, 136, 1024), (1, 64, 8), (9, 264, 512), (32, 136, 1024),
+                    (17, 72, 8), (9, 256, 512), (64, 128, 1032), (128, 192, 264), (33, 1536, 264),
+                    (17, 64, 8), (65, 256, 136)]:
         X, Wg, Wu = synth.integer_inputs(M, K, N, seed=M + K)
-        H = run_fwd(X, Wg, Wu, _capi.ROUTE_DECODE_BF16)
+        H = run_fwd(X, Wg, Wu)
+        routes.add(_capi.swiglu_last_route())
         G = X.to(torch.float64) @ Wg.to(torch.float64).T
         U = X.to(torch.float64) @ Wu.to(torch.float64).T
         assert float(G.min()) >= 17.0
         expect = (G * U).to(torch.float32).to(torch.bfloat16)
         assert torch.equal(H.view(torch.int16), expect.view(torch.int16)), (M, K, N)
+    assert routes == {_capi.ROUTE_DECODE_BF16, _capi.ROUTE_STREAM_TC_BF16, _capi.ROUTE_GEMM_BF16}
 
 
 def test_decode_deterministic():
@@ -82,9 +138,11 @@ def test_decode_deterministic():
 # --------------------------------------------------------------- dual GEMM
 
 @pytest.mark.parametrize("M,K,N", [
-    (9, 256, 512),       # smallest GEMM-route M
-    (128, 64, 128),      # one tile, one k-block
-    (128, 128, 256),     # two k-blocks, two N tiles
+    (129, 256, 512),     # smallest GEMM-route M at K a multiple of 64
+    (33, 264, 512),      # smallest GEMM-route M at other K
+    (9, 65544, 64),      # K not a multiple of 64, X rows too large for decode
+    (129, 64, 128),      # one N tile, one k-block, a one-row second M tile
+    (200, 128, 256),     # two k-blocks, two N tiles
     (129, 72, 136),      # ragged M, ragged K (not a multiple of 64), ragged N
     (300, 520, 392),     # several ragged tiles
     (256, 4096, 512),    # long K: the smem ring wraps many times
@@ -169,6 +227,20 @@ def test_decode_weights_stable_path(K, N):
         assert_bf16_close(f64(H), oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"], f"pdl M={M} K={K}")
 
 
+@pytest.mark.parametrize("K,N", [(1536, 6912), (4096, 11008), (256, 512), (264, 72)])
+def test_decode_weights_stable_mid_m(K, N):
+    """weights_stable at 9 <= M <= 32 on the route the shape takes: the
+    tcgen05 weight stream (its first stages' weights requested before the
+    wait for X), or the dual GEMM where K is not a multiple of 64."""
+    for M in (9, 16, 24, 32):
+        X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M + 9)
+        Xd, Wgd, Wud = to_dev(X, Wg, Wu)
+        H = _capi.swiglu_fwd(Xd, Wgd, Wud, weights_stable=True)
+        assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+        assert _capi.swiglu_last_route() == _capi.swiglu_route_for(M, K, N, 0)
+        assert_bf16_close(f64(H), oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"], f"pdl M={M} K={K}")
+
+
 def test_decode_weights_stable_chain_reads_x_after_producer():
     """A chain of dependent decode calls on one stream, each call's input X
     being the previous call's output H, all with weights_stable: every X read
@@ -205,7 +277,7 @@ def _random_shapes(seed, count, ms):
     return out
 
 
-@pytest.mark.parametrize("M,K,N", _random_shapes(2024, 16, [9, 10, 12, 63, 127, 129, 255, 257]))
+@pytest.mark.parametrize("M,K,N", _random_shapes(2024, 16, [129, 130, 160, 200, 255, 257, 300, 511]))
 def test_gemm_random_odd_shapes(M, K, N):
     """Seeded random shapes around tile boundaries: ragged M (127, 129, 257...),
     K and N any multiple of 8 up to 632, every output against the oracle."""
@@ -213,7 +285,25 @@ def test_gemm_random_odd_shapes(M, K, N):
     check_full(X, Wg, Wu, _capi.ROUTE_GEMM_BF16, f"gemm M={M} K={K} N={N}")
 
 
-@pytest.mark.parametrize("M,K,N", _random_shapes(2025, 10, [1, 2, 3, 5, 7, 8]))
+@pytest.mark.parametrize("M,K,N", _random_shapes(2025, 10, [1, 2, 3, 5, 7, 8])
+                         + _random_shapes(2026, 10, [9, 11, 15, 19, 23, 28, 32]))
 def test_decode_random_odd_shapes(M, K, N):
+    """Random shapes at M <= 32 (decode at M <= 8; above, the tcgen05 stream
+    where K is a multiple of 64, the dual GEMM otherwise)."""
     X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 11 + K * 5 + N)
-    check_full(X, Wg, Wu, _capi.ROUTE_DECODE_BF16, f"decode M={M} K={K} N={N}")
+    route = _capi.swiglu_route_for(M, K, N, 0)
+    assert route == _capi.ROUTE_DECODE_BF16 if M <= 8 else route in (
+        _capi.ROUTE_STREAM_TC_BF16, _capi.ROUTE_GEMM_BF16)
+    check_full(X, Wg, Wu, route, f"small-M M={M} K={K} N={N}")
+
+
+def _random_stream_shapes(seed, count):
+    r = np.random.Generator(np.random.PCG64(seed))
+    return [(int(r.integers(9, 129)), int(r.integers(1, 40)) * 64, int(r.integers(1, 200)) * 8)
+            for _ in range(count)]
+
+
+@pytest.mark.parametrize("M,K,N", _random_stream_shapes(2027, 16))
+def test_stream_tc_random_shapes(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 13 + K * 7 + N)
+    check_full(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16, f"stream M={M} K={K} N={N}")

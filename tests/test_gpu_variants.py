@@ -71,6 +71,9 @@ def run_variant(X, Wg, Wu, which, alpha, store_gu):
 CASES = [  # (M, K, N, dtype, route)
     (1, 256, 512, "bf16", _capi.ROUTE_DECODE_BF16),
     (8, 1536, 1032, "bf16", _capi.ROUTE_DECODE_BF16),
+    (24, 264, 72, "bf16", _capi.ROUTE_GEMM_BF16),
+    (33, 1536, 1032, "bf16", _capi.ROUTE_STREAM_TC_BF16),
+    (128, 256, 264, "bf16", _capi.ROUTE_STREAM_TC_BF16),
     (130, 192, 264, "bf16", _capi.ROUTE_GEMM_BF16),
     (300, 520, 392, "bf16", _capi.ROUTE_GEMM_BF16),
     (130, 96, 136, "f32", _capi.ROUTE_GEMM_TF32X3),
@@ -106,8 +109,8 @@ def test_forward_variants(M, K, N, dtype, route, which, alpha, store_gu):
 def test_training_forward_integer_exact_gu():
     """Stored G and U are the fp32 accumulators rounded once to bf16: with
     integer operands G and U are exact in fp32, so the stored bits must be
-    bf16_rne(G), bf16_rne(U) exactly, on both bf16 routes."""
-    for M, K, N in [(8, 256, 512), (256, 256, 384)]:
+    bf16_rne(G), bf16_rne(U) exactly, on every bf16 route."""
+    for M, K, N in [(8, 256, 512), (256, 256, 384), (40, 256, 1032), (17, 200, 64)]:
         X, Wg, Wu = synth.integer_inputs(M, K, N, seed=M)
         out = run_variant(X, Wg, Wu, SILU, 1.0, True)
         G = (X.double() @ Wg.double().T).float().to(torch.bfloat16)

@@ -45,6 +45,7 @@ ROUTE_GEMM_BF16 = 3
 ROUTE_GEMM_TF32X3 = 4
 ROUTE_BWD_GEMM_BF16 = 5
 ROUTE_BWD_GEMM_TF32X3 = 6
+ROUTE_STREAM_TC_BF16 = 7
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64

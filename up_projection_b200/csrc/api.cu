@@ -85,6 +85,9 @@ int route_of_shape(int64_t M, int64_t K, int64_t N, int dtype, int *route) {
     else if (dtype == SWIGLU_FP32) *route = SWIGLU_ROUTE_GEMM_TF32X3;
     else if (M <= kDecodeMaxM && decode_bf16_supported(static_cast<int>(K)))
         *route = SWIGLU_ROUTE_DECODE_BF16;
+    else if (M <= kStreamTcMaxM &&
+             stream_tc_bf16_supported(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N)))
+        *route = SWIGLU_ROUTE_STREAM_TC_BF16;
     else *route = SWIGLU_ROUTE_GEMM_BF16;
     return SWIGLU_OK;
 }
@@ -276,6 +279,10 @@ SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu
         case SWIGLU_ROUTE_DECODE_BF16:
             e = launch_decode_bf16(X, Wg, Wu, H, m, k, n, ep,
                                    (flags & SWIGLU_FLAG_WEIGHTS_STABLE) != 0, dev, stream);
+            break;
+        case SWIGLU_ROUTE_STREAM_TC_BF16:
+            e = launch_stream_tc_bf16(X, Wg, Wu, H, m, k, n, ep,
+                                      (flags & SWIGLU_FLAG_WEIGHTS_STABLE) != 0, dev, stream);
             break;
         case SWIGLU_ROUTE_GEMM_BF16:
             e = launch_gemm_bf16(X, Wg, Wu, H, m, k, n, ep, dev, stream);
@@ -488,7 +495,7 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0, w6 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0, w6 = 0, w7 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
@@ -501,7 +508,9 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (e != cudaSuccess) return from_cuda(e);
     e = selftest_status_fetch_and_clear(&w6, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2 | w3 | w4 | w5 | w6) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = stream_tc_status_fetch_and_clear(&w7, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3 | w4 | w5 | w6 | w7) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
 }
 
 SWIGLU_API int swiglu_selftest_wait_timeout(cudaStream_t stream) {

@@ -51,6 +51,16 @@ cudaError_t launch_decode_bf16(const void *X, const void *Wg, const void *Wu, vo
                                int M, int K, int N, const Epilogue &epi, bool weights_stable,
                                const DeviceInfo &dev, cudaStream_t stream);
 
+// bf16 forward for 9 <= M <= kStreamTcMaxM: the weight stream on tcgen05
+// (X as the 128-row operand, 8 Wg + 8 Wu rows as the 16-row one).
+// stream_tc_bf16_supported: K a multiple of 64 and the X slices plus a
+// weight ring fit shared memory (a pure function of the shape).
+constexpr int kStreamTcMaxM = 128;
+bool stream_tc_bf16_supported(int M, int K, int N);
+cudaError_t launch_stream_tc_bf16(const void *X, const void *Wg, const void *Wu, void *H,
+                                  int M, int K, int N, const Epilogue &epi, bool weights_stable,
+                                  const DeviceInfo &dev, cudaStream_t stream);
+
 // Elementwise backward of h = act(alpha g) u; dtype 0 = bf16, 1 = fp32.
 cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG,
                            void *dU, int64_t n, int dtype, int activation, float alpha,
@@ -93,6 +103,7 @@ cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void 
 cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+cudaError_t stream_tc_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t selftest_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);

@@ -50,7 +50,7 @@ bool encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtyp
 
 bool encode_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, uint64_t d0,
                     uint64_t d1, uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
-                    uint32_t b0, uint32_t b1, uint32_t b2) {
+                    uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {d0, d1, d2};
@@ -58,7 +58,7 @@ bool encode_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtyp
     const cuuint32_t box[3] = {b0, b1, b2};
     const cuuint32_t elem_strides[3] = {1, 1, 1};
     const CUresult r = fn(map, dtype, 3, const_cast<void *>(base), dims, strides, box,
-                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;

@@ -17,9 +17,11 @@ bool encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtyp
                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // Encode a 3-D tensor: dims {d0, d1, d2} (d0 contiguous), byte strides of
-// dims 1 and 2, moved in boxes of {b0, b1, b2}, no swizzle.
+// dims 1 and 2 (in either order of size), moved in boxes of {b0, b1, b2};
+// the box lands in shared memory as [b2][b1][b0].
 bool encode_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
                     uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
-                    uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+                    uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 }  // namespace swiglu
