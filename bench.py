@@ -15,8 +15,10 @@ prefill at the LLaMA-3 8B shape and its variants (training forward storing
 G and U, GEGLU with a gate multiplier, fp8 output), the backward GEMMs (dX,
 dW, all three in one launch) and a whole training step of the projection
 (TFLOP/s), dSwiGLU on [8192, 14336] bf16 (GB/s), the fp32 3xTF32 forward and
-backward at the LLaMA-2 13B and GPT-NeoX 20B shapes, and the LLaMA-2 7B
-decode shape (GB/s), each with its roofline fraction and the SM clock seen.
+backward at the LLaMA-2 13B and GPT-NeoX 20B shapes, the LLaMA-2 7B
+decode shape, and batched decode at M in {16, 32, 64} on both decode shapes
+(the tcgen05 weight stream; GB/s), each with its roofline fraction and the
+SM clock seen.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and cuda synchronize, CUDA events on the launching stream, max over ranks.
@@ -56,6 +58,8 @@ PAGE_DECODE_GBS = 702.0
 DECODE_SHAPE = (1536, 6912)
 DECODE_MS = (1, 2, 4, 8)
 DECODE_COPIES = 16
+# batched decode: the tcgen05 weight-streaming route
+BATCHED_MS = (16, 32, 64)
 
 # DRAM traffic of the decode kernel per launch from one ncu capture, keyed by
 # the sha256 of the kernel source it was measured on; reported as null when
@@ -82,6 +86,11 @@ def decode_bytes(M, K, N, elem=2):
     """Algorithmic bytes of one fused call: both weight matrices once, X in,
     H out."""
     return elem * (2 * N * K + M * K + M * N)
+
+
+def up_route_for(M, K, N):
+    from up_projection_b200 import _capi
+    return _capi.swiglu_route_for(M, K, N, 0)
 
 
 def src_sha(name):
@@ -899,6 +908,27 @@ def main(argv=None):
                              "latency_single_call": {str(M): v for M, v in d7["latency"].items()},
                              "comparators_us": {k: round(v, 2) for k, v in
                                                 d7["comparators"]["us"].items()}})
+        # Batched decode (M = 16, 32, 64): the tcgen05 weight stream, same
+        # rotated cold copies, same comparators (at M = 64).
+        for (Kb, Nb, cb, name) in ((1536, 6912, 16, "AstrAI 1B"), (4096, 11008, 8, "LLaMA-2 7B")):
+            sb = max(48, min(1200, args.steps // 4)) // 3 * 3
+            db = run_decode(argparse.Namespace(steps=sb, warmup=6), 1, Kb, Nb, BATCHED_MS, cb,
+                            stream, with_e2e=False)
+            vb = db["step_bytes"] * sb / (db["ms"] * 1e-3) / 1e9
+            line["also"].append({
+                "workload": f"batched decode {name}: M in {{16,32,64}}, K={Kb}, N={Nb}, "
+                            f"{cb} rotated copies (tcgen05 weight stream)",
+                "metric": "GB/s", "value": round(vb, 1),
+                "route": up_route_for(BATCHED_MS[0], Kb, Nb),
+                "per_M": {str(M): {k: round(v, 2) for k, v in d.items()}
+                          for M, d in db["per_M"].items()},
+                "roofline": {"bound": "hbm", "achieved": round(vb, 1), "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(vb / pk["hbm_gbs"], 4)},
+                "read_floor_GB/s": round(db["floor"]["GB/s"], 1),
+                "frac_of_floor": round(vb / db["floor"]["GB/s"], 4),
+                "latency_single_call": {str(M): v for M, v in db["latency"].items()},
+                "comparators_us": {k: round(v, 2) for k, v in db["comparators"]["us"].items()},
+                "clocks": db["clocks"]})
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline_decode(K, N, DECODE_MS, gpu_H=dec["H"])
     if rank == 0:

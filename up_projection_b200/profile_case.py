@@ -1,6 +1,8 @@
 """Run one workload of the library a fixed number of times, for profilers.
 
     python -m up_projection_b200.profile_case decode  --M 8 --K 1536 --N 6912 --copies 4 --launches 3
+    python -m up_projection_b200.profile_case decode  --M 32 --K 4096 --N 11008 --copies 4 --launches 3
+        (9 <= M <= 128 with K a multiple of 64: the tcgen05 weight stream)
     python -m up_projection_b200.profile_case prefill --M 4096 --K 4096 --N 14336 --launches 3
     python -m up_projection_b200.profile_case dswiglu --n 117440512 --launches 3
     python -m up_projection_b200.profile_case fp32    --M 2048 --K 5120 --N 13824 --launches 2
