@@ -121,8 +121,10 @@ struct StreamPlan {
 };
 
 // Two CTAs per SM (half the shared memory and TMEM each) when the stages
-// still hold weight boxes of >= 8 KB in a ring of >= 3; else one CTA per SM
-// (more CTAs, in waves, where an SM's share would exceed 16 units).
+// still hold weight boxes of >= 4 KB in a ring of >= 3; else one CTA per SM
+// (more CTAs, in waves, where an SM's share would exceed 16 units).  (Swept
+// on B200: 8 KB instead of 4 KB costs 16 % at AstrAI-1B M = 64; no threshold
+// costs 4 % at M = 128; a ring of >= 4 costs up to 20 %.)
 inline StreamPlan stream_plan(int M, int K, int N, int sm_count) {
     StreamPlan p{};
     p.geo.ok = false;
@@ -139,7 +141,7 @@ inline StreamPlan stream_plan(int M, int K, int N, int sm_count) {
         const int q1 = (units + grid - 1) / grid;
         const int budget = cps == 2 ? 110 * 1024 : 220 * 1024;
         StreamGeo g = stream_geometry(M, K, q1, budget, 3);
-        if (cps == 2 && (!g.ok || g.wbytes < 8 * 1024)) continue;
+        if (cps == 2 && (!g.ok || g.wbytes < 4 * 1024)) continue;
         if (!g.ok) g = stream_geometry(M, K, q1, budget, 2);
         if (!g.ok) return p;
         g.ctas_per_sm = cps;
