@@ -101,6 +101,35 @@ def test_stream_tc_many_units_per_cta():
     assert_bf16_close(f64(H[im, inn]), ref, "stream many units")
 
 
+@pytest.mark.parametrize("layout", ["same", "halves", "halves_swapped", "far"])
+def test_stream_tc_weight_layouts(layout):
+    """The gate and up rows come through one 4-D view whose matrix stride is
+    the distance between the buffers (either order), or, for Wg == Wu,
+    through two 3-D views: same results in every layout."""
+    M, K, N = 24, 512, 1032
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=31)
+    if layout == "same":
+        Wu = Wg
+    both = torch.stack([Wg, Wu]).to(dev())
+    if layout == "same":
+        Wgd = Wud = both[0]
+    elif layout == "halves":
+        Wgd, Wud = both[0], both[1]
+    elif layout == "halves_swapped":
+        both = torch.stack([Wu, Wg]).to(dev())
+        Wgd, Wud = both[1], both[0]
+    else:  # separate allocations with a large buffer between them
+        Wgd = Wg.to(dev())
+        gap = torch.empty(64 << 20, dtype=torch.uint8, device=dev())
+        Wud = Wu.to(dev())
+        del gap
+    Xd = X.to(dev())
+    H = _capi.swiglu_fwd(Xd, Wgd, Wud)
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+    assert _capi.swiglu_last_route() == _capi.ROUTE_STREAM_TC_BF16
+    assert_bf16_close(f64(H), oracle.swiglu_fwd(X, Wg, Wu, "bf16")["H"], f"stream layout {layout}")
+
+
 def test_stream_tc_deterministic():
     X, Wg, Wu = synth.swiglu_inputs(32, 1536, 6912, "bf16", seed=4)
     a = run_fwd(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16)

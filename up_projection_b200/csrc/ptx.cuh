@@ -100,6 +100,15 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(const CUtensorMap *map, uint32_t bar, uint32_t dst,
+                                            int32_t x, int32_t y, int32_t z, int32_t w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+        : "memory");
+}
+
 // Non-tensor bulk copy global -> shared (this CTA); addresses 16-byte
 // aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,

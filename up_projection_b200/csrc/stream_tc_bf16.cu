@@ -16,13 +16,16 @@
 //
 // A CTA owns a contiguous, balanced range of cnt units of 8 output columns
 // (within one unit of even over the SMs): rows 8 u0 .. 8 (u0 + cnt) of each
-// weight matrix are consecutive, so per k-slice ONE tall TMA box per matrix
-// covers all of them (8 cnt rows x kc: 5-40 KB, few large copies), and the
-// X box of the slice rides in the same ring stage.  The boxes come from 3-D
-// views [k/64][rows][64] with the 128-byte swizzle and land as
-// [k-block][rows][128 B]: per k-block a run of 1024-byte swizzle atoms, the
-// K-major operand layout.  Per-CTA unit counts differ by at most one, so two
-// tensor maps per matrix (box heights 8 q and 8 (q + 1)) serve every CTA.
+// weight matrix are consecutive.  Per k-slice ONE TMA box covers them in both
+// matrices: a 4-D view [k/64][matrix][rows][64] whose matrix stride is the
+// distance between the two weight buffers lands as [k-block][Wg rows; Wu rows]
+// [128 B] -- per k-block one run of 1024-byte 128-byte-swizzle atoms, the
+// K-major operand layout -- so ONE MMA per k16 step computes gate and up
+// together (N = 16 cnt).  (Where that view does not exist -- Wg == Wu, or
+// buffers 1 TB apart -- two 3-D boxes and two MMAs per step do the same.)
+// The X box of the slice rides in the same ring stage.  Per-CTA unit counts
+// differ by at most one, so two tensor maps (box heights 8 q and 8 (q + 1))
+// serve every CTA.
 // The k16 steps alternate between two accumulator sets (no MMA waits on its
 // predecessor's accumulator); the epilogue sums them, forms
 // h = act(alpha g) u in fp32, rounds once to bf16 and stores 16 bytes per
@@ -166,13 +169,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// tm_w*_lo: box height 8 q (CTAs with q units), tm_w*_hi: 8 (q + 1).
+// tm_w*_lo: box height 8 q (CTAs with q units), tm_w*_hi: 8 (q + 1).  pair:
+// tm_wg_* are the 4-D views over both matrices (matrix 0 the lower address;
+// swapped: that is Wu) and tm_wu_* are unused.
 __global__ void __launch_bounds__(kThreads, 1)
     swiglu_stream_tc_bf16_kernel(const __grid_constant__ CUtensorMap tm_x,
                                  const __grid_constant__ CUtensorMap tm_wg_lo,
                                  const __grid_constant__ CUtensorMap tm_wu_lo,
                                  const __grid_constant__ CUtensorMap tm_wg_hi,
                                  const __grid_constant__ CUtensorMap tm_wu_hi, int q,
+                                 int pair, int swapped,
                                  __nv_bfloat16 *__restrict__ H, int M, int N, int weights_stable,
                                  int which_act, float alpha, __nv_bfloat16 *__restrict__ Gout,
                                  __nv_bfloat16 *__restrict__ Uout, const StreamGeo geo) {
@@ -185,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap *tm_wu = cnt > q ? &tm_wu_hi : &tm_wu_lo;
     if (threadIdx.x == 0) {
         tma_prefetch_desc(tm_wg);
-        tma_prefetch_desc(tm_wu);
+        if (!pair) tma_prefetch_desc(tm_wu);
         tma_prefetch_desc(&tm_x);
     }
     // Programmatic dependent launch: the next call may start prefetching its
@@ -254,8 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t fb = bar_full + 8 * stage;
                 const uint32_t st = sbase + stage * geo.stage;
                 mbar_arrive_expect_tx(fb, tx);
-                tma_load_3d(tm_wg, fb, st, 0, row, j * geo.kb);
-                tma_load_3d(tm_wu, fb, st + geo.wbytes, 0, row, j * geo.kb);
+                if (pair) {
+                    tma_load_4d(tm_wg, fb, st, 0, row, 0, j * geo.kb);
+                } else {
+                    tma_load_3d(tm_wg, fb, st, 0, row, j * geo.kb);
+                    tma_load_3d(tm_wu, fb, st + geo.wbytes, 0, row, j * geo.kb);
+                }
                 if (j >= deferred) issue_x(j);
                 ++issued;
                 if (++stage == geo.ring) {
@@ -281,11 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && cnt > 0) {
             // ------------------------------------------------- MMA issuer
-            // D regions (TMEM columns): g0 [0, R), u0 [R, 2R), g1, u1; k16
-            // steps alternate between set 0 and set 1.  For M = 128 the MMA's
-            // N is a multiple of 16: an odd cnt reads 8 rows past its box
-            // (columns that are never read).
-            const int n_mma = geo.mma_m == 128 ? (8 * cnt + 15) / 16 * 16 : 8 * cnt;
+            // D (TMEM columns): accumulator set p at [2pR, 2pR + 2R); k16
+            // steps alternate between set 0 and set 1.  pair: one MMA writes
+            // [matrix 0 | matrix 1] (N = 16 cnt).  Split: gate at [0, R), up
+            // at [R, 2R) of the set; for M = 128 the MMA's N is a multiple of
+            // 16, so an odd cnt reads 8 rows past its box (columns never read).
+            const int n_mma = pair ? 16 * cnt
+                                   : (geo.mma_m == 128 ? (8 * cnt + 15) / 16 * 16 : 8 * cnt);
             const uint32_t idesc = make_idesc(1u, static_cast<uint32_t>(geo.mma_m),
                                               static_cast<uint32_t>(n_mma));
             const uint32_t R = static_cast<uint32_t>(geo.region);
@@ -303,16 +315,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nbv = left < geo.kb ? left : geo.kb;
                 for (int b = 0; b < nbv; ++b) {
                     const uint64_t ad = sw128_kmajor_desc(xs + b * geo.mpad * 128);
-                    const uint64_t bg = sw128_kmajor_desc(st + b * cnt * 1024);
-                    const uint64_t bu = sw128_kmajor_desc(st + geo.wbytes + b * cnt * 1024);
                     const uint32_t acc = (j > 0 || b > 0) ? 1u : 0u;
+                    if (pair) {
+                        // block b: [matrix 0 rows; matrix 1 rows], 2 cnt atoms
+                        const uint64_t bw = sw128_kmajor_desc(st + b * cnt * 2048);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        // +32 bytes along k inside the swizzled row per k16
-                        const uint32_t set = static_cast<uint32_t>(kk & 1) * 2u * R;
-                        const uint32_t a = (kk < 2) ? acc : 1u;
-                        mma_f16(tmem_base + set, ad + 2u * kk, bg + 2u * kk, idesc, a);
-                        mma_f16(tmem_base + set + R, ad + 2u * kk, bu + 2u * kk, idesc, a);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            // +32 bytes along k inside the swizzled row per k16
+                            const uint32_t set = static_cast<uint32_t>(kk & 1) * 2u * R;
+                            mma_f16(tmem_base + set, ad + 2u * kk, bw + 2u * kk, idesc,
+                                    (kk < 2) ? acc : 1u);
+                        }
+                    } else {
+                        const uint64_t bg = sw128_kmajor_desc(st + b * cnt * 1024);
+                        const uint64_t bu = sw128_kmajor_desc(st + geo.wbytes + b * cnt * 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t set = static_cast<uint32_t>(kk & 1) * 2u * R;
+                            const uint32_t a = (kk < 2) ? acc : 1u;
+                            mma_f16(tmem_base + set, ad + 2u * kk, bg + 2u * kk, idesc, a);
+                            mma_f16(tmem_base + set + R, ad + 2u * kk, bu + 2u * kk, idesc, a);
+                        }
                     }
                 }
                 mma_commit(bar_empty + 8 * stage);
@@ -341,13 +364,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t R = static_cast<uint32_t>(geo.region);
                 const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+                // column offsets of gate and up within an accumulator set
+                const uint32_t c8 = static_cast<uint32_t>(8 * cnt);
+                const uint32_t goff = pair ? (swapped ? c8 : 0u) : 0u;
+                const uint32_t uoff = pair ? (swapped ? 0u : c8) : R;
                 for (int i = 0; i < cnt; ++i) {
                     const uint32_t col = tmem_base + row_off + static_cast<uint32_t>(8 * i);
                     uint32_t g0[8], u0[8], g1[8], u1[8];
-                    tmem_ld_32x32b_x8(col, g0);
-                    tmem_ld_32x32b_x8(col + R, u0);
-                    tmem_ld_32x32b_x8(col + 2 * R, g1);
-                    tmem_ld_32x32b_x8(col + 3 * R, u1);
+                    tmem_ld_32x32b_x8(col + goff, g0);
+                    tmem_ld_32x32b_x8(col + uoff, u0);
+                    tmem_ld_32x32b_x8(col + 2 * R + goff, g1);
+                    tmem_ld_32x32b_x8(col + 2 * R + uoff, u1);
                     tmem_ld_wait8(g0);
                     tmem_ld_wait8(u0);
                     tmem_ld_wait8(g1);
@@ -414,7 +441,10 @@ cudaError_t launch_stream_tc_bf16(const void *X, const void *Wg, const void *Wu,
     if (!geo.ok || plan.q < 1) return cudaErrorInvalidValue;
     // 3-D views [K/64 blocks][rows][64] (rows K*2 bytes apart, blocks 128 B
     // apart) with the 128-byte swizzle: a box {64, rows, kb} lands as
-    // [kb][rows][128 B].  Weight boxes are 8 q and 8 (q + 1) rows high.
+    // [kb][rows][128 B].  Weight boxes are 8 q and 8 (q + 1) rows high.  The
+    // pair view adds the matrix dimension (stride: the distance between the
+    // buffers, from the lower one): a box {64, rows, 2, kb} lands as
+    // [kb][2][rows][128 B].
     CUtensorMap tx, tg_lo, tu_lo, tg_hi, tu_hi;
     const uint64_t kblocks = static_cast<uint64_t>(geo.kblocks);
     const uint64_t row_bytes = 2ull * K;
@@ -424,11 +454,28 @@ cudaError_t launch_stream_tc_bf16(const void *X, const void *Wg, const void *Wu,
     const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!encode_tmap_3d(&tx, X, bf, 64, M, kblocks, row_bytes, 128, 64,
-                        static_cast<uint32_t>(geo.mpad), kb, sw) ||
-        !encode_tmap_3d(&tg_lo, Wg, bf, 64, N, kblocks, row_bytes, 128, 64, lo, kb, sw) ||
-        !encode_tmap_3d(&tu_lo, Wu, bf, 64, N, kblocks, row_bytes, 128, 64, lo, kb, sw) ||
-        !encode_tmap_3d(&tg_hi, Wg, bf, 64, N, kblocks, row_bytes, 128, 64, hi, kb, sw) ||
-        !encode_tmap_3d(&tu_hi, Wu, bf, 64, N, kblocks, row_bytes, 128, 64, hi, kb, sw)) {
+                        static_cast<uint32_t>(geo.mpad), kb, sw)) {
+        return cudaErrorInvalidValue;
+    }
+    const uintptr_t pg = reinterpret_cast<uintptr_t>(Wg), pu = reinterpret_cast<uintptr_t>(Wu);
+    const int swapped = pu < pg ? 1 : 0;
+    const uint64_t dist = swapped ? pg - pu : pu - pg;
+    const void *w0 = swapped ? Wu : Wg;
+    int pair = 0;
+    if (dist != 0 && dist % 16 == 0 && dist < (1ull << 40)) {
+        const uint64_t dims[4] = {64, static_cast<uint64_t>(N), 2, kblocks};
+        const uint64_t strides[3] = {row_bytes, dist, 128};
+        const uint32_t box_lo[4] = {64, lo, 2, kb}, box_hi[4] = {64, hi, 2, kb};
+        pair = encode_tmap_4d(&tg_lo, w0, bf, dims, strides, box_lo, sw) &&
+               encode_tmap_4d(&tg_hi, w0, bf, dims, strides, box_hi, sw);
+        tu_lo = tg_lo;
+        tu_hi = tg_hi;
+    }
+    if (!pair &&
+        (!encode_tmap_3d(&tg_lo, Wg, bf, 64, N, kblocks, row_bytes, 128, 64, lo, kb, sw) ||
+         !encode_tmap_3d(&tu_lo, Wu, bf, 64, N, kblocks, row_bytes, 128, 64, lo, kb, sw) ||
+         !encode_tmap_3d(&tg_hi, Wg, bf, 64, N, kblocks, row_bytes, 128, 64, hi, kb, sw) ||
+         !encode_tmap_3d(&tu_hi, Wu, bf, 64, N, kblocks, row_bytes, 128, 64, hi, kb, sw))) {
         return cudaErrorInvalidValue;
     }
     const unsigned bit = 1u << (dev.device & 31);
@@ -453,7 +500,8 @@ cudaError_t launch_stream_tc_bf16(const void *X, const void *Wg, const void *Wu,
     __nv_bfloat16 *up = static_cast<__nv_bfloat16 *>(epi.U);
     const int ws = weights_stable ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_stream_tc_bf16_kernel, tx, tg_lo, tu_lo, tg_hi,
-                                       tu_hi, plan.q, hp, M, N, ws, epi.activation,
+                                       tu_hi, plan.q, pair, pair ? swapped : 0, hp, M, N, ws,
+                                       epi.activation,
                                        epi.gate_multiplier, gp, up, geo);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

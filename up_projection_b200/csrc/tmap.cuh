@@ -24,4 +24,11 @@ bool encode_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtyp
                     uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
+// Encode a 4-D tensor (dims[0] contiguous; byte strides of dims 1..3 in any
+// order of size), moved in boxes `box`; the box lands as
+// [box[3]][box[2]][box[1]][box[0]].
+bool encode_tmap_4d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
+                    const uint64_t dims[4], const uint64_t strides_bytes[3],
+                    const uint32_t box[4], CUtensorMapSwizzle swizzle);
+
 }  // namespace swiglu
