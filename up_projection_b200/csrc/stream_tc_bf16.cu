@@ -59,7 +59,8 @@ constexpr int kThreads = 192;   // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epi
 constexpr int kMaxRing = 8;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kNumBars = 2 * kMaxRing + 2;  // full, empty, acc, drain
-constexpr int kTail = 8 * kNumBars + 64 + 1024;  // barriers, abort flag, TMEM slot, alignment
+// barriers, then abort flag (+0), TMEM slot (+16), epilogue flag (+32); alignment
+constexpr int kTail = 8 * kNumBars + 64 + 1024;
 
 struct StreamGeo {
     int mpad;      // X rows per box (M rounded up to 8)
@@ -74,6 +75,7 @@ struct StreamGeo {
     int stage;     // 2 wbytes + mpad * kb * 128
     int off_bar, smem;
     int tmem_cols;
+    int epi_units;  // units per epilogue chunk: mpad x 64 B each fit the ring
     int ctas_per_sm;
     bool ok;
 };
@@ -113,6 +115,9 @@ inline StreamGeo stream_geometry(int M, int K, int q1, int budget, int min_ring)
     int cols = 32;
     while (cols < 4 * g.region) cols *= 2;
     g.tmem_cols = cols;
+    g.epi_units = (g.ring * g.stage) / (g.mpad * 64);
+    if (g.epi_units > q1) g.epi_units = q1;
+    if (g.epi_units < 1) g.ok = false;
     if (g.smem > kMaxSmem || cols > 512) g.ok = false;
     return g;
 }
@@ -162,6 +167,11 @@ __device__ __forceinline__ void griddep_wait() {
 
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Barrier `id` (1..15) over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -352,23 +362,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue
-        const int quad = warp & 3;  // TMEM lane quadrant this warp may read
+        // M = 128 MMA (M > 64): every quadrant's warp holds 32 rows and
+        // forms h for them directly from TMEM, 16-byte stores per unit.
+        // M = 64 MMA: the warps holding D rows (16 per quadrant, a single
+        // warp at M <= 16) copy g and u (both accumulator sets summed) from
+        // TMEM to shared memory -- the ring, idle once every MMA has
+        // completed -- and then all 128 epilogue threads form the
+        // activations and store H, two columns each, so that serial
+        // activations in few lanes do not become the kernel's tail (B200,
+        // AstrAI-1B M = 16: 11.7 -> 10.2 us; at M = 128 the round trip
+        // costs more than it saves).  Units go through in chunks that fit
+        // the ring.
+        const int et = threadIdx.x - 64;  // 0..127
+        const int quad = warp & 3;        // TMEM lane quadrant this warp may read
         // D row m sits in lane m (M = 128 MMA), or for M = 64 in lanes 0..15
         // of each quadrant: row 16 quad + lane.
         const int rows_per_quad = geo.mma_m == 64 ? 16 : 32;
-        const int m = lane < rows_per_quad ? quad * rows_per_quad + lane : M;
-        if (quad * rows_per_quad < M && cnt > 0) {
-            if (!mbar_wait(bar_acc, 0, abort_flag)) {
-                failed = true;
-            } else {
-                tc_fence_after();
-                const uint32_t R = static_cast<uint32_t>(geo.region);
-                const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
-                // column offsets of gate and up within an accumulator set
-                const uint32_t c8 = static_cast<uint32_t>(8 * cnt);
-                const uint32_t goff = pair ? (swapped ? c8 : 0u) : 0u;
-                const uint32_t uoff = pair ? (swapped ? 0u : c8) : R;
-                for (int i = 0; i < cnt; ++i) {
+        const int m_lane = lane < rows_per_quad ? quad * rows_per_quad + lane : M;
+        volatile int *epi_ok =
+            reinterpret_cast<volatile int *>(gbase + geo.off_bar + 8 * kNumBars + 32);
+        if (warp == 2 && lane == 0) {
+            const bool ok = cnt > 0 && mbar_wait(bar_acc, 0, abort_flag);
+            if (cnt > 0 && !ok) failed = true;
+            *epi_ok = ok ? 1 : 0;
+        }
+        named_bar_sync(1, 128);
+        if (*epi_ok) {
+            tc_fence_after();
+            const uint32_t R = static_cast<uint32_t>(geo.region);
+            const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
+            // column offsets of gate and up within an accumulator set
+            const uint32_t c8 = static_cast<uint32_t>(8 * cnt);
+            const uint32_t goff = pair ? (swapped ? c8 : 0u) : 0u;
+            const uint32_t uoff = pair ? (swapped ? 0u : c8) : R;
+            float *E = reinterpret_cast<float *>(gbase);  // [m][unit][g 8, u 8]
+            if (geo.mma_m == 128) {
+                for (int i = 0; i < cnt && quad * rows_per_quad < M; ++i) {
                     const uint32_t col = tmem_base + row_off + static_cast<uint32_t>(8 * i);
                     uint32_t g0[8], u0[8], g1[8], u1[8];
                     tmem_ld_32x32b_x8(col + goff, g0);
@@ -379,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_wait8(u0);
                     tmem_ld_wait8(g1);
                     tmem_ld_wait8(u1);
-                    if (m < M) {
+                    if (m_lane < M) {
                         float g[8], u[8];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
@@ -395,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           act::gated<false>(which_act, alpha, g[5], u[5]));
                         h.w = pack_bf16x2(act::gated<false>(which_act, alpha, g[6], u[6]),
                                           act::gated<false>(which_act, alpha, g[7], u[7]));
-                        const size_t o = static_cast<size_t>(m) * N + 8 * (u_begin + i);
+                        const size_t o = static_cast<size_t>(m_lane) * N + 8 * (u_begin + i);
                         *reinterpret_cast<uint4 *>(H + o) = h;
                         if (Gout) {
                             *reinterpret_cast<uint4 *>(Gout + o) =
@@ -407,6 +436,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+            }
+            for (int i0 = 0; i0 < cnt && geo.mma_m == 64; i0 += geo.epi_units) {
+                const int uc = cnt - i0 < geo.epi_units ? cnt - i0 : geo.epi_units;
+                if (quad * rows_per_quad < M) {
+                    for (int ii = 0; ii < uc; ++ii) {
+                        const uint32_t col =
+                            tmem_base + row_off + static_cast<uint32_t>(8 * (i0 + ii));
+                        uint32_t g0[8], u0[8], g1[8], u1[8];
+                        tmem_ld_32x32b_x8(col + goff, g0);
+                        tmem_ld_32x32b_x8(col + uoff, u0);
+                        tmem_ld_32x32b_x8(col + 2 * R + goff, g1);
+                        tmem_ld_32x32b_x8(col + 2 * R + uoff, u1);
+                        tmem_ld_wait8(g0);
+                        tmem_ld_wait8(u0);
+                        tmem_ld_wait8(g1);
+                        tmem_ld_wait8(u1);
+                        if (m_lane < M) {
+                            float4 *e = reinterpret_cast<float4 *>(E + (m_lane * uc + ii) * 16);
+#pragma unroll
+                            for (int v = 0; v < 2; ++v) {
+                                e[v] = make_float4(
+                                    __uint_as_float(g0[4 * v]) + __uint_as_float(g1[4 * v]),
+                                    __uint_as_float(g0[4 * v + 1]) + __uint_as_float(g1[4 * v + 1]),
+                                    __uint_as_float(g0[4 * v + 2]) + __uint_as_float(g1[4 * v + 2]),
+                                    __uint_as_float(g0[4 * v + 3]) + __uint_as_float(g1[4 * v + 3]));
+                                e[2 + v] = make_float4(
+                                    __uint_as_float(u0[4 * v]) + __uint_as_float(u1[4 * v]),
+                                    __uint_as_float(u0[4 * v + 1]) + __uint_as_float(u1[4 * v + 1]),
+                                    __uint_as_float(u0[4 * v + 2]) + __uint_as_float(u1[4 * v + 2]),
+                                    __uint_as_float(u0[4 * v + 3]) + __uint_as_float(u1[4 * v + 3]));
+                            }
+                        }
+                    }
+                }
+                named_bar_sync(1, 128);
+                // (m, unit, column pair) items; consecutive items are
+                // consecutive columns of one row of H
+                const int items = M * uc * 4;
+                for (int it = et; it < items; it += 128) {
+                    const int m = it / (uc * 4);
+                    const int r = it - m * uc * 4;
+                    const int ii = r >> 2;
+                    const int c = (r & 3) * 2;
+                    const float2 g = *reinterpret_cast<const float2 *>(E + (m * uc + ii) * 16 + c);
+                    const float2 u =
+                        *reinterpret_cast<const float2 *>(E + (m * uc + ii) * 16 + 8 + c);
+                    const size_t o = static_cast<size_t>(m) * N + 8 * (u_begin + i0 + ii) + c;
+                    *reinterpret_cast<uint32_t *>(H + o) =
+                        pack_bf16x2(act::gated<false>(which_act, alpha, g.x, u.x),
+                                    act::gated<false>(which_act, alpha, g.y, u.y));
+                    if (Gout) {
+                        *reinterpret_cast<uint32_t *>(Gout + o) = pack_bf16x2(g.x, g.y);
+                        *reinterpret_cast<uint32_t *>(Uout + o) = pack_bf16x2(u.x, u.y);
+                    }
+                }
+                named_bar_sync(1, 128);  // E is rewritten by the next chunk
             }
         }
     }
