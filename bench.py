@@ -64,12 +64,13 @@ BATCHED_MS = (16, 32, 64)
 # DRAM traffic of the decode kernel per launch from one ncu capture, keyed by
 # the sha256 of the kernel source it was measured on; reported as null when
 # the source has changed since.
-DECODE_TRAFFIC = {"src_sha256": "ef1daca510de86805982f295a069effd2229c6179030b1411c747e85d8d7cee8",
+DECODE_TRAFFIC = {"src_sha256": "952211d94952fc45bf09e8e59fc464fdd5a4f911d2ca79c76429eba5a12347f6",
                   # one ncu capture of this kernel at M = 8 (AstrAI-1B shape,
-                  # weights-stable launch); X and H add < 0.3 % per M, so it
-                  # stands for every M.
-                  "bytes_per_launch_by_M": {"1": 42523136, "2": 42523136, "4": 42523136,
-                                            "8": 42523136}}
+                  # weights-stable launch): dram__bytes_read.sum 42523648,
+                  # dram__bytes_write.sum 0 (H stays in L2 within the launch);
+                  # X and H add < 0.3 % per M, so it stands for every M.
+                  "bytes_per_launch_by_M": {"1": 42523648, "2": 42523648, "4": 42523648,
+                                            "8": 42523648}}
 
 
 def peaks():

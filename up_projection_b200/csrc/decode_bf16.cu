@@ -339,7 +339,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             mine[3] = d[3];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_red_full);
-            if (cw == 0) {
+            // The unit's reduction and epilogue rotate over the consumer
+            // warps, so that no warp falls an epilogue behind per unit (the
+            // stages are released only when all four have read them).  The
+            // sum runs over the warps in the same fixed order whichever warp
+            // forms it.
+            if (cw == (u - u_begin) % kConsumerWarps) {
                 if (!mbar_wait(bar_red_full, par, abort_flag)) {
                     failed = true;
                     break;
