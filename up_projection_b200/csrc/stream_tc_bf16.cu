@@ -243,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0 && cnt > 0) {
             // ------------------------------------------------ TMA producer
-            // stage: [Wg box 8 cnt x kc][Wu box][X box mpad x kc]
+            // stage: [weights: pair box [kb][2][8 cnt][64], or Wg box then
+            //         Wu box (wbytes apart)][X box [kb][mpad][64]]
             const uint32_t tx = static_cast<uint32_t>(geo.kb * 128 * (16 * cnt + geo.mpad));
             const int row = 8 * u_begin;
             auto issue_x = [&](int j) {
