@@ -150,7 +150,8 @@ def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
     does), Wg/Wu [N, K]; bf16 or fp32, all contiguous on one GPU.
 
     weights_stable=True promises that no earlier work on the stream writes
-    Wg or Wu (SWIGLU_FLAG_WEIGHTS_STABLE): the decode kernel may then start
+    Wg or Wu (SWIGLU_FLAG_WEIGHTS_STABLE): the weight-streaming kernels (bf16
+    decode at M <= 8, the tcgen05 stream at 9 <= M <= 128) may then start
     streaming them while the preceding kernel finishes.
 
     activation / gate_multiplier select the epilogue variant
