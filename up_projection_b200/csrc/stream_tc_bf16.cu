@@ -58,7 +58,7 @@ using gemm::mbar_wait_drain;
 constexpr int kThreads = 192;   // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
 constexpr int kMaxRing = 8;
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kNumBars = 2 * kMaxRing + 2;  // full, empty, acc, drain
+constexpr int kNumBars = 2 * kMaxRing + 3;  // full, empty, acc, drain[2]
 // barriers, then abort flag (+0), TMEM slot (+16), epilogue flag (+32); alignment
 constexpr int kTail = 8 * kNumBars + 64 + 1024;
 
@@ -223,10 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < geo.ring; ++s) {
             mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 2);  // one commit per MMA issuer
         }
-        mbar_init(bar_acc, 1);
+        mbar_init(bar_acc, 2);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_drain + 8, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -240,6 +241,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
     bool failed = false;
+    // ----------------------------------------------------- MMA issuers
+    // D (TMEM columns): accumulator set p at [2pR, 2pR + 2R); set p takes the
+    // k16 steps kk = p, p + 2 of every k-block and is issued by its own
+    // thread (warp 1 lane 0: set 0; warp 2 lane 0: set 1), so that two
+    // threads keep the tensor pipe fed.  pair: one MMA writes [matrix 0 |
+    // matrix 1] (N = 16 cnt).  Split: gate at [0, R), up at [R, 2R) of the
+    // set; for M = 128 the MMA's N is a multiple of 16, so an odd cnt reads 8
+    // rows past its box (columns never read).  Each issuer commits to the
+    // stage's empty barrier (two arrivals free it) and to the accumulator
+    // barrier (two arrivals), and drains its own MMAs before TMEM is freed.
+    auto run_mma = [&](int p) {
+        const int n_mma = pair ? 16 * cnt
+                               : (geo.mma_m == 128 ? (8 * cnt + 15) / 16 * 16 : 8 * cnt);
+        const uint32_t idesc = make_idesc(1u, static_cast<uint32_t>(geo.mma_m),
+                                          static_cast<uint32_t>(n_mma));
+        const uint32_t R = static_cast<uint32_t>(geo.region);
+        const uint32_t d = tmem_base + static_cast<uint32_t>(p) * 2u * R;
+        const uint32_t drain = bar_drain + 8 * p;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int j = 0; j < geo.slices && !failed; ++j) {
+            if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t st = sbase + stage * geo.stage;
+            const uint32_t xs = st + 2 * geo.wbytes;
+            const int left = geo.kblocks - j * geo.kb;
+            const int nbv = left < geo.kb ? left : geo.kb;
+            for (int b = 0; b < nbv; ++b) {
+                const uint64_t ad = sw128_kmajor_desc(xs + b * geo.mpad * 128);
+                const uint32_t acc = (j > 0 || b > 0) ? 1u : 0u;
+                if (pair) {
+                    // block b: [matrix 0 rows; matrix 1 rows], 2 cnt atoms
+                    const uint64_t bw = sw128_kmajor_desc(st + b * cnt * 2048);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        // +32 bytes along k inside the swizzled row per k16
+                        const uint32_t kk = static_cast<uint32_t>(p + 2 * h);
+                        mma_f16(d, ad + 2u * kk, bw + 2u * kk, idesc, h == 0 ? acc : 1u);
+                    }
+                } else {
+                    const uint64_t bg = sw128_kmajor_desc(st + b * cnt * 1024);
+                    const uint64_t bu = sw128_kmajor_desc(st + geo.wbytes + b * cnt * 1024);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t kk = static_cast<uint32_t>(p + 2 * h);
+                        const uint32_t a = h == 0 ? acc : 1u;
+                        mma_f16(d, ad + 2u * kk, bg + 2u * kk, idesc, a);
+                        mma_f16(d + R, ad + 2u * kk, bu + 2u * kk, idesc, a);
+                    }
+                }
+            }
+            mma_commit(bar_empty + 8 * stage);
+            if (++stage == geo.ring) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (failed) *abort_flag = 1;
+        else mma_commit(bar_acc);
+        // Every MMA issued here must finish before TMEM is released.
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+    };
     if (warp == 0) {
         if (lane == 0 && cnt > 0) {
             // ------------------------------------------------ TMA producer
@@ -300,67 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && cnt > 0) {
-            // ------------------------------------------------- MMA issuer
-            // D (TMEM columns): accumulator set p at [2pR, 2pR + 2R); k16
-            // steps alternate between set 0 and set 1.  pair: one MMA writes
-            // [matrix 0 | matrix 1] (N = 16 cnt).  Split: gate at [0, R), up
-            // at [R, 2R) of the set; for M = 128 the MMA's N is a multiple of
-            // 16, so an odd cnt reads 8 rows past its box (columns never read).
-            const int n_mma = pair ? 16 * cnt
-                                   : (geo.mma_m == 128 ? (8 * cnt + 15) / 16 * 16 : 8 * cnt);
-            const uint32_t idesc = make_idesc(1u, static_cast<uint32_t>(geo.mma_m),
-                                              static_cast<uint32_t>(n_mma));
-            const uint32_t R = static_cast<uint32_t>(geo.region);
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int j = 0; j < geo.slices && !failed; ++j) {
-                if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
-                    failed = true;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t st = sbase + stage * geo.stage;
-                const uint32_t xs = st + 2 * geo.wbytes;
-                const int left = geo.kblocks - j * geo.kb;
-                const int nbv = left < geo.kb ? left : geo.kb;
-                for (int b = 0; b < nbv; ++b) {
-                    const uint64_t ad = sw128_kmajor_desc(xs + b * geo.mpad * 128);
-                    const uint32_t acc = (j > 0 || b > 0) ? 1u : 0u;
-                    if (pair) {
-                        // block b: [matrix 0 rows; matrix 1 rows], 2 cnt atoms
-                        const uint64_t bw = sw128_kmajor_desc(st + b * cnt * 2048);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            // +32 bytes along k inside the swizzled row per k16
-                            const uint32_t set = static_cast<uint32_t>(kk & 1) * 2u * R;
-                            mma_f16(tmem_base + set, ad + 2u * kk, bw + 2u * kk, idesc,
-                                    (kk < 2) ? acc : 1u);
-                        }
-                    } else {
-                        const uint64_t bg = sw128_kmajor_desc(st + b * cnt * 1024);
-                        const uint64_t bu = sw128_kmajor_desc(st + geo.wbytes + b * cnt * 1024);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t set = static_cast<uint32_t>(kk & 1) * 2u * R;
-                            const uint32_t a = (kk < 2) ? acc : 1u;
-                            mma_f16(tmem_base + set, ad + 2u * kk, bg + 2u * kk, idesc, a);
-                            mma_f16(tmem_base + set + R, ad + 2u * kk, bu + 2u * kk, idesc, a);
-                        }
-                    }
-                }
-                mma_commit(bar_empty + 8 * stage);
-                if (++stage == geo.ring) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (failed) *abort_flag = 1;
-            else mma_commit(bar_acc);
-            // Every MMA issued here must finish before TMEM is released.
-            mma_commit(bar_drain);
-            mbar_wait_drain(bar_drain, 0);
-        }
+        if (lane == 0 && cnt > 0) run_mma(0);
     } else {
         // ------------------------------------------------------- epilogue
         // M = 128 MMA (M > 64): every quadrant's warp holds 32 rows and
@@ -382,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int m_lane = lane < rows_per_quad ? quad * rows_per_quad + lane : M;
         volatile int *epi_ok =
             reinterpret_cast<volatile int *>(gbase + geo.off_bar + 8 * kNumBars + 32);
+        if (warp == 2 && lane == 0 && cnt > 0) run_mma(1);
         if (warp == 2 && lane == 0) {
-            const bool ok = cnt > 0 && mbar_wait(bar_acc, 0, abort_flag);
+            const bool ok = cnt > 0 && !failed && mbar_wait(bar_acc, 0, abort_flag);
             if (cnt > 0 && !ok) failed = true;
             *epi_ok = ok ? 1 : 0;
         }
