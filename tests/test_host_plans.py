@@ -1,4 +1,6 @@
-"""Launch plans of the batched-decode stream kernel, checked on the host.
+"""Launch plans and schedules of the kernels, checked on the host.
+
+Launch plans of the batched-decode stream kernel:
 
 `stream_plan_check.cu` includes the kernel's translation unit (the kernel is
 compiled, never launched) and runs its planning code for every routed shape
@@ -23,19 +25,30 @@ def _nvcc():
     return None
 
 
-def test_stream_plans_keep_memory_bounds():
+def _build_and_run(sources, min_checked):
     nvcc = _nvcc()
     if nvcc is None:
         pytest.skip("nvcc not available")
     with tempfile.TemporaryDirectory() as d:
-        exe = os.path.join(d, "stream_plan_check")
+        exe = os.path.join(d, "check")
         cmd = [nvcc, "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a",
                "-I" + os.path.join(ROOT, "include"),
                "-I" + os.path.join(ROOT, "up_projection_b200", "csrc"),
-               os.path.join(ROOT, "tests", "stream_plan_check.cu"),
-               os.path.join(ROOT, "up_projection_b200", "csrc", "tmap.cu"), "-o", exe]
+               *[os.path.join(ROOT, s) for s in sources], "-o", exe]
         p = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
         assert p.returncode == 0, p.stdout + p.stderr
         r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
         assert r.returncode == 0 and r.stdout.startswith("ok"), r.stdout + r.stderr
-        assert int(r.stdout.split()[1]) > 100000
+        assert int(r.stdout.split()[1]) >= min_checked
+
+
+def test_stream_plans_keep_memory_bounds():
+    _build_and_run(["tests/stream_plan_check.cu", "up_projection_b200/csrc/tmap.cu"], 100000)
+
+
+def test_backward_schedule_is_an_exact_partition():
+    """The backward GEMMs' static schedule (dX tiles round-robin, then dW
+    tiles in the order the CTAs free up) covers every dX and dW tile exactly
+    once, dX before dW within each CTA, for tile counts, grids and cost
+    ratios including the edge cases (bwd_sched_check.cu)."""
+    _build_and_run(["tests/bwd_sched_check.cu"], 8000)

@@ -67,7 +67,8 @@ inline BwdSched make_bwd_sched(int T_dx, int T_dw, int G, long long c_dx, long l
 enum : int { kTileDx = 0, kTileDw = 1 };
 
 // The seq-th tile of CTA `cta` of G: returns false once the CTA is done.
-__device__ __forceinline__ bool bwd_tile_of(const BwdSched &s, int cta, int G, int seq,
+// (Host-callable too, so that the partition can be checked without a GPU.)
+__host__ __device__ __forceinline__ bool bwd_tile_of(const BwdSched &s, int cta, int G, int seq,
                                             int &kind, int &t) {
     const int ndx = s.q + (cta < s.r ? 1 : 0);
     if (seq < ndx) {
