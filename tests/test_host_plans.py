@@ -1,4 +1,6 @@
-"""Launch plans and schedules of the kernels, checked on the host.
+"""Launch plans, geometries and schedules of the kernels, checked on the host
+(each checker includes the kernel's translation unit and calls its own
+planning code; nothing is launched).
 
 Launch plans of the batched-decode stream kernel:
 
@@ -52,3 +54,11 @@ def test_backward_schedule_is_an_exact_partition():
     once, dX before dW within each CTA, for tile counts, grids and cost
     ratios including the edge cases (bwd_sched_check.cu)."""
     _build_and_run(["tests/bwd_sched_check.cu"], 8000)
+
+
+def test_decode_geometry_for_every_supported_k():
+    """Decode kernel: for every K it accepts, both launch forms and M <= 8,
+    the shared-memory layout fits (two CTAs per SM on the small budget), the
+    TMA boxes and regions are legal and aligned, and the transaction counts
+    stay below the mbarrier limit (decode_geometry_check.cu)."""
+    _build_and_run(["tests/decode_geometry_check.cu", "up_projection_b200/csrc/tmap.cu"], 20000)
