@@ -26,12 +26,14 @@
 // The X box of the slice rides in the same ring stage.  Per-CTA unit counts
 // differ by at most one, so two tensor maps (box heights 8 q and 8 (q + 1))
 // serve every CTA.
-// The k16 steps alternate between two accumulator sets (no MMA waits on its
-// predecessor's accumulator); the epilogue sums them, forms
-// h = act(alpha g) u in fp32, rounds once to bf16 and stores 16 bytes per
-// unit and row.  Where a CTA's stages are small enough two CTAs share an SM,
-// so that one's tail overlaps the other's stream (and, with
-// weights_stable, the next call's weight prefetch).
+// The k16 steps alternate between two accumulator sets, each issued by its
+// own thread (no MMA waits on its predecessor's accumulator, and two threads
+// keep the tensor pipe fed); the epilogue sums them, forms
+// h = act(alpha g) u in fp32 and rounds once to bf16 -- spread over all 128
+// epilogue threads through shared memory when few warps hold the rows.
+// Where a CTA's stages are small enough two CTAs share an SM, so that one's
+// tail overlaps the other's stream (and, with weights_stable, the next
+// call's weight prefetch).
 //
 // Waits are bounded; a stuck pipeline sets the status word, the MMAs and
 // copies in flight are drained and TMEM is freed before the kernel returns.
