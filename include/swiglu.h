@@ -120,8 +120,8 @@ enum swiglu_route {
     SWIGLU_ROUTE_BWD_GEMM_TF32X3 = 6, /* fp32 backward GEMM, 3xTF32         */
     SWIGLU_ROUTE_STREAM_TC_BF16 = 7 /* bf16, 9 <= M <= 128, K a multiple of
                                      64: weight streaming on tcgen05 (X the
-                                     128-row operand, 8 gate + 8 up weight
-                                     rows the 16-row one)                   */
+                                     MMA's M operand, each CTA's gate and up
+                                     weight rows its N operand)             */
 };
 
 /*
