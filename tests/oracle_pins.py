@@ -28,6 +28,12 @@ What pins what:
                         U = Wu[:, k] exactly.
   fwd_asymptotes        G = +40 => H ~ 40 U, G = -40 => H ~ 0.
   fwd_points            the sampled forward equals the full forward.
+  fwd_nonfinite         NaN and +-Inf in X, Wg, Wu: silu(+Inf) = +Inf,
+                        silu(-Inf) and silu(NaN) are NaN as torch's silu gives
+                        them in float64 (an independent library routine); G, U
+                        against a brute-force loop of Python float products;
+                        H against torch's silu(G) * U, class by class (NaN,
+                        +-Inf, finite) and value by value.
   bf16_decoder          all 65536 bf16 patterns decode like torch's bf16.
   dswiglu_finite_diff   dG, dU against central differences of the forward.
   dswiglu_special       dh = 0, u = 0, g = 0, g = +-40, g = x*.
@@ -239,6 +245,61 @@ def fwd_points(o):
         Wgd = Wg.to(torch.float64).numpy()
         G_np = np.einsum("ik,ik->i", Xd[im], Wgd[inn])
         assert np.all(np.abs(pts["G"] - G_np) <= 1e-13 * pts["AG"] + 1e-300)
+
+
+def _same_ieee(a, b, rtol=0.0):
+    """a and b agree element by element: NaN where the other is NaN, the same
+    signed infinity, and finite values within rtol (relative)."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    na, nb = np.isnan(a), np.isnan(b)
+    if not np.array_equal(na, nb):
+        return False
+    ia, ib = np.isinf(a), np.isinf(b)
+    if not np.array_equal(ia, ib) or not np.array_equal(a[ia], b[ib]):
+        return False
+    f = ~(na | ia)
+    return bool(np.all(np.abs(a[f] - b[f]) <= rtol * np.abs(b[f])))
+
+
+def fwd_nonfinite(o):
+    inf, nan = math.inf, math.nan
+    # closed forms, and torch's float64 silu at the same points
+    assert o.silu(inf) == inf and math.isnan(o.silu(-inf)) and math.isnan(o.silu(nan))
+    pts = torch.tensor([inf, -inf, nan, -90.0, 0.0, 90.0], dtype=torch.float64)
+    theirs = torch.nn.functional.silu(pts).numpy()
+    ours = np.array([o.silu(float(v)) for v in pts])
+    assert _same_ieee(ours, theirs, rtol=1e-15)
+    # a small problem with non-finite operands planted in rows of each input
+    M, K, N = 5, 9, 7
+    X, Wg, Wu = _random_problem(M, K, N, 90)
+    X[1, 2] = nan
+    X[2, 4] = inf
+    X[3, 0] = -inf
+    Wg[2, 5] = nan
+    Wg[4, 1] = inf
+    Wu[5, 7] = -inf
+    Wu[6, 3] = nan
+    Wg[0, 4] = 0.0          # X[2, 4] * Wg[0, 4] = Inf * 0 = NaN
+    out = o.swiglu_fwd_f64(X, Wg, Wu)
+    G = np.empty((M, N))
+    U = np.empty((M, N))
+    for m in range(M):
+        for n in range(N):
+            g = 0.0
+            u = 0.0
+            for k in range(K):
+                g += float(X[m, k]) * float(Wg[n, k])
+                u += float(X[m, k]) * float(Wu[n, k])
+            G[m, n] = g
+            U[m, n] = u
+    assert _same_ieee(out["G"], G, rtol=1e-13) and _same_ieee(out["U"], U, rtol=1e-13)
+    H = (torch.nn.functional.silu(torch.from_numpy(G)) * torch.from_numpy(U)).numpy()
+    assert _same_ieee(out["H"], H, rtol=1e-13)
+    # every class occurs, so the comparison above is not vacuous
+    assert np.isnan(out["H"]).any() and np.isposinf(out["H"]).any()
+    assert np.isneginf(out["H"]).any() and np.isfinite(out["H"]).any()
+    assert np.isnan(out["H"][1]).all() and np.isnan(out["H"][:, 2]).all()
 
 
 def bf16_decoder(o):
@@ -495,7 +556,7 @@ def quant_blocks(o):
 
 ALL_PINS = [scalar_closed_forms, fwd_library, fwd_brute_force,
             fwd_gate_up_roles, fwd_zero_cases, fwd_linear_in_up, fwd_one_hot,
-            fwd_asymptotes, fwd_points, bf16_decoder, dswiglu_finite_diff,
+            fwd_asymptotes, fwd_points, fwd_nonfinite, bf16_decoder, dswiglu_finite_diff,
             dswiglu_special, dswiglu_storage, gelu_closed_forms, variants_fwd,
             variants_bwd, backward_gemms, gelu_high_precision, e4m3_codec, ue8m0_scale,
             quant_blocks]
