@@ -806,6 +806,43 @@ def reference_arm(args, metric, config, K, N, budget_s=120.0):
     return 0
 
 
+def summary_of(line):
+    """Compact record of the line: value and roofline fraction per workload
+    (decode GB/s, prefill and backward TFLOP/s, dSwiGLU GB/s, fp32 TFLOP/s),
+    taken from the headline and the "also" entries."""
+    out = {"decode_astrai_gbs": line["value"], "decode_astrai_frac": line["roofline"]["frac"],
+           "decode_astrai_us_per_call": round(line["ms_per_step"] * 1e3 / len(DECODE_MS), 3),
+           "e2e_gbs": line["e2e"]["value"]}
+    keys = [("prefill LLaMA-3 8B", "prefill"),
+            ("prefill training forward", "prefill_training_fwd"),
+            ("prefill GEGLU", "prefill_geglu"),
+            ("prefill, fp8", "prefill_fp8_out"),
+            ("backward dX = ", "bwd_dx"),
+            ("backward dWg", "bwd_dw"),
+            ("backward dX, dWg, dWu in one launch", "bwd_gemms"),
+            ("training step", "training_step"),
+            ("dSwiGLU", "dswiglu"),
+            ("fp32 3xTF32 LLaMA-2 13B", "fp32_13b"),
+            ("fp32 3xTF32 GPT-NeoX 20B", "fp32_neox"),
+            ("fp32 3xTF32 backward dX = ", "fp32_13b_bwd_dx"),
+            ("fp32 3xTF32 backward dX, dWg, dWu in one launch", "fp32_13b_bwd_gemms"),
+            ("decode LLaMA-2 7B", "decode_llama7b"),
+            ("batched decode AstrAI", "batched_astrai"),
+            ("batched decode LLaMA-2 7B", "batched_llama7b")]
+    for entry in line.get("also", []):
+        w = entry.get("workload", "")
+        for prefix, key in keys:
+            if w.startswith(prefix) and key + "_value" not in out:
+                if "value" in entry:
+                    out[key + "_value"] = entry["value"]
+                    out[key + "_unit"] = entry.get("metric")
+                    out[key + "_frac"] = entry.get("roofline", {}).get("frac")
+                break
+    if "cpu_baseline" in line:
+        out["cpu_oracle_gbs"] = line["cpu_baseline"]["value"]
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -933,6 +970,9 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline_decode(K, N, DECODE_MS, gpu_H=dec["H"])
     if rank == 0:
+        # last key of the line: the headline figures of every workload in one
+        # short object, so that a reader of the line's tail has all of them
+        line["summary"] = summary_of(line)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -141,6 +141,10 @@ enum swiglu_route {
  *  one round-to-nearest-even to bf16; NaN/Inf propagate (no saturation).
  *  fp32: each operand is split a = hi + lo (hi, lo TF32), and the three
  *  products hi*hi + hi*lo + lo*hi are accumulated in fp32 on tensor cores.
+ *  The split turns an infinite operand into NaN terms (Inf - Inf, Inf * 0),
+ *  so a second, light kernel scans H and re-evaluates each NaN or infinite
+ *  output in plain fp32 arithmetic: NaN and +-Inf operands give the IEEE
+ *  classes of the definition, as for bf16 (finite outputs are untouched).
  *  The route (swiglu_route_for) is a pure function of M, K, N and dtype.
  *  No call allocates device memory.
  */
@@ -240,7 +244,8 @@ SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U
  *
  *  Both products accumulate in ONE fp32 accumulator (tcgen05, TMEM); bf16:
  *  dX is rounded once to bf16 (RNE); fp32: 3xTF32 products accumulated in
- *  256-deep chunks folded with round-to-nearest adds, as swiglu_fwd's fp32.  M == 0 or K == 0: nothing enqueued.  N == 0:
+ *  256-deep chunks folded with round-to-nearest adds, as swiglu_fwd's fp32,
+ *  and (as there) NaN or infinite outputs re-evaluated in plain fp32.  M == 0 or K == 0: nothing enqueued.  N == 0:
  *  dX is set to +0.  dX must not overlap an input (SWIGLU_ERR_OVERLAP).
  *  Allocates no device memory.
  */
@@ -261,7 +266,8 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
  *  SWIGLU_BF16 or SWIGLU_FP32.
  *
  *  fp32 accumulation over all M rows in TMEM (fp32: 3xTF32, chunked as in
- *  swiglu_bwd_dx), one rounding per output.
+ *  swiglu_bwd_dx, non-finite outputs re-evaluated as there), one rounding
+ *  per output.
  *  N == 0 or K == 0: nothing enqueued.  M == 0: dWg and dWu are set to +0.
  *  Outputs must not overlap each other or an input (SWIGLU_ERR_OVERLAP).
  *  Allocates no device memory.
@@ -289,10 +295,12 @@ SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg,
  * swiglu_route, or -1 for arguments swiglu_fwd would reject). */
 SWIGLU_API int swiglu_route_for(int64_t M, int64_t K, int64_t N, int dtype);
 
-/* Route of the last swiglu_fwd* or swiglu_bwd_dx/_dw call on this host
- * thread that returned SWIGLU_OK (SWIGLU_ROUTE_NONE before the first; an
- * empty reduction reports SWIGLU_ROUTE_ZERO_K).  Lets tests assert that
- * the fused kernel actually ran. */
+/* Route of the last swiglu_fwd* or swiglu_bwd_dx/_dw/_gemms call on this
+ * host thread that returned SWIGLU_OK (SWIGLU_ROUTE_NONE before the first;
+ * an empty reduction reports SWIGLU_ROUTE_ZERO_K).  Lets tests assert that
+ * the fused kernel actually ran.  Kept per host thread (not per stream):
+ * calls from other threads never change it, and it names the route chosen
+ * on the host, not a kernel's completion. */
 SWIGLU_API int swiglu_last_route(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -303,6 +311,16 @@ SWIGLU_API const char *swiglu_status_string(int status);
  * current device.  Returns SWIGLU_ERR_TIMEOUT if any kernel's bounded wait
  * gave up since the last call, SWIGLU_ERR_CUDA if the stream reports an
  * error, else SWIGLU_OK.
+ *
+ * The status words are per device and shared by every stream and host
+ * thread of the process (one word per kernel family, set with an atomic OR,
+ * never cleared by the kernels).  So a timeout is reported to whichever
+ * swiglu_sync_status call reads the word first, whatever stream the failing
+ * kernel ran on; with work on several streams, synchronise all of them (or
+ * the device) before relying on which call failed.  Reading and clearing is
+ * not atomic with respect to kernels still running on other streams: a wait
+ * that gives up while this call runs may be reported by this call or by the
+ * next one, never lost.
  */
 SWIGLU_API int swiglu_sync_status(cudaStream_t stream);
 

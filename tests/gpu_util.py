@@ -76,3 +76,47 @@ def assert_guards_intact(full: torch.Tensor, fill: float = 1234.5):
     g0 = full[:GUARD]
     g1 = full[-GUARD:]
     assert bool((g0 == fill).all()) and bool((g1 == fill).all()), "output guard overwritten"
+
+
+# Smallest magnitudes that round to infinity (round-to-nearest-even, no
+# saturation): the midpoint between the largest finite value and 2^128.
+BF16_OVERFLOW = 2.0 ** 128 - 2.0 ** 119
+FP32_OVERFLOW = 2.0 ** 128 - 2.0 ** 103
+
+
+def assert_ieee_close(gpu, ref, what: str, dtype: str = "bf16", bound=None):
+    """Outputs that may hold NaN and infinities, against the fp64 reference:
+    NaN exactly where the reference is NaN; the same signed infinity where the
+    reference is infinite or rounds to infinity in the output type; finite
+    elsewhere and within the tolerance (bf16: 1e-2 |ref| + 1e-3; fp32: the
+    per-element `bound`).  Returns the count of each class."""
+    gpu = np.asarray(gpu, dtype=np.float64).ravel()
+    ref = np.asarray(ref, dtype=np.float64).ravel()
+    assert gpu.shape == ref.shape
+    over = BF16_OVERFLOW if dtype == "bf16" else FP32_OVERFLOW
+    nan_r = np.isnan(ref)
+    inf_r = ~nan_r & (np.abs(ref) >= over)
+    fin_r = ~(nan_r | inf_r)
+    bad = np.isnan(gpu) != nan_r
+    if bad.any():
+        i = np.flatnonzero(bad)[:5]
+        raise AssertionError(f"{what}: NaN positions differ ({int(bad.sum())}); first at "
+                             f"{i.tolist()}: gpu={gpu[i].tolist()} ref={ref[i].tolist()}")
+    want_inf = np.where(ref > 0, np.inf, -np.inf)
+    bad = inf_r & (gpu != want_inf)
+    if bad.any():
+        i = np.flatnonzero(bad)[:5]
+        raise AssertionError(f"{what}: {int(bad.sum())} infinities differ; first at "
+                             f"{i.tolist()}: gpu={gpu[i].tolist()} ref={ref[i].tolist()}")
+    bad = fin_r & ~np.isfinite(gpu)
+    if bad.any():
+        i = np.flatnonzero(bad)[:5]
+        raise AssertionError(f"{what}: {int(bad.sum())} non-finite where the reference is "
+                             f"finite; first at {i.tolist()}: gpu={gpu[i].tolist()} "
+                             f"ref={ref[i].tolist()}")
+    if dtype == "bf16":
+        assert_bf16_close(gpu[fin_r], ref[fin_r], what)
+    else:
+        b = np.asarray(bound, dtype=np.float64).ravel()[fin_r]
+        assert_within(np.abs(gpu[fin_r] - ref[fin_r]), b, what)
+    return {"nan": int(nan_r.sum()), "inf": int(inf_r.sum()), "finite": int(fin_r.sum())}

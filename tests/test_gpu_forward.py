@@ -336,3 +336,96 @@ def _random_stream_shapes(seed, count):
 def test_stream_tc_random_shapes(M, K, N):
     X, Wg, Wu = synth.swiglu_inputs(M, K, N, "bf16", seed=M * 13 + K * 7 + N)
     check_full(X, Wg, Wu, _capi.ROUTE_STREAM_TC_BF16, f"stream M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M", [16, 64, 128])
+def test_stream_weights_stable_chain_reads_x_after_producer(M):
+    """The tcgen05 weight stream under weights_stable requests its first
+    stages' weights before waiting for the preceding grid and X only after
+    it: a chain of dependent calls, each call's X the previous call's H
+    (K = N, a multiple of 64), must see every finished output."""
+    K = N = 512
+    steps = 8
+    X0, _, _ = synth.swiglu_inputs(M, K, N, "bf16", seed=23 + M)
+    Ws = [synth.swiglu_inputs(1, K, N, "bf16", seed=200 + i)[1:] for i in range(steps)]
+    dev_ws = [(g.to(dev()), u.to(dev())) for g, u in Ws]
+    assert _capi.swiglu_route_for(M, K, N, 0) == _capi.ROUTE_STREAM_TC_BF16
+    x = X0.to(dev())
+    outs = []
+    for g, u in dev_ws:
+        x = _capi.swiglu_fwd(x, g, u, weights_stable=True)
+        outs.append(x)
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+    assert _capi.swiglu_last_route() == _capi.ROUTE_STREAM_TC_BF16
+    prev = X0
+    for i, (g, u) in enumerate(Ws):
+        got = outs[i].cpu()
+        assert_bf16_close(f64(got), oracle.swiglu_fwd(prev, g, u, "bf16")["H"], f"chain M={M} {i}")
+        prev = got
+
+
+def test_mixed_route_chain_weights_stable():
+    """Decode and tcgen05-stream calls interleaved on one stream through two
+    buffers: each call reads rows another call just wrote (read after write)
+    and writes rows another call just read (write after read).  The chain
+    runs once with plain stream ordering, checked step by step against the
+    oracle, and once with weights_stable and nothing between the calls (so
+    consecutive calls overlap under programmatic dependent launch); at
+    K = N = 512 both launch forms sum in the same order, so the final
+    buffers must agree bit for bit."""
+    K = N = 512
+    A0, _, _ = synth.swiglu_inputs(16, K, N, "bf16", seed=41)
+    # (X buffer, rows), (H buffer, rows)
+    plan = [(("A", 0, 16), ("B", 0, 16)),     # stream
+            (("B", 0, 8), ("A", 0, 8)),       # decode; overwrites rows step 0 read
+            (("A", 0, 16), ("B", 0, 16)),     # stream; rows 0..7 from step 1
+            (("B", 8, 16), ("A", 8, 16)),     # decode
+            (("A", 8, 16), ("B", 0, 8)),      # decode
+            (("B", 0, 16), ("A", 0, 16)),     # stream
+            (("A", 0, 8), ("B", 8, 16))]      # decode
+    Ws = [synth.swiglu_inputs(1, K, N, "bf16", seed=300 + i)[1:] for i in range(len(plan))]
+    dev_ws = [(g.to(dev()), u.to(dev())) for g, u in Ws]
+    assert (_capi.swiglu_route_for(16, K, N, 0), _capi.swiglu_route_for(8, K, N, 0)) == \
+        (_capi.ROUTE_STREAM_TC_BF16, _capi.ROUTE_DECODE_BF16)
+
+    def run(ws, check):
+        bufs = {"A": A0.to(dev()), "B": torch.zeros_like(A0, device=dev())}
+        host = {"A": A0.clone(), "B": torch.zeros_like(A0)}
+        for i, (((xn, x0, x1), (hn, h0, h1)), (g, u)) in enumerate(zip(plan, dev_ws)):
+            _capi.swiglu_fwd(bufs[xn][x0:x1], g, u, bufs[hn][h0:h1], weights_stable=ws)
+            if check:
+                x = host[xn][x0:x1].clone()
+                h = bufs[hn][h0:h1].cpu()
+                assert_bf16_close(f64(h), oracle.swiglu_fwd(x, Ws[i][0], Ws[i][1], "bf16")["H"],
+                                  f"mixed chain step {i}")
+                host[hn][h0:h1] = h
+        assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+        return bufs["A"].cpu(), bufs["B"].cpu()
+
+    ref_a, ref_b = run(False, True)
+    for _ in range(3):
+        a, b = run(True, False)
+        assert torch.equal(a.view(torch.int16), ref_a.view(torch.int16))
+        assert torch.equal(b.view(torch.int16), ref_b.view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [65, 128])
+def test_stream_tc_split_form_odd_units(M):
+    """Wg == Wu takes the split form (two boxes, two MMAs per step); at MMA
+    M = 128 its N is rounded up to 16 and an odd unit count per CTA reads 8
+    rows past the box (accumulator columns never read).  N = 264: 33 units,
+    one per CTA."""
+    K, N = 512, 264
+    X, Wg, _ = synth.swiglu_inputs(M, K, N, "bf16", seed=M + 77)
+    Xd, Wgd = to_dev(X, Wg)
+    H = _capi.swiglu_fwd(Xd, Wgd, Wgd)
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+    assert _capi.swiglu_last_route() == _capi.ROUTE_STREAM_TC_BF16
+    assert_bf16_close(f64(H), oracle.swiglu_fwd(X, Wg, Wg, "bf16")["H"], f"split M={M}")
+    # distinct gate and up weights in the split form: a swap of the two
+    # accumulator regions would change H (h(g, u) != h(u, g))
+    X2, Wg2, Wu2 = synth.swiglu_inputs(M, K, N, "bf16", seed=M + 78)
+    both = torch.stack([Wg2, Wu2]).to(dev())
+    H2 = _capi.swiglu_fwd(X2.to(dev()), both[0], both[1])
+    assert _capi.swiglu_sync_status() == _capi.SWIGLU_OK
+    assert_bf16_close(f64(H2), oracle.swiglu_fwd(X2, Wg2, Wu2, "bf16")["H"], f"pair M={M}")

@@ -289,6 +289,7 @@ SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu
             break;
         case SWIGLU_ROUTE_GEMM_TF32X3:
             e = launch_gemm_tf32x3(X, Wg, Wu, H, m, k, n, ep, dev, stream);
+            if (e == cudaSuccess) e = launch_nonfinite_fwd_fp32(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             break;
         default:
             return SWIGLU_ERR_BAD_DTYPE;
@@ -398,9 +399,11 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg, con
     else if (route == SWIGLU_ROUTE_BWD_GEMM_BF16)
         e = launch_bwd_dx_bf16(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
                                static_cast<int>(N), dev, stream);
-    else
-        e = launch_bwd_dx_tf32x3(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
-                                 static_cast<int>(N), dev, stream);
+    else {
+        const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+        e = launch_bwd_dx_tf32x3(dG, dU, Wg, Wu, dX, m, k, n, dev, stream);
+        if (e == cudaSuccess) e = launch_nonfinite_bwd_dx_fp32(dG, dU, Wg, Wu, dX, m, k, n, dev, stream);
+    }
     st = from_cuda(e);
     if (st == SWIGLU_OK) t_last_route = route;
     return st;
@@ -428,8 +431,10 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X, void
         e = launch_bwd_dw_bf16(dG, dU, X, dWg, dWu, static_cast<int>(M), static_cast<int>(K),
                                static_cast<int>(N), dev, stream);
     } else {
-        e = launch_bwd_dw_tf32x3(dG, dU, X, dWg, dWu, static_cast<int>(M), static_cast<int>(K),
-                                 static_cast<int>(N), dev, stream);
+        const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+        e = launch_bwd_dw_tf32x3(dG, dU, X, dWg, dWu, m, k, n, dev, stream);
+        if (e == cudaSuccess)
+            e = launch_nonfinite_bwd_dw_fp32(dG, dU, X, dWg, dWu, m, k, n, dev, stream);
     }
     st = from_cuda(e);
     if (st == SWIGLU_OK) t_last_route = route;
@@ -456,9 +461,17 @@ SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg, 
         st = current_device(dev);
         if (st != SWIGLU_OK) return st;
         const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
-        st = from_cuda(dtype == SWIGLU_FP32
-                           ? launch_bwd_all_tf32x3(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream)
-                           : launch_bwd_all_bf16(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream));
+        cudaError_t e;
+        if (dtype == SWIGLU_FP32) {
+            e = launch_bwd_all_tf32x3(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream);
+            if (e == cudaSuccess)
+                e = launch_nonfinite_bwd_dx_fp32(dG, dU, Wg, Wu, dX, m, k, n, dev, stream);
+            if (e == cudaSuccess)
+                e = launch_nonfinite_bwd_dw_fp32(dG, dU, X, dWg, dWu, m, k, n, dev, stream);
+        } else {
+            e = launch_bwd_all_bf16(dG, dU, Wg, Wu, X, dX, dWg, dWu, m, k, n, dev, stream);
+        }
+        st = from_cuda(e);
         if (st == SWIGLU_OK) t_last_route = rx;
         return st;
     }

@@ -89,6 +89,18 @@ cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, 
 cudaError_t launch_bwd_all_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                   const void *X, void *dX, void *dWg, void *dWu, int M, int K,
                                   int N, const DeviceInfo &dev, cudaStream_t stream);
+// After a 3xTF32 GEMM: re-evaluate every non-finite output in plain fp32
+// arithmetic, so that infinite operands give the IEEE classes of the
+// definition (the hi/lo split alone turns them into NaN).
+cudaError_t launch_nonfinite_fwd_fp32(const void *X, const void *Wg, const void *Wu, void *H,
+                                      int M, int K, int N, const Epilogue &epi,
+                                      const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t launch_nonfinite_bwd_dx_fp32(const void *dG, const void *dU, const void *Wg,
+                                         const void *Wu, void *dX, int M, int K, int N,
+                                         const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t launch_nonfinite_bwd_dw_fp32(const void *dG, const void *dU, const void *X,
+                                         void *dWg, void *dWu, int M, int K, int N,
+                                         const DeviceInfo &dev, cudaStream_t stream);
 // Output tile width (128, 192 or 256 columns) the backward GEMMs use for a raster
 // of `row_tiles_total` 128-row tiles by `cols` columns.
 int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);

@@ -206,9 +206,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!pair) tma_prefetch_desc(tm_wu);
         tma_prefetch_desc(&tm_x);
     }
-    // Programmatic dependent launch: the next call may start prefetching its
-    // weights while this one finishes (it waits for this grid before X).
-    if (weights_stable) griddep_launch_dependents();
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (sbase - raw);
@@ -241,6 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    // Programmatic dependent launch: the next call may start prefetching its
+    // weights while this one finishes (it waits for this grid before X).
+    // Triggered only once this CTA holds its TMEM columns, so that a next
+    // call's CTA on the same SM can never take them first and leave this
+    // CTA's allocation waiting on a grid that in turn waits for this one.
+    if (weights_stable) griddep_launch_dependents();
 
     bool failed = false;
     // ----------------------------------------------------- MMA issuers
