@@ -282,9 +282,11 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X,
  * both (and dX must not overlap dWg or dWu).  The three GEMMs run as ONE
  * persistent launch whose static schedule gives every CTA its share of the
  * long dX tiles and fills with the short dW tiles, so the launch ends in one
- * balanced tail (dX alone has few tiles at small M).  fp32: the same results
- * as the two calls, bit for bit; bf16: the same per element as the two calls
- * whenever those pick 256-wide tiles (the combined launch always does).
+ * balanced tail (dX alone has few tiles at small M).  The same results as
+ * the two calls, bit for bit: every output is the same sum in the same order
+ * whatever tile width a launch uses (the single-kind calls pick 128-, 192-
+ * or 256-wide tiles by how many full waves of SMs they fill; the combined
+ * launch always uses 256).
  */
 SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg,
                                 const void *Wu, const void *X, void *dX,

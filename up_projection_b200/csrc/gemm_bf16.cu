@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long issued = 0;
             for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
                 int mt, nt;
-                tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+                tile_coords<gemm::kGroupMForward>(t, num_m_tiles, num_n_tiles, mt, nt);
                 const int m0 = mt * kBM, n0 = nt * kBN;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             int mt, nt;
-            tile_coords(t, num_m_tiles, num_n_tiles, mt, nt);
+            tile_coords<gemm::kGroupMForward>(t, num_m_tiles, num_n_tiles, mt, nt);
             const int m0 = mt * kBM, n0 = nt * kBN;
             if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
                 failed = true;

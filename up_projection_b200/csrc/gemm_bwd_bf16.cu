@@ -121,12 +121,12 @@ __device__ __forceinline__ bool next_tile(const Plan &p, int seq, TileInfo &ti) 
     int mt, nt;
     ti.kind = kind;
     if (kind == gemm::kTileDx) {
-        tile_coords(t, p.dx_num_m, p.num_n, mt, nt);
+        tile_coords<gemm::kGroupMBackward>(t, p.dx_num_m, p.num_n, mt, nt);
         ti.second = 0;
         ti.r0 = mt * kBM;
         ti.num_kb = p.dx_kb;
     } else {
-        tile_coords(t, p.dw_num_m, p.num_n, mt, nt);
+        tile_coords<gemm::kGroupMBackward>(t, p.dw_num_m, p.num_n, mt, nt);
         ti.second = mt >= p.dw_row_tiles ? 1 : 0;
         ti.r0 = (mt - ti.second * p.dw_row_tiles) * kBM;
         ti.num_kb = p.dw_kb;

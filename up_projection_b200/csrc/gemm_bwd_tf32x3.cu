@@ -29,7 +29,7 @@
 // swizzle; MN-major tiles are atoms of 32 fp32 (128 bytes) by 16 reduction
 // rows in the 128-byte swizzle with 32-byte atoms (the layout tf32 MN-major
 // operands take), one TMA box {32, 16} per atom.  Output tile
-// 128 x 256, MMA M=128 N=256 K=8.  Every wait is bounded.
+// 128 x BN, MMA M=128 N=BN K=8, BN = 256, 192 or 128.  Every wait is bounded.
 #include <string.h>
 
 #include <atomic>
@@ -52,12 +52,9 @@ using gemm::mbar_wait_drain;
 using gemm::tile_coords;
 
 constexpr int kBM = 128;                 // output rows per tile (= MMA M)
-constexpr int kBN = 256;                 // output columns per tile (= MMA N)
 constexpr int kBR = 16;                  // reduction depth per stage
 constexpr int kStages = 4;
 constexpr int kUmmaK = 8;                // k per tcgen05.mma, kind::tf32
-constexpr int kAccCols = kBN;
-constexpr int kTmemCols = 2 * kAccCols;  // chunk accumulator + running sum
 constexpr int kChunkKB = 16;             // stages per accumulation chunk (256 deep)
 constexpr int kSplitWarps = 4;
 constexpr int kEpiWarps = 4;
@@ -67,21 +64,30 @@ constexpr int kFirstEpiWarp = kFirstSplitWarp + kSplitWarps;    // 6
 
 constexpr uint32_t kAtomBytes = 32 * kBR * 4;          // MN-major atom: 32 x 16 fp32 = 2 KB
 constexpr uint32_t kABytes = kBM * kBR * 4;            // 8 KB
-constexpr uint32_t kBBytes = kBN * kBR * 4;            // 16 KB
-constexpr uint32_t kRawBytes = kABytes + kBBytes;      // 24 KB loaded per stage
-constexpr uint32_t kStageBytes = 2 * kRawBytes;        // + lo copies
 constexpr uint32_t kEpiBufBytes = 32 * 128;            // 32 rows x 32 fp32
-
-constexpr uint32_t kOffStages = 0;
-constexpr uint32_t kOffEpi = kOffStages + kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
 constexpr uint32_t kNumBars = 3 * kStages + 3;  // full, ready, empty, chunk full/empty, drain
-constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
-constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
-constexpr uint32_t kSmemBytes = kOffAbort + 8 + 1024;
 
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
-static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
+// Everything that depends on the output tile width BN (= the MMA's N; 256,
+// 192 or 128 columns, picked per call by the wave model of bwd_gemm_tile_n).
+template <int BN>
+struct Tile {
+    static constexpr int kBN = BN;
+    static constexpr int kAccCols = BN;
+    // chunk accumulator + running sum, allocated as a power of two
+    static constexpr int kTmemCols = 2 * BN > 256 ? 512 : 256;
+    static constexpr uint32_t kBBytes = BN * kBR * 4;               // 16 KB at BN = 256
+    static constexpr uint32_t kRawBytes = kABytes + kBBytes;        // loaded per stage
+    static constexpr uint32_t kStageBytes = 2 * kRawBytes;          // + lo copies
+    static constexpr uint32_t kOffStages = 0;
+    static constexpr uint32_t kOffEpi = kOffStages + kStages * kStageBytes;
+    static constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
+    static constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+    static constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
+    static constexpr uint32_t kSmemBytes = kOffAbort + 8 + 1024;
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+    static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
+    static_assert(BN % 32 == 0 && 2 * BN <= 512, "tile width");
+};
 
 // Geometry of the two tile kinds and the schedule of one launch.
 struct Plan {
@@ -106,43 +112,51 @@ struct TileInfo {
     int kind, r0, c0, num_kb, second;
 };
 
+template <int BN>
 __device__ __forceinline__ bool next_tile(const Plan &p, int seq, TileInfo &ti) {
     int kind, t;
     if (!gemm::bwd_tile_of(p.sched, blockIdx.x, gridDim.x, seq, kind, t)) return false;
     int mt, nt;
     ti.kind = kind;
     if (kind == gemm::kTileDx) {
-        tile_coords(t, p.dx_num_m, p.num_n, mt, nt);
+        tile_coords<gemm::kGroupMBackward>(t, p.dx_num_m, p.num_n, mt, nt);
         ti.second = 0;
         ti.r0 = mt * kBM;
         ti.num_kb = p.dx_kb;
     } else {
-        tile_coords(t, p.dw_num_m, p.num_n, mt, nt);
+        tile_coords<gemm::kGroupMBackward>(t, p.dw_num_m, p.num_n, mt, nt);
         ti.second = mt >= p.dw_row_tiles ? 1 : 0;
         ti.r0 = (mt - ti.second * p.dw_row_tiles) * kBM;
         ti.num_kb = p.dw_kb;
     }
-    ti.c0 = nt * kBN;
+    ti.c0 = nt * BN;
     return true;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     swiglu_gemm_bwd_tf32x3_kernel(const __grid_constant__ Maps maps, const Plan plan) {
+    using T = Tile<BN>;
+    constexpr int kBN = T::kBN;
+    constexpr int kAccCols = T::kAccCols;
+    constexpr int kTmemCols = T::kTmemCols;
+    constexpr uint32_t kRawBytes = T::kRawBytes;
+    constexpr uint32_t kStageBytes = T::kStageBytes;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
 
-    const uint32_t sst = base + kOffStages;
-    const uint32_t se = base + kOffEpi;
-    const uint32_t bar_full = base + kOffBar;
+    const uint32_t sst = base + T::kOffStages;
+    const uint32_t se = base + T::kOffEpi;
+    const uint32_t bar_full = base + T::kOffBar;
     const uint32_t bar_ready = bar_full + 8 * kStages;
     const uint32_t bar_empty = bar_ready + 8 * kStages;
     const uint32_t bar_cfull = bar_empty + 8 * kStages;
     const uint32_t bar_cempty = bar_cfull + 8;
     const uint32_t bar_drain = bar_cempty + 8;
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + kOffTmemPtr);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(gbase + T::kOffTmemPtr);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + T::kOffAbort);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -191,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+            for (int seq = 0; !failed && next_tile<BN>(plan, seq, ti); ++seq) {
                 for (int kb = 0; kb < ti.num_kb; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
@@ -245,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t chunk_phase = 0;
-            for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+            for (int seq = 0; !failed && next_tile<BN>(plan, seq, ti); ++seq) {
                 const bool dx = ti.kind == gemm::kTileDx;
                 const uint32_t idesc = dx ? idesc_dx : idesc_dw;
                 const int num_chunks = (ti.num_kb + kChunkKB - 1) / kChunkKB;
@@ -299,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sidx = threadIdx.x - 32 * kFirstSplitWarp;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
-        for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+        for (int seq = 0; !failed && next_tile<BN>(plan, seq, ti); ++seq) {
             for (int kb = 0; kb < ti.num_kb; ++kb) {
                 if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
                     failed = true;
@@ -324,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t buf = se + static_cast<uint32_t>(warp - kFirstEpiWarp) * kEpiBufBytes;
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
         uint32_t chunk_phase = 0;
-        for (int seq = 0; !failed && next_tile(plan, seq, ti); ++seq) {
+        for (int seq = 0; !failed && next_tile<BN>(plan, seq, ti); ++seq) {
             const int num_chunks = (ti.num_kb + kChunkKB - 1) / kChunkKB;
             for (int q = 0; q < num_chunks; ++q) {
                 if (!mbar_wait(bar_cfull, chunk_phase, abort_flag)) {
@@ -380,13 +394,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-std::atomic<unsigned> g_attr_set_mask{0};
+std::atomic<unsigned> g_attr_set_mask[3];
+
+template <int BN>
+cudaError_t launch_bn(const Maps &maps, const Plan &plan, int grid, const DeviceInfo &dev,
+                      cudaStream_t stream) {
+    constexpr int idx = BN == 256 ? 0 : (BN == 192 ? 1 : 2);
+    const unsigned bit = 1u << (dev.device & 31);
+    if (!(g_attr_set_mask[idx].load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bwd_tf32x3_kernel<BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(Tile<BN>::kSmemBytes));
+        if (e != cudaSuccess) return e;
+        g_attr_set_mask[idx].fetch_or(bit);
+    }
+    swiglu_gemm_bwd_tf32x3_kernel<BN><<<grid, kThreads, Tile<BN>::kSmemBytes, stream>>>(maps, plan);
+    return cudaGetLastError();
+}
 
 // Encodes the maps of the kinds requested (null pointers: kind not run) and
-// launches one persistent grid over all their tiles.
+// launches one persistent grid over all their tiles, `bn` columns wide.
 cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const void *Wu,
                         const void *X, void *dX, void *dWg, void *dWu, int M, int K, int N,
-                        bool do_dx, bool do_dw, const DeviceInfo &dev, cudaStream_t stream) {
+                        bool do_dx, bool do_dw, int bn, const DeviceInfo &dev,
+                        cudaStream_t stream) {
+    if (bn != 256 && bn != 192 && bn != 128) return cudaErrorInvalidValue;
     const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
     const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -412,7 +444,7 @@ cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const vo
     plan.M = M;
     plan.N = N;
     plan.K = K;
-    plan.num_n = (K + kBN - 1) / kBN;
+    plan.num_n = (K + bn - 1) / bn;
     plan.dx_num_m = (M + kBM - 1) / kBM;
     plan.dw_row_tiles = (N + kBM - 1) / kBM;
     plan.dw_num_m = 2 * plan.dw_row_tiles;
@@ -426,38 +458,39 @@ cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const vo
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
     plan.sched = gemm::make_bwd_sched(static_cast<int>(t_dx), static_cast<int>(t_dw), grid,
                                       plan.dx_kb, plan.dw_kb);
-    const unsigned bit = 1u << (dev.device & 31);
-    if (!(g_attr_set_mask.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bwd_tf32x3_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
-        if (e != cudaSuccess) return e;
-        g_attr_set_mask.fetch_or(bit);
-    }
-    swiglu_gemm_bwd_tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, plan);
-    return cudaGetLastError();
+    if (bn == 256) return launch_bn<256>(maps, plan, grid, dev, stream);
+    if (bn == 192) return launch_bn<192>(maps, plan, grid, dev, stream);
+    return launch_bn<128>(maps, plan, grid, dev, stream);
 }
 
 }  // namespace
 
+// A call of one kind takes the tile width of the wave model the bf16 kernel
+// uses (whole waves of tiles, narrow tiles discounted by their lower MMA
+// efficiency): at M = 2048, K = 5120 dX has 320 tiles of 256 columns (2.2
+// waves of 148, three rounds) but 432 of 192 (2.9 waves).  Every output is
+// the same sum in the same order whatever the width.
 cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                  void *dX, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
-    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, dev,
-                       stream);
+    const int bn = bwd_gemm_tile_n((M + kBM - 1) / kBM, K, dev.sm_count);
+    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, bn,
+                       dev, stream);
 }
 
 cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
                                  void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
-    return launch_plan(dG, dU, nullptr, nullptr, X, nullptr, dWg, dWu, M, K, N, false, true, dev,
-                       stream);
+    const int bn = bwd_gemm_tile_n(2 * ((N + kBM - 1) / kBM), K, dev.sm_count);
+    return launch_plan(dG, dU, nullptr, nullptr, X, nullptr, dWg, dWu, M, K, N, false, true, bn,
+                       dev, stream);
 }
 
+// All three in one launch: the dW tiles fill dX's tail, so the full width.
 cudaError_t launch_bwd_all_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                   const void *X, void *dX, void *dWg, void *dWu, int M, int K,
                                   int N, const DeviceInfo &dev, cudaStream_t stream) {
-    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, dev, stream);
+    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, 256, dev, stream);
 }
 
 cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {

@@ -7,11 +7,22 @@ namespace swiglu {
 
 namespace gemm {
 
-// Tile raster: groups of kGroupM consecutive M tiles sweep all N tiles, so
-// the ~148 tiles in flight at any time share a few X row blocks and weight
-// column blocks in L2.
-constexpr int kGroupM = 16;
+// Tile raster: groups of `group` consecutive M tiles sweep all N tiles, so
+// the ~148 tiles in flight at any time share a few row blocks of A and column
+// blocks of B in L2; a group's A rows stay in L2 while B streams past them,
+// so B is read from HBM once per group.
+//
+// The forward takes groups of 32 M tiles.  Measured on B200 at K = 4096,
+// N = 14336 (ncu DRAM bytes read per launch, time): 16 M tiles: M = 4096
+// 504 MB (1.88x the X + Wg + Wu bytes), M = 8192 1.01 GB (3.3x); 32: 272 MB
+// (1.01x) and 552 MB (1.83x), 2.5-2.8 % faster; 64: 272 MB at M = 4096 but
+// 2.42 GB at M = 8192 (the group's 67 MB of X no longer stays in L2 next to
+// the output stream), 7 % slower there.  The backward GEMMs keep groups of
+// 16 (with 32 their LLaMA-3 8B M = 8192 calls ran 2.6 % slower).
+constexpr int kGroupMForward = 32;
+constexpr int kGroupMBackward = 16;
 
+template <int kGroupM>
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mt, int &nt) {
     const int per_group = kGroupM * num_n;
     const int grp = t / per_group;
