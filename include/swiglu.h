@@ -339,11 +339,15 @@ SWIGLU_API int swiglu_selftest_wait_timeout(cudaStream_t stream);
 
 /*
  * Bench-only probe: stream-read `bytes` bytes from each of A and B (device,
- * 16-byte aligned, bytes a multiple of 16) with the same 128-bit loads the
- * decode kernel uses, and write one 32-bit word per CTA to `sink`
- * (device, at least swiglu_read_floor_sink_words() words).  Measures the
- * practical cold-read floor the decode kernel is compared with (AstrAI
- * swiglu_benchmark.md, "HBM re-measurement and kernel simplification").
+ * 16-byte aligned, bytes a multiple of 16) into shared memory by bulk copies,
+ * and write one 32-bit word per CTA to `sink` (device, at least
+ * swiglu_read_floor_sink_words() words).  Measures the practical cold-read
+ * floor the decode kernel is compared with (AstrAI swiglu_benchmark.md, "HBM
+ * re-measurement and kernel simplification").  Launched with programmatic
+ * dependent launch: it starts reading A and B while the preceding work on
+ * the stream finishes (so that consecutive probes overlap as consecutive
+ * weights-stable decode calls do), so A and B must not be written by earlier
+ * work on the stream; `sink` is written only after that work has completed.
  */
 SWIGLU_API int swiglu_read_floor(const void *A, const void *B, int64_t bytes,
                                  void *sink, cudaStream_t stream);

@@ -78,3 +78,25 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     W = (torch.randn(64, 64, device="cuda") / 8).to(torch.bfloat16)
     H = _capi.swiglu_fwd(X, W, W)
     assert _capi.swiglu_sync_status() == 0 and bool(torch.isfinite(H.float()).all())
+
+
+@pytest.mark.parametrize("nbytes", [16, 12288, 12288 * 7 + 48, 6912 * 1536 * 2])
+def test_read_floor_reads_every_byte_once(nbytes):
+    """The bench's pure-read probe: every CTA folds words 0 and 3 of each
+    16-byte vector it read into its sink word, so the XOR of all sink words is
+    the XOR of those words over both buffers -- each byte read exactly once
+    (a chunk read twice or skipped changes it)."""
+    import numpy as np
+    g = torch.Generator(device="cpu").manual_seed(nbytes)
+    A = torch.randint(0, 2 ** 31 - 1, (nbytes // 4,), generator=g, dtype=torch.int32)
+    B = torch.randint(0, 2 ** 31 - 1, (nbytes // 4,), generator=g, dtype=torch.int32)
+    sink = torch.zeros(int(_capi.lib().swiglu_read_floor_sink_words()), dtype=torch.int32,
+                       device=dev())
+    _capi.swiglu_read_floor(A.to(dev()), B.to(dev()), sink)
+    torch.cuda.synchronize()
+    got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32))
+    want = np.uint32(0)
+    for t in (A, B):
+        v = t.numpy().view(np.uint32).reshape(-1, 4)
+        want ^= np.bitwise_xor.reduce(v[:, 0]) ^ np.bitwise_xor.reduce(v[:, 3])
+    assert int(got) == int(want)

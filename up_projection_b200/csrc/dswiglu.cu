@@ -1,5 +1,5 @@
 // dswiglu.cu -- elementwise dSwiGLU backward (the "dSwiGLU" of Liger-Kernel
-// issue #1383) and the bench-only read-floor probe.
+// issue #1383).
 //
 //   dU = dH * silu(G),   dG = dH * U * silu'(G),
 //   silu(g) = g s,  silu'(g) = s (1 + g (1 - s)),  s = sigmoid(g);
@@ -135,44 +135,6 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// ------------------------------------------------------------ read floor
-
-constexpr int kProbeThreads = 512;
-constexpr int kProbeBlocksPerSm = 4;
-constexpr int kProbeUnroll = 4;
-
-__global__ void __launch_bounds__(kProbeThreads)
-    read_floor_kernel(const uint4 *A, const uint4 *B, int64_t nvec, uint32_t *sink) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kProbeThreads;
-    int64_t i = static_cast<int64_t>(blockIdx.x) * kProbeThreads + threadIdx.x;
-    uint32_t acc = 0;
-    for (; i + (kProbeUnroll - 1) * stride < nvec; i += kProbeUnroll * stride) {
-        uint4 a[kProbeUnroll], b[kProbeUnroll];
-#pragma unroll
-        for (int j = 0; j < kProbeUnroll; ++j) {
-            a[j] = ld_nc_stream_v4(A + i + j * stride);
-            b[j] = ld_nc_stream_v4(B + i + j * stride);
-        }
-#pragma unroll
-        for (int j = 0; j < kProbeUnroll; ++j)
-            acc ^= a[j].x ^ a[j].y ^ a[j].z ^ a[j].w ^ b[j].x ^ b[j].y ^ b[j].z ^ b[j].w;
-    }
-    for (; i < nvec; i += stride) {
-        const uint4 a = ld_nc_stream_v4(A + i), b = ld_nc_stream_v4(B + i);
-        acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    __shared__ uint32_t part[kProbeThreads / 32];
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t x = 0;
-        for (int w = 0; w < kProbeThreads / 32; ++w) x ^= part[w];
-        sink[blockIdx.x] = x;
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *dG, void *dU,
@@ -209,16 +171,6 @@ cudaError_t launch_dswiglu(const void *dH, const void *G, const void *U, void *d
     else
         dswiglu_kernel<false, act::kSilu><<<grid, kThreads, 0, stream>>>(
             a, b, c, og, ou, nvec, tdh, tg, tu, tdg, tdu, tail, alpha);
-    return cudaGetLastError();
-}
-
-int read_floor_grid(const DeviceInfo &dev) { return dev.sm_count * kProbeBlocksPerSm; }
-
-cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
-                              const DeviceInfo &dev, cudaStream_t stream) {
-    read_floor_kernel<<<read_floor_grid(dev), kProbeThreads, 0, stream>>>(
-        static_cast<const uint4 *>(A), static_cast<const uint4 *>(B), bytes / 16,
-        static_cast<uint32_t *>(sink));
     return cudaGetLastError();
 }
 
