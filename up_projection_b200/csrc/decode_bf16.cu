@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         int stage = 0;
         uint32_t phase = 0;
         for (int u = u_begin; u < u_end && !failed; ++u) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            float d[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < geo.slices; ++j) {
                 if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag)) {
                     failed = true;
@@ -366,9 +366,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                     // lane (grp, tig) holds physical k 8*tig + {0..3} of the
                     // chunk for the first MMA and 8*tig + {4..7} for the
-                    // second, in A and B alike.
+                    // second, in A and B alike; the two go to independent
+                    // accumulators d and d1, so that consecutive MMAs do not
+                    // wait on each other (summed once per unit)
                     mma_m16n8k16_bf16(d, wg.x, wu.x, wg.y, wu.y, x.x, x.y);
-                    mma_m16n8k16_bf16(d, wg.z, wu.z, wg.w, wu.w, x.z, x.w);
+                    mma_m16n8k16_bf16(d1, wg.z, wu.z, wg.w, wu.w, x.z, x.w);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
@@ -389,10 +391,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 break;
             }
             float *mine = red + slot * (kRedSlotBytes / 4) + (cw * 32 + lane) * 4;
-            mine[0] = d[0];
-            mine[1] = d[1];
-            mine[2] = d[2];
-            mine[3] = d[3];
+            mine[0] = d[0] + d1[0];
+            mine[1] = d[1] + d1[1];
+            mine[2] = d[2] + d1[2];
+            mine[3] = d[3] + d1[3];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_red_full + 8 * slot);
         }
