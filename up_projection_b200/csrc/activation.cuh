@@ -14,9 +14,12 @@
 // 1 - s both formed without cancellation this keeps the relative accuracy
 // for negative x, where 1 + tanh(y) would cancel.
 //
-// kAccurate = false: hardware exp approximations (bf16 outputs: errors far
-// below the bf16 rounding).  kAccurate = true: expf and IEEE division (fp32
-// outputs, a few ulp).
+// kAccurate = false: the hardware exp and reciprocal approximations (bf16
+// outputs: errors of a few fp32 ulp, far below the bf16 rounding; the IEEE
+// reciprocal's range check and branch would also keep the compiler from
+// interleaving neighbouring activations -- B200, batched decode at
+// AstrAI-1B: 11.05 -> 10.56 us per call).  kAccurate = true: expf and IEEE
+// division (fp32 outputs, a few ulp).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -33,7 +36,7 @@ constexpr float kGeluA = 0.044715f;
 template <bool kAccurate>
 __device__ __forceinline__ void sigmoid_pair(float x, float &s, float &oms) {
     const float t = kAccurate ? expf(-fabsf(x)) : __expf(-fabsf(x));
-    const float r = kAccurate ? 1.0f / (1.0f + t) : __frcp_rn(1.0f + t);
+    const float r = kAccurate ? 1.0f / (1.0f + t) : __fdividef(1.0f, 1.0f + t);
     const float tr = t * r;
     const bool pos = x >= 0.0f;
     s = pos ? r : tr;
