@@ -245,9 +245,21 @@ SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U
  *  Both products accumulate in ONE fp32 accumulator (tcgen05, TMEM); bf16:
  *  dX is rounded once to bf16 (RNE); fp32: 3xTF32 products accumulated in
  *  256-deep chunks folded with round-to-nearest adds, as swiglu_fwd's fp32,
- *  and (as there) NaN or infinite outputs re-evaluated in plain fp32.  M == 0 or K == 0: nothing enqueued.  N == 0:
- *  dX is set to +0.  dX must not overlap an input (SWIGLU_ERR_OVERLAP).
- *  Allocates no device memory.
+ *  and (as there) NaN or infinite outputs re-evaluated in plain fp32.
+ *  M == 0 or K == 0: nothing enqueued.  N == 0: dX is set to +0.  dX must
+ *  not overlap an input (SWIGLU_ERR_OVERLAP).
+ *
+ *  fp32 only: the output tiles beyond the last whole wave of SMs (all of
+ *  them when there are fewer tiles than SMs) may be split along the
+ *  reduction into parts of consecutive chunks, each folded on its own and
+ *  then added in part order -- deterministic (same inputs, same bits), but
+ *  those outputs are the same terms summed in another order than in
+ *  swiglu_bwd_gemms.  The parts' partial tiles live in a workspace of at
+ *  most (SM count) x 128 KB, allocated from the device's default memory
+ *  pool on `stream` for the call and freed on it afterwards (stream-ordered:
+ *  cudaMallocAsync / cudaFreeAsync, so the call can be captured in a CUDA
+ *  graph); SWIGLU_ERR_CUDA if that allocation fails.  bf16 allocates no
+ *  device memory.
  */
 SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
                              const void *Wu, void *dX, int64_t M, int64_t K,
@@ -286,7 +298,8 @@ SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X,
  * the two calls, bit for bit: every output is the same sum in the same order
  * whatever tile width a launch uses (the single-kind calls pick 128-, 192-
  * or 256-wide tiles by how many full waves of SMs they fill; the combined
- * launch always uses 256).
+ * launch always uses 256) -- except fp32 dX where swiglu_bwd_dx splits its
+ * tail tiles (see there): never split here.  Allocates no device memory.
  */
 SWIGLU_API int swiglu_bwd_gemms(const void *dG, const void *dU, const void *Wg,
                                 const void *Wu, const void *X, void *dX,

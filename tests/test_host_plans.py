@@ -56,6 +56,14 @@ def test_backward_schedule_is_an_exact_partition():
     _build_and_run(["tests/bwd_sched_check.cu"], 8000)
 
 
+def test_dx_split_tail_is_an_exact_partition():
+    """fp32 dX alone: the tail tiles split along the reduction are covered
+    chunk by chunk exactly once, the whole tiles round-robin exactly once, at
+    most one part per CTA after its whole tiles, never more parts than CTAs
+    (dx_split_check.cu)."""
+    _build_and_run(["tests/dx_split_check.cu"], 1000)
+
+
 def test_decode_geometry_for_every_supported_k():
     """Decode kernel: for every K it accepts, both launch forms and M <= 8,
     the shared-memory layout fits (two CTAs per SM on the small budget), the

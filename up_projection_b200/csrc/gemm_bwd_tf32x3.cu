@@ -25,6 +25,16 @@
 // which CTAs free up, so the whole backward ends in one balanced wave tail
 // instead of dX's alone (at M = 2048 its 320 tiles are 2.2 waves).
 //
+// dX alone has no dW tiles to fill its tail, so there the tiles of the last
+// partial wave (or all of them, when there are fewer tiles than SMs) are
+// split along the reduction: the r tail tiles become r x S parts of
+// consecutive 256-deep chunks, one per CTA after its round-robin tiles, each
+// folding its chunks into its own fp32 partial tile in a workspace; a second
+// kernel adds the S partials of each tile in part order (round-to-nearest
+// fp32 adds, fixed order: deterministic) and writes dX.  At M = 2048,
+// K = 5120 the 320 tiles become 296 whole tiles and 24 x 6 parts: 2.17
+// tile-times instead of 3.
+//
 // fp32 operands: K-major tiles are 16 fp32 (64 bytes) per row in the 64-byte
 // swizzle; MN-major tiles are atoms of 32 fp32 (128 bytes) by 16 reduction
 // rows in the 128-byte swizzle with 32-byte atoms (the layout tf32 MN-major
@@ -96,6 +106,11 @@ struct Plan {
     int dx_kb, dw_kb;                              // 16-deep reduction blocks per tile
     int kb_pair;                                   // dX: blocks of one pair (dG Wg, dU Wu)
     gemm::BwdSched sched;
+    // Split dX tail (dX-only launches; split.parts = 0: none): part p of
+    // tail tile split.t0 + j is run by CTA j * split.parts + p after its
+    // round-robin tiles and lands in workspace slot j * split.parts + p (a
+    // 128 x BN fp32 tile).
+    gemm::DxSplit split;
 };
 
 // Tensor maps of both kinds (only those of the kinds a launch runs are used).
@@ -106,17 +121,45 @@ struct Maps {
     CUtensorMap dw_a[2];   // dG, dU: MN-major atoms {32, 16}
     CUtensorMap dw_b;      // X: MN-major atoms {32, 16}
     CUtensorMap dw_o[2];   // dWg, dWu
+    CUtensorMap ws;        // split dX partials: [slots * 128 rows][BN] fp32
 };
 
 struct TileInfo {
     int kind, r0, c0, num_kb, second;
+    int kb0;    // first reduction block (a split part starts inside the tile)
+    int slot;   // workspace slot of a split part's partial tile, else -1
 };
+
+// The split tail (gemm_common.cuh, dx_split_shape) of a dX-only launch at
+// tile width bn over sm_count CTAs.
+inline gemm::DxSplit split_shape(int M, int K, int N, int bn, int sm_count) {
+    const long long T = static_cast<long long>((M + kBM - 1) / kBM) * ((K + bn - 1) / bn);
+    const int kb = 2 * ((N + kBR - 1) / kBR);
+    return gemm::dx_split_shape(T, (kb + kChunkKB - 1) / kChunkKB, sm_count);
+}
 
 template <int BN>
 __device__ __forceinline__ bool next_tile(const Plan &p, int seq, TileInfo &ti) {
     int kind, t;
-    if (!gemm::bwd_tile_of(p.sched, blockIdx.x, gridDim.x, seq, kind, t)) return false;
     int mt, nt;
+    ti.kb0 = 0;
+    ti.slot = -1;
+    if (!gemm::bwd_tile_of(p.sched, blockIdx.x, gridDim.x, seq, kind, t)) {
+        // after its round-robin tiles, a CTA may take one part of a split tile
+        const int slot = static_cast<int>(blockIdx.x);
+        int c_begin, c_end;
+        if (seq != p.sched.q || !gemm::dx_split_part(p.split, slot, t, c_begin, c_end))
+            return false;
+        tile_coords<gemm::kGroupMBackward>(t, p.dx_num_m, p.num_n, mt, nt);
+        ti.kind = gemm::kTileDx;
+        ti.second = 0;
+        ti.r0 = mt * kBM;
+        ti.c0 = nt * BN;
+        ti.kb0 = c_begin * kChunkKB;
+        ti.num_kb = min(p.dx_kb, c_end * kChunkKB) - ti.kb0;
+        ti.slot = slot;
+        return true;
+    }
     ti.kind = kind;
     if (kind == gemm::kTileDx) {
         tile_coords<gemm::kGroupMBackward>(t, p.dx_num_m, p.num_n, mt, nt);
@@ -179,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&maps.dx_b[1]);
             tma_prefetch_desc(&maps.dx_o);
         }
+        if (plan.split.parts > 0) tma_prefetch_desc(&maps.ws);
         if (plan.sched.T_dw > 0) {
             tma_prefetch_desc(&maps.dw_a[0]);
             tma_prefetch_desc(&maps.dw_a[1]);
@@ -215,8 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t st = sst + stage * kStageBytes;
                     mbar_arrive_expect_tx(fb, kRawBytes);
                     if (ti.kind == gemm::kTileDx) {
-                        const int pair = kb >= plan.kb_pair ? 1 : 0;
-                        const int red0 = (kb - pair * plan.kb_pair) * kBR;
+                        const int kba = ti.kb0 + kb;  // reduction block within the tile
+                        const int pair = kba >= plan.kb_pair ? 1 : 0;
+                        const int red0 = (kba - pair * plan.kb_pair) * kBR;
                         // A: [128 rows of dG or dU] x [16 of N], K-major.
                         tma_load_2d(&maps.dx_a[pair], fb, st, red0, ti.r0);
                         // B: [16 rows of Wg or Wu] x [256 of K], MN-major atoms.
@@ -354,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (failed) break;
             const bool dx = ti.kind == gemm::kTileDx;
-            const CUtensorMap *out = dx ? &maps.dx_o : &maps.dw_o[ti.second];
+            const bool part = ti.slot >= 0;  // a split part: the partial tile to its slot
+            const CUtensorMap *out = part ? &maps.ws : (dx ? &maps.dx_o : &maps.dw_o[ti.second]);
             const int rows = dx ? plan.M : plan.N;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
@@ -371,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int x = ti.c0 + c * 32;
-                    const int y = ti.r0 + quad * 32;
-                    if (x < plan.K && y < rows) {
+                    const int x = part ? c * 32 : ti.c0 + c * 32;
+                    const int y = part ? ti.slot * kBM + quad * 32 : ti.r0 + quad * 32;
+                    if (part || (x < plan.K && y < rows)) {
                         tma_store_2d(out, buf, x, y);
                         bulk_commit();
                     }
@@ -391,6 +437,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         __syncwarp();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// dX of the split tail tiles: for every element the parts' partial sums are
+// added in part order with round-to-nearest fp32 adds (a fixed order, so the
+// result does not depend on which CTA finished first), then stored if inside
+// dX.  Four consecutive columns per thread.
+__global__ void __launch_bounds__(256)
+    bwd_dx_split_combine_kernel(const float *__restrict__ ws, float *__restrict__ dX,
+                                const Plan plan, int bn) {
+    const int q4 = bn / 4;                           // float4 per partial row
+    const long long per_tile = static_cast<long long>(kBM) * q4;
+    const long long total = per_tile * plan.split.tiles;
+    const int S = plan.split.parts;
+    for (long long idx = blockIdx.x * 256ll + threadIdx.x; idx < total;
+         idx += static_cast<long long>(gridDim.x) * 256) {
+        const int j = static_cast<int>(idx / per_tile);
+        const int rem = static_cast<int>(idx - j * per_tile);
+        const int i = rem / q4, c = (rem - i * q4) * 4;
+        int mt, nt;
+        tile_coords<gemm::kGroupMBackward>(plan.split.t0 + j, plan.dx_num_m, plan.num_n, mt, nt);
+        const int row = mt * kBM + i, col = nt * bn + c;
+        if (row >= plan.M || col >= plan.K) continue;
+        const float4 *p = reinterpret_cast<const float4 *>(ws) +
+                          (static_cast<long long>(j) * S * kBM + i) * q4 + c / 4;
+        float4 acc = p[0];
+        for (int s = 1; s < S; ++s) {
+            const float4 v = p[static_cast<long long>(s) * kBM * q4];
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
+        }
+        float *o = dX + static_cast<long long>(row) * plan.K + col;
+        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (col + e < plan.K) o[e] = a[e];
     }
 }
 
@@ -414,10 +498,13 @@ cudaError_t launch_bn(const Maps &maps, const Plan &plan, int grid, const Device
 
 // Encodes the maps of the kinds requested (null pointers: kind not run) and
 // launches one persistent grid over all their tiles, `bn` columns wide.
+// split_parts > 0 (dX only; it must be the parts of split_shape at this
+// width): the tail tiles' partials go to `ws` (tiles x parts x 128 x bn
+// fp32), which the combine kernel then reduces into dX.
 cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const void *Wu,
                         const void *X, void *dX, void *dWg, void *dWu, int M, int K, int N,
-                        bool do_dx, bool do_dw, int bn, const DeviceInfo &dev,
-                        cudaStream_t stream) {
+                        bool do_dx, bool do_dw, int bn, int split_parts, void *ws,
+                        const DeviceInfo &dev, cudaStream_t stream) {
     if (bn != 256 && bn != 192 && bn != 128) return cudaErrorInvalidValue;
     const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
@@ -451,31 +538,97 @@ cudaError_t launch_plan(const void *dG, const void *dU, const void *Wg, const vo
     plan.kb_pair = (N + kBR - 1) / kBR;
     plan.dx_kb = 2 * plan.kb_pair;
     plan.dw_kb = (M + kBR - 1) / kBR;
-    const long long t_dx = do_dx ? static_cast<long long>(plan.dx_num_m) * plan.num_n : 0;
+    long long t_dx = do_dx ? static_cast<long long>(plan.dx_num_m) * plan.num_n : 0;
     const long long t_dw = do_dw ? static_cast<long long>(plan.dw_num_m) * plan.num_n : 0;
     const long long tiles = t_dx + t_dw;
     if (tiles == 0) return cudaSuccess;
-    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    if (split_parts > 0) {
+        if (do_dw || ws == nullptr) return cudaErrorInvalidValue;
+        const gemm::DxSplit sp = split_shape(M, K, N, bn, dev.sm_count);
+        if (sp.parts != split_parts) return cudaErrorInvalidValue;
+        plan.split = sp;
+        t_dx = sp.t0;  // the round-robin tiles: whole waves
+        grid = dev.sm_count;
+        if (!encode_tmap_2d(&maps.ws, ws, f32, static_cast<uint64_t>(bn),
+                            static_cast<uint64_t>(sp.tiles) * sp.parts * kBM,
+                            static_cast<uint64_t>(bn) * 4, 32, 32, sw128))
+            return cudaErrorInvalidValue;
+    }
     plan.sched = gemm::make_bwd_sched(static_cast<int>(t_dx), static_cast<int>(t_dw), grid,
                                       plan.dx_kb, plan.dw_kb);
-    if (bn == 256) return launch_bn<256>(maps, plan, grid, dev, stream);
-    if (bn == 192) return launch_bn<192>(maps, plan, grid, dev, stream);
-    return launch_bn<128>(maps, plan, grid, dev, stream);
+    cudaError_t e;
+    if (bn == 256) e = launch_bn<256>(maps, plan, grid, dev, stream);
+    else if (bn == 192) e = launch_bn<192>(maps, plan, grid, dev, stream);
+    else e = launch_bn<128>(maps, plan, grid, dev, stream);
+    if (e != cudaSuccess || split_parts == 0) return e;
+    const long long vec = static_cast<long long>(plan.split.tiles) * kBM * (bn / 4);
+    const long long blocks = (vec + 255) / 256;
+    const int cgrid = static_cast<int>(blocks < 4ll * dev.sm_count ? blocks : 4ll * dev.sm_count);
+    bwd_dx_split_combine_kernel<<<cgrid, 256, 0, stream>>>(static_cast<const float *>(ws),
+                                                         static_cast<float *>(dX), plan, bn);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
-// A call of one kind takes the tile width of the wave model the bf16 kernel
-// uses (whole waves of tiles, narrow tiles discounted by their lower MMA
-// efficiency): at M = 2048, K = 5120 dX has 320 tiles of 256 columns (2.2
-// waves of 148, three rounds) but 432 of 192 (2.9 waves).  Every output is
-// the same sum in the same order whatever the width.
+DxSplitPlan dx_split_plan(int M, int K, int N, int sm_count) {
+    // Predicted time of each (width, split): whole rounds of tiles, each
+    // tile its chunk count times one chunk's time at that width (B200, 13B
+    // shape: ~12 us per 256-deep chunk of a 128 x 256 tile; 192-wide tiles
+    // run at 0.83 of that rate per column, 128-wide taken as 0.6), and with a
+    // split one part's chunks plus the combine kernel (a launch and a pass
+    // over the partials).
+    static const int widths[3] = {256, 192, 128};
+    static const double eff[3] = {1.0, 0.83, 0.6};
+    constexpr double kChunkUs = 12.0;
+    DxSplitPlan best{256, 0, 0};
+    double best_t = -1.0;
+    const long long rows = (M + kBM - 1) / kBM;
+    if (rows <= 0 || K <= 0 || sm_count < 1) return best;
+    for (int i = 0; i < 3; ++i) {
+        const int w = widths[i];
+        const long long T = rows * ((K + w - 1) / w);
+        const gemm::DxSplit sp = split_shape(M, K, N, w, sm_count);
+        const double chunk = kChunkUs * w / 256.0 / eff[i];
+        const double tile = sp.chunks * chunk;
+        const double t_plain = static_cast<double>((T + sm_count - 1) / sm_count) * tile;
+        if (best_t < 0.0 || t_plain < best_t) {
+            best = DxSplitPlan{w, 0, 0};
+            best_t = t_plain;
+        }
+        if (sp.parts > 0) {
+            const size_t bytes = static_cast<size_t>(sp.tiles) * sp.parts * kBM * w * 4;
+            const double t_split = static_cast<double>(T / sm_count) * tile +
+                                   ((sp.chunks + sp.parts - 1) / sp.parts) * chunk + 4.0 +
+                                   static_cast<double>(bytes) / 3.0e6;
+            if (t_split < best_t) {
+                best = DxSplitPlan{w, sp.parts, bytes};
+                best_t = t_split;
+            }
+        }
+    }
+    return best;
+}
+
+// dX alone: the tile width and split of the cost model (dx_split_plan);
+// with a split, a workspace for the partial tiles is taken from the stream's
+// memory pool for the call and released after the combine kernel, both in
+// stream order.
 cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                  void *dX, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
-    const int bn = bwd_gemm_tile_n((M + kBM - 1) / kBM, K, dev.sm_count);
-    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, bn,
-                       dev, stream);
+    const DxSplitPlan sp = dx_split_plan(M, K, N, dev.sm_count);
+    if (sp.parts == 0)
+        return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false,
+                           sp.bn, 0, nullptr, dev, stream);
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, sp.workspace_bytes, stream);
+    if (e != cudaSuccess) return e;
+    e = launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, sp.bn,
+                    sp.parts, ws, dev, stream);
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : f;
 }
 
 cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
@@ -483,14 +636,15 @@ cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, 
                                  cudaStream_t stream) {
     const int bn = bwd_gemm_tile_n(2 * ((N + kBM - 1) / kBM), K, dev.sm_count);
     return launch_plan(dG, dU, nullptr, nullptr, X, nullptr, dWg, dWu, M, K, N, false, true, bn,
-                       dev, stream);
+                       0, nullptr, dev, stream);
 }
 
 // All three in one launch: the dW tiles fill dX's tail, so the full width.
 cudaError_t launch_bwd_all_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                   const void *X, void *dX, void *dWg, void *dWu, int M, int K,
                                   int N, const DeviceInfo &dev, cudaStream_t stream) {
-    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, 256, dev, stream);
+    return launch_plan(dG, dU, Wg, Wu, X, dX, dWg, dWu, M, K, N, true, true, 256, 0, nullptr, dev,
+                       stream);
 }
 
 cudaError_t gemm_bwd_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream) {

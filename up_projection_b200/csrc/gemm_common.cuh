@@ -101,5 +101,42 @@ __host__ __device__ __forceinline__ bool bwd_tile_of(const BwdSched &s, int cta,
     return true;
 }
 
+// Split tail of a dX-only launch (the fp32 backward): of T tiles over G
+// CTAs, the r = T mod G beyond the whole waves (all T when T < G) are each
+// split into `parts` runs of consecutive 256-deep chunks of their reduction,
+// parts = min(G / r, chunks) so that every part has a CTA and a chunk.  The
+// whole tiles [0, t0) go round-robin (make_bwd_sched(t0, 0, G, ..): t0 / G
+// each); afterwards CTA `slot` < tiles * parts takes part slot mod parts of
+// tail tile t0 + slot / parts.  parts = 0: no split (whole waves, or fewer
+// than two parts possible).
+struct DxSplit {
+    int t0, tiles, parts, chunks;
+};
+
+__host__ __device__ __forceinline__ DxSplit dx_split_shape(long long T, int chunks, int G) {
+    DxSplit s{0, 0, 0, chunks};
+    if (T <= 0 || G < 2 || chunks < 2) return s;
+    const long long r = T % G;
+    if (r == 0) return s;
+    long long parts = G / r;
+    if (parts > chunks) parts = chunks;
+    if (parts < 2) return s;
+    s.t0 = static_cast<int>(T - r);
+    s.tiles = static_cast<int>(r);
+    s.parts = static_cast<int>(parts);
+    return s;
+}
+
+// The tail tile t and its chunk range [c_begin, c_end) of part `slot`.
+__host__ __device__ __forceinline__ bool dx_split_part(const DxSplit &s, int slot, int &t,
+                                                       int &c_begin, int &c_end) {
+    if (s.parts == 0 || slot < 0 || slot >= s.tiles * s.parts) return false;
+    const int j = slot / s.parts, p = slot - j * s.parts;
+    t = s.t0 + j;
+    c_begin = static_cast<int>(static_cast<long long>(s.chunks) * p / s.parts);
+    c_end = static_cast<int>(static_cast<long long>(s.chunks) * (p + 1) / s.parts);
+    return true;
+}
+
 }  // namespace gemm
 }  // namespace swiglu

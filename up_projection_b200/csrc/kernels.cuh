@@ -105,6 +105,15 @@ cudaError_t launch_nonfinite_bwd_dw_fp32(const void *dG, const void *dU, const v
 // of `row_tiles_total` 128-row tiles by `cols` columns.
 int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
 
+// fp32 dX alone (gemm_bwd_tf32x3.cu): the tile width bn and the number of
+// reduction parts of the tail tiles (0: no split), with the bytes of the
+// partial tiles' workspace.
+struct DxSplitPlan {
+    int bn, parts;
+    size_t workspace_bytes;
+};
+DxSplitPlan dx_split_plan(int M, int K, int N, int sm_count);
+
 // Pure streaming read of two buffers (bench-only floor probe).
 int read_floor_grid(const DeviceInfo &dev);
 cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
