@@ -266,6 +266,35 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
                              int64_t N, int dtype, cudaStream_t stream);
 
 /*
+ * swiglu_bwd_dx_noalloc -- swiglu_bwd_dx that never allocates device memory.
+ * The pages describe no such call; it exists for callers that cannot take
+ * memory from the device while they run: a server or training loop that
+ * reserved (nearly) all device memory for its own allocator at start-up, so
+ * that the default pool swiglu_bwd_dx draws its fp32 workspace from may be
+ * empty, or code that forbids any allocation after initialisation.
+ *
+ *  Arguments, results and errors are those of swiglu_bwd_dx, and the output
+ *  is bit for bit the same.  Where fp32 dX splits its tail tiles, the parts'
+ *  partial tiles go to one fixed array in device memory of 18.5 MiB
+ *  (148 partial tiles of 128 x 256 fp32, one per CTA of a 148-SM B200, the
+ *  most any shape needs there), defined in the library: every GPU that
+ *  loads the library holds it until the process exits.  A shape whose split
+ *  would need more (a GPU with more SMs) returns SWIGLU_ERR_BAD_DIM before
+ *  anything is enqueued.  bf16 needs no scratch and runs as swiglu_bwd_dx.
+ *
+ *  All calls on one GPU share the array; each call writes every part of it
+ *  that it reads, so nothing needs clearing between calls, but two calls
+ *  whose kernels overlap on the GPU (different streams, no ordering between
+ *  them) overwrite each other's partials: order them, e.g. one stream.  The
+ *  first call on each device looks up the array's device address (set-up
+ *  with that device current); make that first call before any stream
+ *  capture.
+ */
+SWIGLU_API int swiglu_bwd_dx_noalloc(const void *dG, const void *dU, const void *Wg,
+                                     const void *Wu, void *dX, int64_t M, int64_t K,
+                                     int64_t N, int dtype, cudaStream_t stream);
+
+/*
  * swiglu_bwd_dw -- weight gradients of the projection:
  *   dWg = dG^T X,  dWu = dU^T X,  dWg[n,k] = sum_m dG[m,n] X[m,k]
  * (same passage as swiglu_bwd_dx).

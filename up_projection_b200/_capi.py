@@ -69,6 +69,7 @@ SIGNATURES = {
     "dswiglu_bwd_dtype": (_I, [_P, _P, _P, _P, _P, _I64, _I, _P]),
     "swiglu_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.POINTER(Epilogue), _P]),
     "swiglu_bwd_dx": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
+    "swiglu_bwd_dx_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_bwd_dw": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_bwd_gemms": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _P]),
     "swiglu_route_for": (_I, [_I64, _I64, _I64, _I]),

@@ -409,6 +409,37 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg, con
     return st;
 }
 
+SWIGLU_API int swiglu_bwd_dx_noalloc(const void *dG, const void *dU, const void *Wg,
+                                     const void *Wu, void *dX, int64_t M, int64_t K, int64_t N,
+                                     int dtype, cudaStream_t stream) {
+    int route = SWIGLU_ROUTE_NONE;
+    int st = check_bwd_dx(dG, dU, Wg, Wu, dX, M, K, N, dtype, &route);
+    if (st != SWIGLU_OK) return st;
+    if (route == SWIGLU_ROUTE_NONE) {
+        t_last_route = route;
+        return SWIGLU_OK;
+    }
+    DeviceInfo dev;
+    st = current_device(dev);
+    if (st != SWIGLU_OK) return st;
+    cudaError_t e;
+    if (route == SWIGLU_ROUTE_ZERO_K)
+        e = cudaMemsetAsync(dX, 0, static_cast<size_t>(M) * K * elem_size(dtype), stream);
+    else if (route == SWIGLU_ROUTE_BWD_GEMM_BF16)
+        e = launch_bwd_dx_bf16(dG, dU, Wg, Wu, dX, static_cast<int>(M), static_cast<int>(K),
+                               static_cast<int>(N), dev, stream);
+    else {
+        const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+        bool too_small = false;
+        e = launch_bwd_dx_tf32x3_static(dG, dU, Wg, Wu, dX, m, k, n, dev, stream, &too_small);
+        if (too_small) return SWIGLU_ERR_BAD_DIM;
+        if (e == cudaSuccess) e = launch_nonfinite_bwd_dx_fp32(dG, dU, Wg, Wu, dX, m, k, n, dev, stream);
+    }
+    st = from_cuda(e);
+    if (st == SWIGLU_OK) t_last_route = route;
+    return st;
+}
+
 SWIGLU_API int swiglu_bwd_dw(const void *dG, const void *dU, const void *X, void *dWg,
                              void *dWu, int64_t M, int64_t K, int64_t N, int dtype,
                              cudaStream_t stream) {

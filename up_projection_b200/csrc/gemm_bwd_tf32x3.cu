@@ -631,6 +631,50 @@ cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg,
     return e != cudaSuccess ? e : f;
 }
 
+// ---------------------------------------------------------------------------
+// dX alone without any allocation, for swiglu_bwd_dx_noalloc: the split
+// tail's partial tiles go to a fixed array in device memory instead of a
+// workspace from the memory pool.  The split never needs more than one
+// partial tile of 128 x 256 fp32 per CTA, so 148 of them (an SM each on
+// B200) cover every shape there; a plan that would need more (a GPU with
+// more SMs) is refused.  Nothing in it must start at zero: each slot a call
+// reads was written earlier in the same call.  Every GPU that loads this
+// library holds the array until the process exits, and all calls on a GPU
+// share it.
+constexpr size_t kStaticScratchBytes = 148ull * kBM * 256 * 4;  // 18.5 MiB
+static __device__ __align__(256) unsigned char g_dx_static_scratch[kStaticScratchBytes];
+
+namespace {
+// The array's device address, looked up once per device (host code only
+// knows a host-side stand-in for the symbol).
+std::atomic<void *> g_dx_static_scratch_ptr[64];
+}  // namespace
+
+cudaError_t launch_bwd_dx_tf32x3_static(const void *dG, const void *dU, const void *Wg,
+                                        const void *Wu, void *dX, int M, int K, int N,
+                                        const DeviceInfo &dev, cudaStream_t stream,
+                                        bool *scratch_too_small) {
+    *scratch_too_small = false;
+    const DxSplitPlan sp = dx_split_plan(M, K, N, dev.sm_count);
+    if (sp.parts == 0)
+        return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false,
+                           sp.bn, 0, nullptr, dev, stream);
+    if (sp.workspace_bytes > kStaticScratchBytes) {
+        *scratch_too_small = true;
+        return cudaErrorInvalidValue;
+    }
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    void *ws = g_dx_static_scratch_ptr[dev.device].load();
+    if (ws == nullptr) {
+        // set-up on this device's first call (the device is current here)
+        const cudaError_t e = cudaGetSymbolAddress(&ws, g_dx_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_dx_static_scratch_ptr[dev.device].store(ws);
+    }
+    return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, sp.bn,
+                       sp.parts, ws, dev, stream);
+}
+
 cudaError_t launch_bwd_dw_tf32x3(const void *dG, const void *dU, const void *X, void *dWg,
                                  void *dWu, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {

@@ -114,6 +114,14 @@ struct DxSplitPlan {
 };
 DxSplitPlan dx_split_plan(int M, int K, int N, int sm_count);
 
+// fp32 dX alone with the split tail's partials in a static device array
+// (no allocation); *scratch_too_small is set when the plan needs more than
+// the array holds.
+cudaError_t launch_bwd_dx_tf32x3_static(const void *dG, const void *dU, const void *Wg,
+                                        const void *Wu, void *dX, int M, int K, int N,
+                                        const DeviceInfo &dev, cudaStream_t stream,
+                                        bool *scratch_too_small);
+
 // Pure streaming read of two buffers (bench-only floor probe).
 int read_floor_grid(const DeviceInfo &dev);
 cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void *sink,
