@@ -13,8 +13,8 @@
 // kernel (gemm_bwd_bf16.cu): dX accumulates both products in one accumulator
 // over the 2N-long reduction [dG | dU] x [Wg ; Wu]; dW treats [dWg ; dWu] as
 // one [2N x K] output.  The 3xTF32 machinery is that of the fp32 forward
-// (tf32x3.cuh): the split warps rewrite each raw stage as hi in place and
-// write lo beside it; per 8-deep step three kind::tf32 MMAs (lo*hi, hi*lo,
+// (tf32x3.cuh): each raw stage serves as hi as it landed and the split
+// warps write lo beside it; per 8-deep step three kind::tf32 MMAs (lo*hi, hi*lo,
 // hi*hi) accumulate into a chunk accumulator; the epilogue warps fold every
 // 256-deep chunk into a running sum with round-to-nearest fp32 adds, then
 // store the fp32 tile by TMA.

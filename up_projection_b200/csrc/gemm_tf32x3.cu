@@ -5,7 +5,7 @@
 // Convergence Tests ...", Root Cause) shows a fused gate/up kernel whose fp32
 // matmuls ran on the TF32 tensor-core path failing fp32 parity, while forcing
 // IEEE FMA overflowed shared memory.  Here every fp32 operand is split
-//     a = hi + lo,   hi = rna_tf32(a),   lo = rna_tf32(a - hi)
+//     a = hi + lo,   hi = trunc_tf32(a),   lo = rna_tf32(a - hi)
 // and each product is formed as hi*hi + hi*lo + lo*hi (the lo*lo term, below
 // 2^-22 relative, is dropped), all accumulated in fp32 in tensor memory.
 // This is the split-precision refinement of Markidis et al. (2018, "NVIDIA
@@ -18,8 +18,9 @@
 //  * warp 0 (one thread): TMA producer -- raw fp32 X [128 x 16] and the
 //    stacked [Wg; Wu] tile [256 x 16] per 16-deep k-block, 64-byte swizzle,
 //    into a 4-stage ring;
-//  * warps 2..5: split -- each raw stage is rewritten in place as hi and a
-//    lo copy is written to a parallel buffer with the same (swizzled) layout;
+//  * warps 2..5: split -- each raw stage serves as hi as it landed (the MMA
+//    reads the top 19 bits of each element: trunc_tf32) and lo is written to
+//    a parallel buffer with the same (swizzled) layout;
 //  * warp 1 (one thread): MMA issuer -- per 8-deep step three
 //    tcgen05.mma kind::tf32 (M=128, N=256): Xhi*[Wg;Wu]hi, Xhi*[Wg;Wu]lo,
 //    Xlo*[Wg;Wu]hi into the chunk accumulator (gate columns 0..127, up
