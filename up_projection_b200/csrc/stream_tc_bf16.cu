@@ -29,8 +29,8 @@
 // The k16 steps alternate between two accumulator sets, each issued by its
 // own thread (no MMA waits on its predecessor's accumulator, and two threads
 // keep the tensor pipe fed); the epilogue sums them, forms
-// h = act(alpha g) u in fp32 and rounds once to bf16 -- spread over all 128
-// epilogue threads through shared memory when few warps hold the rows.
+// h = act(alpha g) u in fp32 and rounds once to bf16 -- spread over all 192
+// threads through shared memory when few warps hold the rows.
 // Where a CTA's stages are small enough two CTAs share an SM, so that one's
 // tail overlaps the other's stream (and, with weights_stable, the next
 // call's weight prefetch).
@@ -373,20 +373,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && cnt > 0) run_mma(0);
-    } else {
+    }
+    __syncwarp();  // warps 0 and 1 reconverge and join the epilogue
+    {
         // ------------------------------------------------------- epilogue
         // M = 128 MMA (M > 64): every quadrant's warp holds 32 rows and
         // forms h for them directly from TMEM, 16-byte stores per unit.
         // M = 64 MMA: the warps holding D rows (16 per quadrant, a single
         // warp at M <= 16) copy g and u (both accumulator sets summed) from
         // TMEM to shared memory -- the ring, idle once every MMA has
-        // completed -- and then all 128 epilogue threads form the
-        // activations and store H, two columns each, so that serial
-        // activations in few lanes do not become the kernel's tail (B200,
-        // AstrAI-1B M = 16: 11.7 -> 10.2 us; at M = 128 the round trip
-        // costs more than it saves).  Units go through in chunks that fit
-        // the ring.
-        const int et = threadIdx.x - 64;  // 0..127
+        // completed -- and then all 192 threads (the copy and MMA warps
+        // join once their roles end) form the activations and store H, two
+        // columns each, so that serial activations in few lanes do not
+        // become the kernel's tail (B200, AstrAI-1B M = 16: 11.7 -> 10.2 us
+        // with the 128 epilogue threads, M = 64: 10.96 -> 10.76 us with all
+        // 192; at M = 128 the round trip costs more than it saves).  Units
+        // go through in chunks that fit the ring.  Only warps 2..5 touch
+        // TMEM (warp w may read lanes 32 (w mod 4) .. +31).
+        const int et = threadIdx.x;  // 0..191
         const int quad = warp & 3;        // TMEM lane quadrant this warp may read
         // D row m sits in lane m (M = 128 MMA), or for M = 64 in lanes 0..15
         // of each quadrant: row 16 quad + lane.
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cnt > 0 && !ok) failed = true;
             *epi_ok = ok ? 1 : 0;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kThreads);
         if (*epi_ok) {
             tc_fence_after();
             const uint32_t R = static_cast<uint32_t>(geo.region);
@@ -411,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t uoff = pair ? (swapped ? 0u : c8) : R;
             float *E = reinterpret_cast<float *>(gbase);  // [m][unit][g 8, u 8]
             if (geo.mma_m == 128) {
-                for (int i = 0; i < cnt && quad * rows_per_quad < M; ++i) {
+                for (int i = 0; i < cnt && warp >= 2 && quad * rows_per_quad < M; ++i) {
                     const uint32_t col = tmem_base + row_off + static_cast<uint32_t>(8 * i);
                     uint32_t g0[8], u0[8], g1[8], u1[8];
                     tmem_ld_32x32b_x8(col + goff, g0);
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int i0 = 0; i0 < cnt && geo.mma_m == 64; i0 += geo.epi_units) {
                 const int uc = cnt - i0 < geo.epi_units ? cnt - i0 : geo.epi_units;
-                if (quad * rows_per_quad < M) {
+                if (warp >= 2 && quad * rows_per_quad < M) {
                     for (int ii = 0; ii < uc; ++ii) {
                         const uint32_t col =
                             tmem_base + row_off + static_cast<uint32_t>(8 * (i0 + ii));
@@ -484,11 +488,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kThreads);
                 // (m, unit, column pair) items; consecutive items are
                 // consecutive columns of one row of H
                 const int items = M * uc * 4;
-                for (int it = et; it < items; it += 128) {
+                for (int it = et; it < items; it += kThreads) {
                     const int m = it / (uc * 4);
                     const int r = it - m * uc * 4;
                     const int ii = r >> 2;
@@ -505,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint32_t *>(Uout + o) = pack_bf16x2(u.x, u.y);
                     }
                 }
-                named_bar_sync(1, 128);  // E is rewritten by the next chunk
+                named_bar_sync(1, kThreads);  // E is rewritten by the next chunk
             }
         }
     }
