@@ -56,6 +56,42 @@ def test_fp32_small(M, K, N):
                   f"fp32 M={M} K={K} N={N}")
 
 
+# M > 128 runs each MMA over a pair of SMs (256 rows: the even CTA's 128
+# rows of X with the Wg rows, the odd one's with the Wu rows): pairs whose
+# second half is partly or wholly beyond M, several pairs, ragged N and K,
+# the training forward's G and U from the pair's halves.
+@pytest.mark.parametrize("M,K,N", [(129, 64, 136), (255, 48, 264), (256, 128, 128),
+                                   (257, 100, 392), (640, 1040, 520), (1000, 256, 1032)])
+def test_fp32_pair_of_sms(M, K, N):
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=M + 3 * K)
+    H = run(X, Wg, Wu)
+    ref = oracle.swiglu_fwd(X, Wg, Wu, "f32", want_magnitudes=True)
+    assert_within(np.abs(f64(H) - ref["H"]),
+                  fp32_bound(ref["G"], ref["U"], ref["H"], ref["AG"], ref["AU"]),
+                  f"fp32 pair M={M} K={K} N={N}")
+    Xd, Wgd, Wud = to_dev(X, Wg, Wu)
+    H2, G, U = _capi.swiglu_fwd(Xd, Wgd, Wud, return_gu=True)
+    assert _capi.swiglu_sync_status() == 0
+    assert torch.equal(H2.cpu(), H)
+    for got, r in ((G, ref["G"]), (U, ref["U"])):
+        mag = ref["AG"] if got is G else ref["AU"]
+        assert np.all(np.abs(f64(got.cpu()) - r) <= 1e-5 * (np.abs(r) + mag) + 1e-30)
+
+
+def test_fp32_pair_integer_exact():
+    """Integer operands through the pair of SMs: every product and sum exact,
+    gate >= 17 (sigmoid 1 in fp32), so H = fp32(G * U) bit for bit -- each
+    row lands in the right CTA's half and each column in the right matrix."""
+    M, K, N = 520, 64, 264
+    X, Wg, Wu = synth.integer_inputs(M, K, N, seed=5, dtype="f32")
+    H = run(X, Wg, Wu)
+    G = X.double() @ Wg.double().T
+    U = X.double() @ Wu.double().T
+    assert float(G.min()) >= 17.0
+    expect = (G * U).float()
+    assert torch.equal(H.view(torch.int32), expect.view(torch.int32))
+
+
 def test_fp32_integer_exact():
     """Small integers are exact in TF32 (lo = 0); gate >= 17 makes sigmoid 1
     in fp32, so H must equal fp32(G * U) bit for bit."""

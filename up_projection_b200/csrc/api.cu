@@ -288,7 +288,11 @@ SWIGLU_API int swiglu_fwd_epilogue(const void *X, const void *Wg, const void *Wu
             e = launch_gemm_bf16(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             break;
         case SWIGLU_ROUTE_GEMM_TF32X3:
-            e = launch_gemm_tf32x3(X, Wg, Wu, H, m, k, n, ep, dev, stream);
+            // one SM per 128-row block, or (more than one block) pairs of SMs
+            // sharing each MMA
+            e = gemm_tf32x3_2sm_worth(m)
+                    ? launch_gemm_tf32x3_2sm(X, Wg, Wu, H, m, k, n, ep, dev, stream)
+                    : launch_gemm_tf32x3(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             if (e == cudaSuccess) e = launch_nonfinite_fwd_fp32(X, Wg, Wu, H, m, k, n, ep, dev, stream);
             break;
         default:
@@ -539,7 +543,7 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (st != SWIGLU_OK) return st;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0, w6 = 0, w7 = 0;
+    unsigned int w1 = 0, w2 = 0, w3 = 0, w4 = 0, w5 = 0, w6 = 0, w7 = 0, w8 = 0;
     e = gemm_bf16_status_fetch_and_clear(&w1, stream);
     if (e != cudaSuccess) return from_cuda(e);
     e = gemm_tf32x3_status_fetch_and_clear(&w2, stream);
@@ -554,7 +558,9 @@ SWIGLU_API int swiglu_sync_status(cudaStream_t stream) {
     if (e != cudaSuccess) return from_cuda(e);
     e = stream_tc_status_fetch_and_clear(&w7, stream);
     if (e != cudaSuccess) return from_cuda(e);
-    return (w1 | w2 | w3 | w4 | w5 | w6 | w7) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
+    e = gemm_tf32x3_2sm_status_fetch_and_clear(&w8, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (w1 | w2 | w3 | w4 | w5 | w6 | w7 | w8) ? SWIGLU_ERR_TIMEOUT : SWIGLU_OK;
 }
 
 SWIGLU_API int swiglu_selftest_wait_timeout(cudaStream_t stream) {

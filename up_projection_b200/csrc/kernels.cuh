@@ -131,6 +131,14 @@ cudaError_t launch_read_floor(const void *A, const void *B, int64_t bytes, void 
 // one into *host_out, reset it, and wait for the stream.
 cudaError_t gemm_bf16_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_tf32x3_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
+
+// The fp32 forward with each MMA over a pair of SMs (gemm_tf32x3_2sm.cu):
+// taken where M has more than one 128-row block.
+bool gemm_tf32x3_2sm_worth(int M);
+cudaError_t launch_gemm_tf32x3_2sm(const void *X, const void *Wg, const void *Wu, void *H, int M,
+                                   int K, int N, const Epilogue &epi, const DeviceInfo &dev,
+                                   cudaStream_t stream);
+cudaError_t gemm_tf32x3_2sm_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t decode_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t stream_tc_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
 cudaError_t gemm_bwd_status_fetch_and_clear(unsigned int *host_out, cudaStream_t stream);
