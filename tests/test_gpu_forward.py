@@ -190,7 +190,9 @@ def test_gemm_many_tiles_per_cta():
 
 
 def test_gemm_integer_exact():
-    for M, K, N in [(256, 256, 384), (130, 64, 136)]:
+    # M > 128 runs the pair form (256-row tiles over two SMs): a partly
+    # empty second half (130), one full pair (256), several pairs (520)
+    for M, K, N in [(256, 256, 384), (130, 64, 136), (520, 64, 264)]:
         X, Wg, Wu = synth.integer_inputs(M, K, N, seed=M + N)
         H = run_fwd(X, Wg, Wu, _capi.ROUTE_GEMM_BF16)
         G = X.to(torch.float64) @ Wg.to(torch.float64).T

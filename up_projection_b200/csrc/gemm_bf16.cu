@@ -23,6 +23,17 @@
 //    bf16, written to a swizzled staging buffer and stored by TMA.  G and U
 //    never reach global memory.
 //
+// Pair mode (M > 128): each MMA covers 256 rows over the two CTAs of a
+// cluster (tcgen05 cta_group::2); a CTA holds its own 128 rows of X and half
+// of the stacked weight rows -- the even CTA the tile's Wg rows, the odd one
+// its Wu rows -- so each SM loads and reads 32 KB per stage instead of 48;
+// both CTAs' copies are counted on the even CTA's barrier, whose warp 1
+// issues the pair's MMAs and commits to the barriers of both CTAs, and each
+// CTA's epilogue drains its own 128 accumulator rows.  (B200, LLaMA-3 8B
+// shapes: the same speed at M = 8192 and 4096, +2.4 % at M = 1024, +10 % at
+// M = 256: the single-SM kernel is not bound by shared-memory traffic, as
+// the fp32 one is.)
+//
 // Edge tiles: TMA zero-fills rows/columns/k beyond the tensor on load and
 // clips the store.  Every wait is bounded (ptx.cuh): a stuck pipeline sets
 // the status word and the kernel returns after releasing what it holds.
@@ -48,32 +59,107 @@ using namespace dev;
 using gemm::mbar_wait_drain;
 using gemm::tile_coords;
 
-constexpr int kBM = 128;                // rows of X per tile (= MMA M)
+constexpr int kBM = 128;                // rows of X per CTA and tile (= MMA M per SM)
 constexpr int kBN = 128;                // columns of H per tile (gate, up each)
 constexpr int kBK = 64;                 // k per stage: one 128-byte bf16 row
-constexpr int kStages = 4;
 constexpr int kUmmaK = 16;              // k per tcgen05.mma, kind::f16
 constexpr int kAccCols = 2 * kBN;       // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 2 * kAccCols; // double buffered: all 512 columns
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-
 constexpr uint32_t kABytes = kBM * kBK * 2;           // 16 KB
-constexpr uint32_t kBBytes = 2 * kBN * kBK * 2;       // 32 KB: Wg rows, Wu rows
-constexpr uint32_t kStageBytes = kABytes + kBBytes;   // 48 KB
 constexpr uint32_t kEpiBufBytes = 32 * 128;           // 32 rows x 64 bf16
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffEpi = kOffB + kStages * kBBytes;
-constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tfull, tempty, drain
-constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
-constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
-constexpr uint32_t kSmemUsed = kOffAbort + 8;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;       // slack for 1024-B alignment
+
+// Shared-memory layout of one CTA.  kPair: each MMA covers 256 rows over the
+// two CTAs of a cluster (tcgen05 cta_group::2); a CTA then holds its own 128
+// rows of X and half of the stacked weight rows -- the even CTA the tile's
+// 128 Wg rows, the odd one its 128 Wu rows -- so a stage is 32 KB, not 48.
+template <bool kPair>
+struct Layout {
+    static constexpr int kStages = kPair ? 6 : 4;
+    static constexpr uint32_t kBBytes = (kPair ? 1 : 2) * kBN * kBK * 2;  // Wg [and Wu] rows
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+    static constexpr uint32_t kOffEpi = kOffB + kStages * kBBytes;
+    static constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * kEpiBufBytes;
+    static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tfull, tempty, drain
+    static constexpr uint32_t kOffTmemPtr = kOffBar + 8 * kNumBars;
+    static constexpr uint32_t kOffAbort = kOffTmemPtr + 8;
+    static constexpr uint32_t kSmemUsed = kOffAbort + 8;
+    static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;       // slack for 1024-B alignment
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+};
 
 static_assert(kBN % 64 == 0, "epilogue works in 64-column chunks");
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// even CTA's barrier (`bar_r0`: its cluster address) -- the pair form.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_r0,
+                                                 uint32_t dst, int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_r0)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    const uint32_t z = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
+        "\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+        : "memory");
+}
+
+// Arrive once on `bar` (this CTA's barrier, or the other CTA's cluster
+// address) when every MMA issued so far by this thread for the pair is done.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
 
 __device__ __forceinline__ float gated_fast(int which, float alpha, uint32_t gbits,
                                             uint32_t ubits) {
@@ -135,6 +221,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     swiglu_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_x,
                             const __grid_constant__ CUtensorMap tm_wg,
@@ -144,6 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tm_u, int M, int N, int K,
                             int num_m_tiles, int num_n_tiles, int which_act, float alpha,
                             int store_gu, uint8_t *__restrict__ scales) {
+    using L = Layout<kPair>;
+    constexpr int kStages = L::kStages;
+    constexpr uint32_t kBBytes = L::kBBytes;
+    constexpr uint32_t kStageBytes = L::kStageBytes;
+    constexpr uint32_t kOffA = L::kOffA, kOffB = L::kOffB, kOffEpi = L::kOffEpi;
+    constexpr uint32_t kOffBar = L::kOffBar, kOffTmemPtr = L::kOffTmemPtr, kOffAbort = L::kOffAbort;
+    constexpr int kGroup = kPair ? gemm::kGroupMForward / 2 : gemm::kGroupMForward;
+    constexpr int kRowsPerTile = kPair ? 2 * kBM : kBM;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -162,8 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int num_tiles = num_m_tiles * num_n_tiles;
+    const int num_tiles = num_m_tiles * num_n_tiles;   // kPair: 256-row tiles
     const int num_kb = (K + kBK - 1) / kBK;
+    // kPair: CTA `rank` of pair `unit`; rank 0 issues the pair's MMAs
+    const uint32_t rank = kPair ? cluster_rank() : 0u;
+    const int unit = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+    const int units = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -172,14 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
-            mbar_init(bar_tempty + 8 * b, kEpiWarps);
+            mbar_init(bar_tempty + 8 * b, (kPair ? 2 : 1) * kEpiWarps);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_x);
-        tma_prefetch_desc(&tm_wg);
-        tma_prefetch_desc(&tm_wu);
+        if (!kPair || rank == 0) tma_prefetch_desc(&tm_wg);
+        if (!kPair || rank == 1) tma_prefetch_desc(&tm_wu);
         tma_prefetch_desc(&tm_h);
         if (store_gu) {
             tma_prefetch_desc(&tm_g);
@@ -187,11 +286,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(smem_u32(tmem_ptr), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair) {
+        // both CTAs' barriers initialised and TMEM allocated before any
+        // copy, arrive or MMA that reaches the other CTA
+        cluster_sync_all();
+    } else {
+        __syncthreads();
+    }
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tmem_ptr);
 
@@ -203,10 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            // kPair: every copy of both CTAs is counted on the even CTA's
+            // full barrier, whose producer expects the pair's bytes
+            const uint32_t full_r0 = kPair ? map_to_rank(bar_full, 0) : 0u;
+            const CUtensorMap *tm_w = rank == 0 ? &tm_wg : &tm_wu;
+            for (int t = unit; t < num_tiles && !failed; t += units) {
                 int mt, nt;
-                tile_coords<gemm::kGroupMForward>(t, num_m_tiles, num_n_tiles, mt, nt);
-                const int m0 = mt * kBM, n0 = nt * kBN;
+                tile_coords<kGroup>(t, num_m_tiles, num_n_tiles, mt, nt);
+                const int m0 = mt * kRowsPerTile + static_cast<int>(rank) * kBM, n0 = nt * kBN;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag)) {
                         failed = true;
@@ -215,10 +329,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t a_dst = sa + stage * kABytes;
                     const uint32_t b_dst = sb + stage * kBBytes;
-                    mbar_arrive_expect_tx(fb, kStageBytes);
-                    tma_load_2d(&tm_x, fb, a_dst, kb * kBK, m0);
-                    tma_load_2d(&tm_wg, fb, b_dst, kb * kBK, n0);
-                    tma_load_2d(&tm_wu, fb, b_dst + kBBytes / 2, kb * kBK, n0);
+                    if constexpr (kPair) {
+                        if (rank == 0) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+                        const uint32_t fb_r0 = full_r0 + 8 * stage;
+                        tma_load_2d_pair(&tm_x, fb_r0, a_dst, kb * kBK, m0);
+                        tma_load_2d_pair(tm_w, fb_r0, b_dst, kb * kBK, n0);
+                    } else {
+                        mbar_arrive_expect_tx(fb, kStageBytes);
+                        tma_load_2d(&tm_x, fb, a_dst, kb * kBK, m0);
+                        tma_load_2d(&tm_wg, fb, b_dst, kb * kBK, n0);
+                        tma_load_2d(&tm_wu, fb, b_dst + kBBytes / 2, kb * kBK, n0);
+                    }
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -226,8 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // Never leave while a load issued here may still write shared memory.
-            for (int s = 0; s < kStages; ++s) {
+            // Never leave while a load issued here may still write shared
+            // memory.  (kPair: the even CTA's full barriers count the copies
+            // of both CTAs; the odd CTA's copies are consumed by the pair's
+            // MMAs before the final cluster barrier.)
+            for (int s = 0; s < kStages && (!kPair || rank == 0); ++s) {
                 if (issued > s) {
                     const long long uses = (issued - 1 - s) / kStages + 1;
                     mbar_wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1));
@@ -235,14 +359,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             // ------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = make_idesc(1u, kBM, 2 * kBN);
+            constexpr uint32_t idesc = make_idesc(1u, kRowsPerTile, 2 * kBN);
+            // kPair: the odd CTA's barriers, as addresses in the cluster window
+            const uint32_t empty_r1 = kPair ? map_to_rank(bar_empty, 1) : 0u;
+            const uint32_t tfull_r1 = kPair ? map_to_rank(bar_tfull, 1) : 0u;
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int t = blockIdx.x; t < num_tiles && !failed; t += gridDim.x) {
+            for (int t = unit; t < num_tiles && !failed; t += units) {
                 if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag)) {
                     failed = true;
                     break;
@@ -261,24 +388,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         // +32 bytes along K inside the swizzled row = +2 in the
                         // descriptor's start-address field.
-                        mma_f16(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc,
-                                (kb > 0 || kk > 0) ? 1u : 0u);
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (kPair)
+                            mma_f16_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, accum);
+                        else
+                            mma_f16(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, accum);
                     }
-                    mma_commit(bar_empty + 8 * stage);
+                    if constexpr (kPair) {
+                        // the stage is free in both CTAs
+                        mma_commit_pair(bar_empty + 8 * stage);
+                        mma_commit_pair(empty_r1 + 8 * stage);
+                    } else {
+                        mma_commit(bar_empty + 8 * stage);
+                    }
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (failed) break;
-                mma_commit(bar_tfull + 8 * acc);
+                if constexpr (kPair) {
+                    mma_commit_pair(bar_tfull + 8 * acc);
+                    mma_commit_pair(tfull_r1 + 8 * acc);
+                } else {
+                    mma_commit(bar_tfull + 8 * acc);
+                }
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
             // Every MMA issued here must finish before TMEM is released.
-            mma_commit(bar_drain);
+            if constexpr (kPair)
+                mma_commit_pair(bar_drain);
+            else
+                mma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0);
         }
     } else {
@@ -287,12 +431,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t row_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t buf = se + static_cast<uint32_t>(warp - 2) * kEpiBufBytes;
         const uint32_t swz = static_cast<uint32_t>(lane & 7);
+        // kPair: the accumulator is released on the even CTA's barrier
+        const uint32_t tempty_r0 = kPair ? map_to_rank(bar_tempty, 0) : 0u;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        for (int t = unit; t < num_tiles; t += units) {
             int mt, nt;
-            tile_coords<gemm::kGroupMForward>(t, num_m_tiles, num_n_tiles, mt, nt);
-            const int m0 = mt * kBM, n0 = nt * kBN;
+            tile_coords<kGroup>(t, num_m_tiles, num_n_tiles, mt, nt);
+            const int m0 = mt * kRowsPerTile + static_cast<int>(rank) * kBM, n0 = nt * kBN;
             if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag)) {
                 failed = true;
                 break;
@@ -389,7 +535,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // All tcgen05.ld of this buffer have completed (waited above).
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (lane == 0) {
+                if constexpr (kPair)
+                    mbar_arrive_remote(tempty_r0 + 8 * acc);
+                else
+                    mbar_arrive(bar_tempty + 8 * acc);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -402,14 +553,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    // kPair: the pair's MMAs have completed (the issuer drained them) and
+    // both epilogues are done before either CTA frees TMEM or leaves
+    if constexpr (kPair) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
         __syncwarp();
-        tmem_dealloc(tmem_base, kTmemCols);
+        if constexpr (kPair)
+            tmem_dealloc_pair(tmem_base, kTmemCols);
+        else
+            tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
-std::atomic<unsigned> g_attr_set_mask{0};
+std::atomic<unsigned> g_attr_set_mask[2];
 
 }  // namespace
 
@@ -435,21 +592,57 @@ cudaError_t launch_gemm_bf16(const void *X, const void *Wg, const void *Wu, void
                         sw)) {
         return cudaErrorInvalidValue;
     }
+    const int num_n = (N + kBN - 1) / kBN;
+    const int store = store_gu ? 1 : 0;
+    uint8_t *sc = static_cast<uint8_t *>(epi.scales);
     const unsigned bit = 1u << (dev.device & 31);
-    if (!(g_attr_set_mask.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bf16_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
+    if (M > kBM) {
+        // pairs of SMs: tiles of 256 rows, a cluster of two CTAs per tile
+        auto kernel = swiglu_gemm_bf16_kernel<true>;
+        if (!(g_attr_set_mask[1].load() & bit)) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(Layout<true>::kSmemBytes));
+            if (e != cudaSuccess) return e;
+            g_attr_set_mask[1].fetch_or(bit);
+        }
+        const int num_m2 = (M + 2 * kBM - 1) / (2 * kBM);
+        const long long tiles = static_cast<long long>(num_m2) * num_n;
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = Layout<true>::kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(2);
+        int max_clusters = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg);
         if (e != cudaSuccess) return e;
-        g_attr_set_mask.fetch_or(bit);
+        if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+        const long long pairs = tiles < max_clusters ? tiles : max_clusters;
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+        e = cudaLaunchKernelEx(&cfg, kernel, tx, twg, twu, th, tg, tu, M, N, K, num_m2, num_n,
+                               epi.activation, epi.gate_multiplier, store, sc);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    if (!(g_attr_set_mask[0].load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_gemm_bf16_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(Layout<false>::kSmemBytes));
+        if (e != cudaSuccess) return e;
+        g_attr_set_mask[0].fetch_or(bit);
     }
     const int num_m = (M + kBM - 1) / kBM;
-    const int num_n = (N + kBN - 1) / kBN;
     const long long tiles = static_cast<long long>(num_m) * num_n;
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    swiglu_gemm_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+    swiglu_gemm_bf16_kernel<false><<<grid, kThreads, Layout<false>::kSmemBytes, stream>>>(
         tx, twg, twu, th, tg, tu, M, N, K, num_m, num_n, epi.activation, epi.gate_multiplier,
-        store_gu ? 1 : 0, static_cast<uint8_t *>(epi.scales));
+        store, sc);
     return cudaGetLastError();
 }
 
