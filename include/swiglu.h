@@ -275,9 +275,10 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
  *
  *  Arguments, results and errors are those of swiglu_bwd_dx, and the output
  *  is bit for bit the same.  Where fp32 dX splits its tail tiles, the parts'
- *  partial tiles go to one fixed array in device memory of 18.5 MiB
- *  (148 partial tiles of 128 x 256 fp32, one per CTA of a 148-SM B200, the
- *  most any shape needs there), defined in the library: every GPU that
+ *  partial tiles go to one fixed array in device memory of 18.5 MiB (the
+ *  bytes of 148 partial tiles of 128 x 256 fp32, one per SM of a 148-SM
+ *  B200 -- or of 74 tiles of 256 rows, one per pair of SMs -- the most any
+ *  shape needs there), defined in the library: every GPU that
  *  loads the library holds it until the process exits.  A shape whose split
  *  would need more (a GPU with more SMs) returns SWIGLU_ERR_BAD_DIM before
  *  anything is enqueued.  bf16 needs no scratch and runs as swiglu_bwd_dx.

@@ -105,14 +105,16 @@ cudaError_t launch_nonfinite_bwd_dw_fp32(const void *dG, const void *dU, const v
 // of `row_tiles_total` 128-row tiles by `cols` columns.
 int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
 
-// fp32 dX alone (gemm_bwd_tf32x3.cu): the tile width bn and the number of
-// reduction parts of the tail tiles (0: no split), with the bytes of the
-// partial tiles' workspace.
+// fp32 dX alone (gemm_bwd_tf32x3.cu): the tile width bn, the number of
+// reduction parts of the tail tiles (0: no split) with the bytes of the
+// partial tiles' workspace, and whether the pair form (256-row tiles over a
+// pair of SMs) runs.
 struct DxSplitPlan {
     int bn, parts;
     size_t workspace_bytes;
+    bool pair;
 };
-DxSplitPlan dx_split_plan(int M, int K, int N, int sm_count);
+DxSplitPlan dx_split_plan(int M, int K, int N, const DeviceInfo &dev);
 
 // fp32 dX alone with the split tail's partials in a static device array
 // (no allocation); *scratch_too_small is set when the plan needs more than
