@@ -50,13 +50,17 @@ def run_dw(dG, dU, X):
 
 
 # (M, K, N): single tile, ragged tails in every dimension (K not a multiple of
-# 64, N not a multiple of 64 or 128), several tiles each way.  With 148 SMs
-# the tile-width model picks 256-wide tiles for dX of (1300, 2560, 136) and
-# dW of (200, 2048, 1032), 192-wide ones for dX of (4800, 448, 72) and dW of
-# (100, 448, 2376), and 128-wide ones elsewhere, so all three are covered.
+# 64, N not a multiple of 64 or 128), several tiles each way.  dX takes the
+# pair form (256-row tiles over two SMs) where M > 128 and dW where N > 128,
+# else one SM per tile.  With 148 SMs (74 pairs) the tile-width model picks:
+# pairs 256 wide for dX of (1300, 2560, 136) and (4800, 448, 72) and dW of
+# (200, 2048, 1032) and (100, 448, 2376), pairs 128 wide for dX and dW of
+# (130, 264, 200) and (300, 520, 136); single SMs 128 wide for the small-M dX
+# and small-N dW, 192 wide for dW of (64, 9600, 104).  M = 257 and N = 1544
+# leave the odd CTA of the last pair wholly outside the matrix.
 SHAPES = [(1, 8, 8), (130, 264, 200), (300, 520, 136), (257, 1032, 72), (64, 128, 64),
           (1300, 2560, 136), (200, 2048, 1032), (9, 64, 1544), (4800, 448, 72),
-          (100, 448, 2376)]
+          (100, 448, 2376), (64, 9600, 104)]
 
 
 @pytest.mark.parametrize("M,K,N", SHAPES)
@@ -80,7 +84,7 @@ def test_bwd_dw_matches_oracle(M, K, N):
     assert_bf16_close(f64(dWu), ru, f"dWu {M}x{K}x{N}")
 
 
-@pytest.mark.parametrize("M,K,N", [(300, 264, 200), (130, 1032, 1544)])
+@pytest.mark.parametrize("M,K,N", [(300, 264, 200), (130, 1032, 1544), (1300, 2560, 136)])
 def test_bwd_integer_exact(M, K, N):
     """Ternary operands: every sum is a small integer, exact in fp32 in any
     order and, below 256 in magnitude, exact in bf16 -- so the outputs must

@@ -77,69 +77,6 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB opt-in shared memory");
 static_assert(kRawBytes % 1024 == 0, "lo copies must keep the swizzle alignment");
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-
-// Arrive on a barrier of any CTA of the cluster.  (The shared-memory data
-// this publishes is read by the tensor cores: the writer fences it to the
-// async proxy first; a cluster-scope release here measured as a memory
-// barrier stall on every stage.)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
-                 "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-
-// D (both CTAs' TMEM) (+)= A (each CTA's 128 rows) * B (each CTA's half of N).
-__device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-    const uint32_t z = 0;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
-        "\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
-        : "memory");
-}
-
-// Arrive once on `bar` -- this CTA's barrier, or the other CTA's through its
-// cluster address -- when every tcgen05.mma issued so far by this thread
-// (for the pair) has completed.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ float gated_accurate(int which, float alpha, uint32_t gbits,
                                                 uint32_t ubits) {
     return act::gated<true>(which, alpha, __uint_as_float(gbits), __uint_as_float(ubits));
@@ -318,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tf32x3::split_stage<kRawBytes, 32 * kSplitWarps>(sst + stage * kStageBytes, sidx);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(ready_r0 + 8 * stage);
+                if (lane == 0) mbar_arrive_remote(ready_r0 + 8 * stage);
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -348,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tf32x3::fold_chunk<kAccCols>(chunk_acc, run_acc, q);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(cempty_r0);
+                if (lane == 0) mbar_arrive_remote(cempty_r0);
             }
             if (failed) break;
             const int outputs = store_gu ? 3 : 1;

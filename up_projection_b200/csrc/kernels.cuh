@@ -103,7 +103,7 @@ cudaError_t launch_nonfinite_bwd_dw_fp32(const void *dG, const void *dU, const v
                                          const DeviceInfo &dev, cudaStream_t stream);
 // Output tile width (128, 192 or 256 columns) the backward GEMMs use for a raster
 // of `row_tiles_total` 128-row tiles by `cols` columns.
-int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count);
+int bwd_gemm_tile_n(int row_tiles_total, int cols, int sm_count, bool allow_192 = true);
 
 // fp32 dX alone (gemm_bwd_tf32x3.cu): the tile width bn, the number of
 // reduction parts of the tail tiles (0: no split) with the bytes of the
