@@ -22,9 +22,12 @@ SM clock seen.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and cuda synchronize, CUDA events on the launching stream, max over ranks.
-The steps are replayed from CUDA graphs holding one full rotation of the
-copies (4 steps, 16 calls) so host launch overhead does not starve the GPU
-and consecutive calls overlap under programmatic dependent launch.  Multi-GPU (torchrun): every
+The steps are replayed from CUDA graphs holding 8 full rotations of the
+copies (32 steps, 128 calls) so host launch overhead does not starve the GPU
+and consecutive calls overlap under programmatic dependent launch (a graph
+boundary costs about one call's overlap, ~4 us, which a decoding step that
+captures a whole model amortises over all of its layers; 16 calls per graph
+cost ~0.25 us per call against 64).  Multi-GPU (torchrun): every
 rank runs the same per-GPU workload on its own GPU (independent problems, no
 data-path collective): weak scaling, value = all ranks' bytes / max time.
 
@@ -58,6 +61,9 @@ PAGE_DECODE_GBS = 702.0
 DECODE_SHAPE = (1536, 6912)
 DECODE_MS = (1, 2, 4, 8)
 DECODE_COPIES = 16
+# Full rotations of the copies held by each CUDA graph the decode timings
+# replay (the headline, per-M, read-floor, comparator and e2e graphs alike).
+GRAPH_ROTATIONS = 8
 # batched decode: the tcgen05 weight-streaming route
 BATCHED_MS = (16, 32, 64)
 
@@ -223,16 +229,20 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
     Hd = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
     per_step = len(Ms)
     groups = copies // per_step   # steps per full rotation of the copies
+    g_steps = groups * GRAPH_ROTATIONS   # steps per graph
+    g_calls = copies * GRAPH_ROTATIONS   # calls per graph of the single-kind timings
 
     def step_calls(g):
+        # step g's calls, each on the next copy (no copy is used again within
+        # the copies - 1 calls that follow it)
         for i, M in enumerate(Ms):
-            c = g * per_step + i
+            c = (g * per_step + i) % copies
             up.swiglu_fwd(Xd[M], Wg_all[c], Wu_all[c], Hd[M], stream=stream, weights_stable=True)
 
-    # eager warm-up (tensor maps, function attributes), then capture: one graph
-    # per full rotation (groups steps, so consecutive calls overlap under
-    # programmatic dependent launch across the whole rotation), plus graphs of
-    # the first r steps for a remainder, so that exactly K steps are timed.
+    # eager warm-up (tensor maps, function attributes), then capture: graphs
+    # of g_steps steps (consecutive calls overlap under programmatic
+    # dependent launch across the whole graph), plus a graph of the first r
+    # steps for a remainder, so that exactly K steps are timed.
     with torch.cuda.stream(stream):
         for g in range(groups):
             step_calls(g)
@@ -246,15 +256,15 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
                 step_calls(g)
         return gr
 
-    full = capture(groups)
-    partial = {r: capture(r) for r in range(1, groups)}
+    full = capture(g_steps)
+    partial = {r: capture(r) for r in sorted({args.warmup % g_steps, args.steps % g_steps}) if r}
     torch.cuda.synchronize()
 
     def run_steps(k):
-        for _ in range(k // groups):
+        for _ in range(k // g_steps):
             full.replay()
-        if k % groups:
-            partial[k % groups].replay()
+        if k % g_steps:
+            partial[k % g_steps].replay()
 
     with torch.cuda.stream(stream):
         run_steps(args.warmup)
@@ -287,20 +297,20 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
                               weights_stable=True)
                 j["c"] += 1
             gr = torch.cuda.CUDAGraph()
-            # a graph of one full rotation of this M alone
+            # a graph of GRAPH_ROTATIONS full rotations of this M alone
             with torch.cuda.graph(gr, stream=stream):
-                for _ in range(copies):
+                for _ in range(g_calls):
                     call()
-            reps = min(500, max(1, 4 * args.steps // copies))
+            reps = max(1, min(500 * copies, 4 * args.steps) // g_calls)
             for _ in range(2):
                 gr.replay()
-            t = timed_events(gr.replay, reps, stream) / (reps * copies)
+            t = timed_events(gr.replay, reps, stream) / (reps * g_calls)
             per_m[M] = {"us": t * 1e3, "GB/s": decode_bytes(M, K, N) / (t * 1e-3) / 1e9}
             del gr
     out["per_M"] = per_m
 
     # The pure-read floor on the same rotated copies (the AstrAI page's
-    # "pure-read floor" probe): one graph of a full rotation of reads.
+    # "pure-read floor" probe): graphs of GRAPH_ROTATIONS rotations of reads.
     sink = torch.empty(int(up.lib().swiglu_read_floor_sink_words()), dtype=torch.int32,
                        device=dev)
     with torch.cuda.stream(stream):
@@ -308,12 +318,13 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
             up.swiglu_read_floor(Wg_all[c], Wu_all[c], sink, stream=stream)
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            for c in range(copies):
+            for j in range(g_calls):
+                c = j % copies
                 up.swiglu_read_floor(Wg_all[c], Wu_all[c], sink, stream=stream)
-        reps = min(500, max(1, 4 * args.steps // copies))
+        reps = max(1, min(500 * copies, 4 * args.steps) // g_calls)
         for _ in range(2):
             gr.replay()
-        t = timed_events(gr.replay, reps, stream) / (reps * copies)
+        t = timed_events(gr.replay, reps, stream) / (reps * g_calls)
         del gr
     out["floor"] = {"us": t * 1e3, "GB/s": 4.0 * N * K / (t * 1e-3) / 1e9}
 
@@ -339,7 +350,7 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
     out["latency"] = lat
 
     # Comparators for context at the largest M, timed A-B-C-C-B-A, each a
-    # graph of one rotation of the copies: A = this library's fused call,
+    # graph of GRAPH_ROTATIONS rotations of the copies: A = this library's fused call,
     # B = torch F.linear twice + silu * mul (library GEMMs, G and U through
     # HBM), C = torch F.linear on the stacked [2N, K] weights + silu * mul of
     # the two halves.
@@ -363,15 +374,16 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
                 fn(c)
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=stream):
-                for c in range(copies):
-                    fn(c)
+                for j in range(g_calls):
+                    fn(j % copies)
             graphs[name] = gr
-        reps = min(200, max(1, 2 * args.steps // copies))
+        reps = max(1, min(200 * copies, 2 * args.steps) // g_calls)
         samples = {"A": [], "B": [], "C": []}
         for name in "ABCCBA":
             for _ in range(2):
                 graphs[name].replay()
-            samples[name].append(timed_events(graphs[name].replay, reps, stream) / (reps * copies))
+            samples[name].append(timed_events(graphs[name].replay, reps, stream) /
+                                 (reps * g_calls))
     del graphs, Wcat_all
     cmp_us = {k: 1e3 * sum(v) / len(v) for k, v in samples.items()}
     out["comparators"] = {"M": M, "order": "A-B-C-C-B-A", "us": cmp_us,
@@ -419,7 +431,7 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
         if not torch.equal(Hpack_h[offs[max(Ms)]:], out["H"][max(Ms)]):
             raise RuntimeError("e2e: H read back differs from the device-timed run")
         e_ms = max_over_ranks(e_ms, world)
-        # The same steps replayed from a CUDA graph of one rotation, with the
+        # The same steps replayed from a CUDA graph of g_steps steps, with the
         # copies pipelined on a second stream (two device buffer sets): step
         # g's input copy and step g-1's read-back overlap step g-1's / g's
         # calls.  Still, every step: one host->device copy of its X, its four
@@ -434,9 +446,9 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
         def e2e_rotation():
             # software pipeline: the copy stream runs step g+1's input copy
             # and step g-1's read-back while step g's calls run
-            ev_in = [torch.cuda.Event() for _ in range(groups)]
-            ev_c = [torch.cuda.Event() for _ in range(groups)]
-            ev_out = [torch.cuda.Event() for _ in range(groups)]
+            ev_in = [torch.cuda.Event() for _ in range(g_steps)]
+            ev_c = [torch.cuda.Event() for _ in range(g_steps)]
+            ev_out = [torch.cuda.Event() for _ in range(g_steps)]
             cs.wait_stream(stream)
 
             def copy_in(g):
@@ -446,15 +458,15 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
                     Xd2[g % 2].copy_(Xpack_h, non_blocking=True)
                     ev_in[g].record(cs)
             copy_in(0)
-            for g in range(groups):
+            for g in range(g_steps):
                 b = g % 2
-                if g + 1 < groups:
+                if g + 1 < g_steps:
                     copy_in(g + 1)
                 stream.wait_event(ev_in[g])
                 if g >= 2:
                     stream.wait_event(ev_out[g - 2])  # buffer b's H has been read back
                 for i, M in enumerate(Ms):
-                    c = g * per_step + i
+                    c = (g * per_step + i) % copies
                     up.swiglu_fwd(Xv2[b][M], Wg_all[c], Wu_all[c], Hv2[b][M], stream=stream,
                                   weights_stable=True)
                 ev_c[g].record(stream)
@@ -469,7 +481,7 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
             eg = torch.cuda.CUDAGraph()
             with torch.cuda.graph(eg, stream=stream):
                 e2e_rotation()
-            g_reps = max(1, e_steps // groups)
+            g_reps = max(1, e_steps // g_steps)
             for _ in range(2):
                 eg.replay()
             torch.cuda.synchronize()
@@ -477,12 +489,12 @@ def run_decode(args, world, K, N, Ms, copies, stream, with_e2e):
             eg_ms = timed_events(eg.replay, g_reps, stream)
         barrier(world)
         torch.cuda.synchronize()
-        last = (groups - 1) % 2
+        last = (g_steps - 1) % 2
         if not torch.equal(Hh2[last][offs[max(Ms)]:], out["H"][max(Ms)]):
             raise RuntimeError("e2e: pipelined read-back differs from the device-timed run")
         eg_ms = max_over_ranks(eg_ms, world)
         del eg
-        out["e2e"] = {"ms": eg_ms, "steps": g_reps * groups, "h2d": h2d, "d2h": d2h,
+        out["e2e"] = {"ms": eg_ms, "steps": g_reps * g_steps, "h2d": h2d, "d2h": d2h,
                       "eager_ms": e_ms, "eager_steps": e_steps}
     del full, partial
     del Wg_all, Wu_all
@@ -865,7 +877,9 @@ def main(argv=None):
               "l2": f"inputs larger than L2 ({DECODE_COPIES} rotated copies, "
                     f"{DECODE_COPIES * 4 * N * K / 1e6:.0f} MB)",
               "launch": "SWIGLU_FLAG_WEIGHTS_STABLE (programmatic dependent launch: weights "
-                        "are model parameters no earlier work writes)"}
+                        "are model parameters no earlier work writes)",
+              "graph": f"CUDA graphs of {GRAPH_ROTATIONS} rotations "
+                       f"({GRAPH_ROTATIONS * DECODE_COPIES} calls), replayed"}
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -907,8 +921,8 @@ def main(argv=None):
                 "unit": "GB/s", "h2d_bytes_per_step": dec["e2e"]["h2d"],
                 "d2h_bytes_per_step": dec["e2e"]["d2h"],
                 "launch": "public API calls and the per-step pinned copies (on a second stream, "
-                          "double-buffered, overlapping the calls) captured in a CUDA graph of "
-                          "one rotation, replayed",
+                          "double-buffered, overlapping the calls) captured in CUDA graphs of "
+                          f"{GRAPH_ROTATIONS} rotations, replayed",
                 "eager_value": round(dec["step_bytes"] * dec["e2e"]["eager_steps"] * world
                                      / (dec["e2e"]["eager_ms"] * 1e-3) / 1e9, 1)},
         "gpu_launches": dec["launches"],
