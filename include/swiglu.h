@@ -255,10 +255,14 @@ SWIGLU_API int dswiglu_bwd_epilogue(const void *dH, const void *G, const void *U
  *  then added in part order -- deterministic (same inputs, same bits), but
  *  those outputs are the same terms summed in another order than in
  *  swiglu_bwd_gemms.  The parts' partial tiles live in a workspace of at
- *  most (SM count) x 128 KB, allocated from the device's default memory
- *  pool on `stream` for the call and freed on it afterwards (stream-ordered:
- *  cudaMallocAsync / cudaFreeAsync, so the call can be captured in a CUDA
- *  graph); SWIGLU_ERR_CUDA if that allocation fails.  bf16 allocates no
+ *  most (SM count) x 128 KB, allocated on `stream` for the call and freed on
+ *  it afterwards (stream-ordered: cudaMallocFromPoolAsync / cudaFreeAsync,
+ *  so the call can be captured in a CUDA graph) from a memory pool the
+ *  library creates for the device on its first such call and keeps until
+ *  the process exits; the pool keeps the memory it has mapped (the most
+ *  that calls in flight at once have used: 18.5 MiB for one stream on a
+ *  148-SM B200) instead of returning it at each synchronisation.
+ *  SWIGLU_ERR_CUDA if the pool or the allocation fails.  bf16 allocates no
  *  device memory.
  */
 SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
@@ -270,8 +274,8 @@ SWIGLU_API int swiglu_bwd_dx(const void *dG, const void *dU, const void *Wg,
  * The pages describe no such call; it exists for callers that cannot take
  * memory from the device while they run: a server or training loop that
  * reserved (nearly) all device memory for its own allocator at start-up, so
- * that the default pool swiglu_bwd_dx draws its fp32 workspace from may be
- * empty, or code that forbids any allocation after initialisation.
+ * that the pool swiglu_bwd_dx draws its fp32 workspace from may find none
+ * free, or code that forbids any allocation after initialisation.
  *
  *  Arguments, results and errors are those of swiglu_bwd_dx, and the output
  *  is bit for bit the same.  Where fp32 dX splits its tail tiles, the parts'

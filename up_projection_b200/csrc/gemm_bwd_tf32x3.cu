@@ -54,6 +54,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "gemm_common.cuh"
 #include "kernels.cuh"
@@ -772,10 +773,42 @@ DxSplitPlan dx_split_plan(int M, int K, int N, const DeviceInfo &dev) {
     return best;
 }
 
+namespace {
+std::mutex g_ws_pool_mu;
+cudaMemPool_t g_ws_pool[64];
+
+// The memory pool the split workspaces come from: one per device, created by
+// the library, that keeps the memory it has mapped between calls.  (The
+// device's default pool returns its memory at every synchronisation, and a
+// call after one then maps its workspace again: up to a few hundred us.)
+cudaError_t workspace_pool(int device, cudaMemPool_t *out) {
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_ws_pool_mu);
+    if (g_ws_pool[device] == nullptr) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            (void)cudaMemPoolDestroy(pool);
+            return e;
+        }
+        g_ws_pool[device] = pool;
+    }
+    *out = g_ws_pool[device];
+    return cudaSuccess;
+}
+}  // namespace
+
 // dX alone: the tile width and split of the cost model (dx_split_plan);
-// with a split, a workspace for the partial tiles is taken from the stream's
-// memory pool for the call and released after the combine kernel, both in
-// stream order.
+// with a split, a workspace for the partial tiles is taken from the
+// library's pool for the device on `stream` and released after the combine
+// kernel, both in stream order.
 cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg, const void *Wu,
                                  void *dX, int M, int K, int N, const DeviceInfo &dev,
                                  cudaStream_t stream) {
@@ -783,8 +816,11 @@ cudaError_t launch_bwd_dx_tf32x3(const void *dG, const void *dU, const void *Wg,
     if (sp.parts == 0)
         return launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false,
                            sp.bn, sp.pair, 0, nullptr, dev, stream);
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = workspace_pool(dev.device, &pool);
+    if (e != cudaSuccess) return e;
     void *ws = nullptr;
-    cudaError_t e = cudaMallocAsync(&ws, sp.workspace_bytes, stream);
+    e = cudaMallocFromPoolAsync(&ws, sp.workspace_bytes, pool, stream);
     if (e != cudaSuccess) return e;
     e = launch_plan(dG, dU, Wg, Wu, nullptr, dX, nullptr, nullptr, M, K, N, true, false, sp.bn,
                     sp.pair, sp.parts, ws, dev, stream);
