@@ -171,6 +171,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tm_wg);
         tma_prefetch_desc(&tm_wu);
+        // X is read only after the dependency wait below; the first CTA to
+        // start brings it into L2 now (each call's X may have been evicted
+        // by the weights streamed since its last use).
+        if (weights_stable && blockIdx.x == 0)
+            bulk_prefetch_l2(X, static_cast<uint32_t>(M * K * 2));
     }
     // Under programmatic dependent launch the next call may be scheduled as
     // soon as every CTA of this one is running: it only prefetches weights

@@ -74,6 +74,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
 
 // -------------------------------------------------------------------- TMA
 
+// Hint: bring global [p, p + bytes) into L2 (p 16-byte aligned, bytes a
+// multiple of 16).  Not a read of the data: L2 is the device's point of
+// coherence, so a later read after a dependency wait still sees any write
+// made meanwhile.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map))
                  : "memory");

@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  int pair, int swapped,
                                  __nv_bfloat16 *__restrict__ H, int M, int N, int weights_stable,
                                  int which_act, float alpha, __nv_bfloat16 *__restrict__ Gout,
-                                 __nv_bfloat16 *__restrict__ Uout, const StreamGeo geo) {
+                                 __nv_bfloat16 *__restrict__ Uout, const StreamGeo geo,
+                                 const void *__restrict__ X, uint32_t x_bytes) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int units = N / 8;
     const int u_begin = static_cast<int>((static_cast<long long>(units) * blockIdx.x) / gridDim.x);
@@ -205,6 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(tm_wg);
         if (!pair) tma_prefetch_desc(tm_wu);
         tma_prefetch_desc(&tm_x);
+        // X is read only after the dependency wait; the first CTA to start
+        // brings it into L2 now (it may have been evicted by the weights
+        // streamed since its last use).
+        if (weights_stable && blockIdx.x == 0) bulk_prefetch_l2(X, x_bytes);
     }
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -604,8 +609,8 @@ cudaError_t launch_stream_tc_bf16(const void *X, const void *Wg, const void *Wu,
     const int ws = weights_stable ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, swiglu_stream_tc_bf16_kernel, tx, tg_lo, tu_lo, tg_hi,
                                        tu_hi, plan.q, pair, pair ? swapped : 0, hp, M, N, ws,
-                                       epi.activation,
-                                       epi.gate_multiplier, gp, up, geo);
+                                       epi.activation, epi.gate_multiplier, gp, up, geo, X,
+                                       static_cast<uint32_t>(static_cast<size_t>(M) * K * 2));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
