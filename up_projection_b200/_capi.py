@@ -8,6 +8,7 @@ call raises -- there is no fallback of any kind.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 
@@ -94,6 +95,8 @@ class SwigluError(RuntimeError):
 def lib() -> ctypes.CDLL:
     """The loaded library (raises if it is not built)."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
@@ -159,24 +162,31 @@ def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
     H = act(gate_multiplier * G) * U (SWIGLU_ACT_SILU or
     SWIGLU_ACT_GELU_TANH).  return_gu=True also stores G = X Wg^T and
     U = X Wu^T (training forward) and returns (H, G, U)."""
-    for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
-        _dev(t, n)
-    if not (X.dtype == Wg.dtype == Wu.dtype):
+    # (the checks are ordered for the per-call cost of the decode path: one
+    # pass of cheap attribute reads, the detailed messages only on failure)
+    if not (X.is_cuda and Wg.is_cuda and Wu.is_cuda and X.is_contiguous()
+            and Wg.is_contiguous() and Wu.is_contiguous()):
+        for t, n in ((X, "X"), (Wg, "Wg"), (Wu, "Wu")):
+            _dev(t, n)
+    dt = X.dtype
+    if Wg.dtype != dt or Wu.dtype != dt:
         raise TypeError("X, Wg and Wu must share a dtype")
-    K = X.shape[-1]
-    N = Wg.shape[0]
-    if Wg.shape != (N, K) or Wu.shape != (N, K):
+    code = _DT.get(dt)
+    if code is None:
+        _dtype_code(X)
+    xs = X.shape
+    K = xs[-1]
+    ws = Wg.shape
+    N = ws[0]
+    if len(ws) != 2 or ws[1] != K or Wu.shape != ws:
         raise ValueError(f"weights must be [N, K] = [{N}, {K}]")
-    lead = X.shape[:-1]
-    M = 1
-    for d in lead:
-        M *= d
+    M = X.numel() // K if K else math.prod(xs[:-1])
     if H is None:
-        H = torch.empty((*lead, N), dtype=X.dtype, device=X.device)
-    else:
+        H = torch.empty((*xs[:-1], N), dtype=dt, device=X.device)
+    elif not (H.is_cuda and H.is_contiguous()):
         _dev(H, "H")
-        if H.dtype != X.dtype or H.numel() != M * N:
-            raise ValueError("H has the wrong dtype or size")
+    elif H.dtype != dt or H.numel() != M * N:
+        raise ValueError("H has the wrong dtype or size")
     flags = SWIGLU_FLAG_WEIGHTS_STABLE if weights_stable else 0
     G = U = None
     if return_gu:
@@ -184,13 +194,13 @@ def swiglu_fwd(X: torch.Tensor, Wg: torch.Tensor, Wu: torch.Tensor,
         U = torch.empty_like(H)
     if activation == SWIGLU_ACT_SILU and gate_multiplier == 1.0 and not return_gu:
         st = lib().swiglu_fwd_ex(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
-                                 M, K, N, _dtype_code(X), flags, _stream(stream))
+                                 M, K, N, code, flags, _stream(stream))
     else:
         epi = Epilogue(int(activation), float(gate_multiplier),
                        G.data_ptr() if G is not None else None,
                        U.data_ptr() if U is not None else None)
         st = lib().swiglu_fwd_epilogue(X.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), H.data_ptr(),
-                                       M, K, N, _dtype_code(X), ctypes.byref(epi), flags,
+                                       M, K, N, code, ctypes.byref(epi), flags,
                                        _stream(stream))
     _check("swiglu_fwd", st)
     return (H, G, U) if return_gu else H
