@@ -253,7 +253,7 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
 }
 
 // TMA load into this CTA's shared memory whose completion is counted on the
-// even CTA's barrier (`bar_r0`: its cluster address).  No multicast.
+// even CTA's barrier (`bar_r0`: its cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_r0,
                                                  uint32_t dst, int32_t x, int32_t y) {
     asm volatile(
