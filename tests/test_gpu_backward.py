@@ -290,6 +290,33 @@ def test_bwd_fp32_split_tail(M, K, N, rows):
     assert np.linalg.norm(f64(dX)[r] - ref) <= 1e-5 * np.linalg.norm(ref)
 
 
+def test_bwd_fp32_split_tail_in_cuda_graph():
+    """fp32 dX alone with its split tail -- whose workspace is allocated and
+    freed in stream order inside the call -- captured in a CUDA graph: two
+    replays give the eager call's bits."""
+    M, K, N = 1280, 4096, 1024
+    X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=M + 7)
+    dG = synth.normal((M, N), N + 42, 1.0, "f32")
+    dU = synth.normal((M, N), N + 43, 1.0, "f32")
+    d = [t.to(dev()) for t in (dG, dU, Wg, Wu)]
+    ref = _run_f32(_capi.swiglu_bwd_dx, *d)
+    s = torch.cuda.Stream()
+    out = torch.empty_like(ref)
+    with torch.cuda.stream(s):
+        _capi.swiglu_bwd_dx(*d, dX=out, stream=s)   # warm-up outside the capture
+    torch.cuda.synchronize()
+    out.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        _capi.swiglu_bwd_dx(*d, dX=out, stream=s)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert _capi.swiglu_sync_status() == 0
+        assert torch.equal(out, ref)
+    del g
+
+
 def test_bwd_fp32_split_tail_integer_exact():
     """Integer operands with exact fp32 sums: every part's partial sum and
     their total are exact, so dX alone with a split tail equals the oracle
