@@ -317,6 +317,30 @@ def test_bwd_fp32_split_tail_in_cuda_graph():
     del g
 
 
+def test_bwd_fp32_split_tail_two_streams():
+    """Two fp32 dX calls with split tails on two streams at once: each takes
+    its own workspace from the pool in its stream's order, so both give the
+    bits of the same calls made one after the other."""
+    M, K, N = 1280, 4096, 1024
+    ins = []
+    for s in (0, 1):
+        X, Wg, Wu = synth.swiglu_inputs(M, K, N, "f32", seed=M + 20 + s)
+        dG = synth.normal((M, N), N + 50 + s, 1.0, "f32")
+        dU = synth.normal((M, N), N + 60 + s, 1.0, "f32")
+        ins.append([t.to(dev()) for t in (dG, dU, Wg, Wu)])
+    refs = [_run_f32(_capi.swiglu_bwd_dx, *d) for d in ins]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(r) for r in refs]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for d, o, s in zip(ins, outs, streams):
+            _capi.swiglu_bwd_dx(*d, dX=o, stream=s)
+    torch.cuda.synchronize()
+    assert _capi.swiglu_sync_status() == 0
+    for o, r in zip(outs, refs):
+        assert torch.equal(o, r)
+
+
 def test_bwd_fp32_split_tail_integer_exact():
     """Integer operands with exact fp32 sums: every part's partial sum and
     their total are exact, so dX alone with a split tail equals the oracle
