@@ -28,14 +28,15 @@ import torch
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode", "prefill", "dswiglu", "fp32", "floor", "bwd_dx",
-                                       "bwd_dw", "fp8"])
+                                       "bwd_dw", "bwd_all", "fp8"])
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--K", type=int, default=1536)
     ap.add_argument("--N", type=int, default=6912)
     ap.add_argument("--n", type=int, default=8192 * 14336)
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--launches", type=int, default=3)
-    ap.add_argument("--fp32", action="store_true", help="bwd_dx / bwd_dw: fp32 (3xTF32) operands")
+    ap.add_argument("--fp32", action="store_true",
+                    help="bwd_dx / bwd_dw / bwd_all: fp32 (3xTF32) operands")
     ap.add_argument("--weights-stable", action="store_true",
                     help="decode: SWIGLU_FLAG_WEIGHTS_STABLE (programmatic dependent launch)")
     a = ap.parse_args(argv)
@@ -74,11 +75,18 @@ def main(argv=None):
         Wu = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
         for _ in range(L):
             up.swiglu_fwd_fp8(X, Wg, Wu)
-    elif a.case in ("bwd_dx", "bwd_dw"):
+    elif a.case in ("bwd_dx", "bwd_dw", "bwd_all"):
         bf = torch.float32 if a.fp32 else torch.bfloat16
         dG = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
         dU = torch.randn((a.M, a.N), generator=g, device=dev).to(bf)
-        if a.case == "bwd_dx":
+        if a.case == "bwd_all":
+            # dX, dWg and dWu in one launch (swiglu_bwd_gemms)
+            X = torch.randn((a.M, a.K), generator=g, device=dev).to(bf)
+            Wg = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+            Wu = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
+            for _ in range(L):
+                up.swiglu_bwd_gemms(dG, dU, Wg, Wu, X)
+        elif a.case == "bwd_dx":
             Wg = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
             Wu = (torch.randn((a.N, a.K), generator=g, device=dev) / a.K ** 0.5).to(bf)
             dX = torch.empty((a.M, a.K), dtype=bf, device=dev)
