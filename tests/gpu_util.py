@@ -14,6 +14,16 @@ FP32_FWD_TOL = 1e-5
 FP32_BWD_TOL = 1e-6
 
 
+def fp32_bound(G, U, H, AG, AU):
+    """Per-element bound of the fp32-input mode: 1e-5 of the size of the terms
+    before cancellation, propagated through h = silu(g) u (AG, AU: the sums of
+    |x w| behind G and U)."""
+    s = 1.0 / (1.0 + np.exp(-np.clip(G, -700, 700)))
+    silu = G * s
+    dsilu = s * (1.0 + G * (1.0 - s))
+    return FP32_FWD_TOL * (np.abs(H) + np.abs(silu) * AU + np.abs(U) * np.abs(dsilu) * AG) + 1e-30
+
+
 def dev():
     return torch.device("cuda:0")
 

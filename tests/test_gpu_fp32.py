@@ -12,18 +12,11 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import FP32_FWD_TOL, assert_guards_intact, assert_within, f64, guarded_empty, \
-    sample_indices, to_dev
+from gpu_util import FP32_FWD_TOL, assert_guards_intact, assert_within, f64, fp32_bound, \
+    guarded_empty, sample_indices, to_dev
 from up_projection_b200 import _capi, synth
 
 pytestmark = pytest.mark.gpu
-
-
-def fp32_bound(G, U, H, AG, AU):
-    s = 1.0 / (1.0 + np.exp(-np.clip(G, -700, 700)))
-    silu = G * s
-    dsilu = s * (1.0 + G * (1.0 - s))
-    return FP32_FWD_TOL * (np.abs(H) + np.abs(silu) * AU + np.abs(U) * np.abs(dsilu) * AG) + 1e-30
 
 
 def run(X, Wg, Wu):
